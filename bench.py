@@ -1,0 +1,482 @@
+#!/usr/bin/env python
+"""Benchmark of the routed-MoE FFN decode path on B200.
+
+Default workload: the 48-layer decode stack (512 Q2 experts per layer, hidden
+2048, intermediate 768, top-10, one token per step, residual RMSNorm), one CUDA
+graph replay per token. Prints one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode48|verify48]
+
+N > 1 runs N independent replicas (one process per GPU under torchrun; the
+path has no exchange step), timed on the device, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE decode tokens/s over 48 layers; HBM GB/s on weight bytes vs peak"
+SEED = 0
+WORKLOADS = {"decode48": 2, "verify48": 3, "layer": 1}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="decode48", choices=sorted(WORKLOADS))
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def workload_desc(cfg, T):
+    return {"workload": f"{cfg.L}-layer routed-MoE decode stack: {cfg.E} experts/layer, hidden {cfg.H}, "
+                        f"intermediate {cfg.I}, top-{cfg.k}, Q{cfg.fmt} blocks, {T} token(s)/step, residual RMSNorm",
+            "layers": cfg.L, "experts_per_layer": cfg.E, "hidden": cfg.H, "intermediate": cfg.I, "top_k": cfg.k,
+            "format": f"Q{cfg.fmt}", "tokens_per_step": T, "seed": SEED,
+            "l2": "no flush: each step streams ~0.85-3.5 GB of distinct experts (> 126 MB L2); "
+                  "a fresh token is drawn for every step"}
+
+
+# ------------------------------------------------------------------ clocks --
+class Clocks:
+    Q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_uuid):
+        self.path = tempfile.mktemp(suffix=".csv")
+        self.f = open(self.path, "w")
+        args = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if dev_uuid:
+            args[1:1] = ["-i", dev_uuid]
+        try:
+            self.p = subprocess.Popen(args, stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.p.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------- dist helpers --
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------ traffic file --
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in ("ffn_decode.cu", "common.cuh", "layout.cuh"):
+        with open(os.path.join(ROOT, "quantised_expert_decode_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(workload):
+    """dram bytes per FFN launch from the committed ncu summary, if still current."""
+    path = os.path.join(ROOT, "profiles", f"ffn_decode_{workload}_ncu.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if line.startswith("- ") and ":" in line:
+                k, v = line[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# --------------------------------------------------------- oracle timing --
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_token_time(cfg, x0, n_layers):
+    """Seconds the float64 oracle takes for one step over n_layers (routing,
+    dequantisation, expert FFNs, combine, residual RMSNorm). Weight bytes are
+    drawn from the generator before each timed layer and are not counted."""
+    import numpy as np
+    from oracle import moe
+    from synth import gen
+    x = x0.astype(np.float64)
+    spent = 0.0
+    bits = cfg.format.bits
+    for l in range(n_layers):
+        Wr, b = gen.router(SEED, cfg, l), gen.bias(SEED, cfg, l)
+        t0 = time.perf_counter()
+        idx, g, _ = moe.route(x, Wr, b, cfg.k)
+        spent += time.perf_counter() - t0
+        raw = {int(e): gen.expert(SEED, cfg, l, int(e)) for e in set(idx.ravel().tolist())}
+        t0 = time.perf_counter()
+
+        def get(e):
+            r = raw[e]
+            return tuple(moe.dequantize(r[n + "_codes"], r[n + "_scales"], bits) for n in ("gate", "up", "down"))
+        y = moe.moe_layer(x, idx, g, get)
+        x = moe.rmsnorm_residual(x, y, cfg.eps)
+        spent += time.perf_counter() - t0
+    return spent
+
+
+def cpu_baseline(cfg, T):
+    from synth import gen
+    n = cfg.L if T == 1 else 4
+    x0 = gen.tokens(SEED, cfg, 0)
+    s = oracle_token_time(cfg, x0, n)
+    tok_s = T / (s * cfg.L / n)
+    return {"value": tok_s, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{T} token(s) through {n} of {cfg.L} layers (float64 NumPy, weight generation "
+                      f"excluded), scaled to {cfg.L} layers; {s:.1f} s of CPU work"}
+
+
+# -------------------------------------------------------------- reference --
+def run_reference(args, cfg, T):
+    """The oracle timed as the reference arm: a step is one expert FFN of one
+    token slot (1/k of a layer; the layer's routing is charged to its first
+    step, its combine + RMSNorm to its last)."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import numpy as np
+    from oracle import moe
+    from synth import gen
+    bits = cfg.format.bits
+    x = gen.tokens(SEED, cfg, 0).astype(np.float64)
+    state = {"l": 0, "idx": None, "g": None, "raw": None, "outs": {}}
+
+    def step():
+        l = state["l"] % cfg.L
+        j = len(state["outs"])
+        t = 0.0
+        if j == 0:
+            Wr, b = gen.router(SEED, cfg, l), gen.bias(SEED, cfg, l)
+            t0 = time.perf_counter()
+            idx, g, _ = moe.route(state.get("x", x), Wr, b, cfg.k)
+            t += time.perf_counter() - t0
+            state["idx"], state["g"] = idx, g
+            e0 = int(idx[0, 0])
+        e = int(state["idx"][0, j])
+        raw = gen.expert(SEED, cfg, l, e)
+        t0 = time.perf_counter()
+        W = tuple(moe.dequantize(raw[n + "_codes"], raw[n + "_scales"], bits) for n in ("gate", "up", "down"))
+        xx = state.get("x", x)
+        state["outs"][j] = moe.expert_ffn(xx[:1], *W)[0]
+        if j == cfg.k - 1:
+            y = moe.combine(np.stack([state["outs"][i] for i in range(cfg.k)]), state["g"][0])
+            state["x"] = moe.rmsnorm_residual(xx[:1], y[None], cfg.eps)
+            state["outs"] = {}
+            state["l"] += 1
+        t += time.perf_counter() - t0
+        return t
+
+    for _ in range(args.warmup):
+        step()
+    spent = sum(step() for _ in range(args.steps))
+    tokens = args.steps / (cfg.L * cfg.k)
+    value = tokens / spent
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * spent / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_desc(cfg, 1),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{args.steps} steps of one expert FFN each (1/{cfg.k} of a layer of one "
+                                       f"token), weight generation excluded"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- ours --
+def run_ours(args, cfg):
+    import numpy as np
+    import torch
+
+    from quantised_expert_decode_b200.model import DecodeStack
+    from synth import gen
+    from synth.workload import device_layers
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+    T = cfg.T
+    layers, routers, biases = device_layers(SEED, cfg)
+    stack = DecodeStack(layers, routers, biases, T, cfg.k, cfg.eps)
+    tstack = DecodeStack(layers, routers, biases, T, cfg.k, cfg.eps, timing=True)
+    n_in = min(args.steps + args.warmup, 4096)
+    xs_host = np.stack([gen.tokens(SEED + 1000 * rank, cfg, s) for s in range(n_in)])   # [n, T, H]
+    xs = torch.from_numpy(xs_host).cuda()
+    stream = torch.cuda.current_stream()
+
+    def step(s):
+        stack.x_in.copy_(xs[s % n_in], non_blocking=True)
+        stack.decode(stream)
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+    if stack.status() != 0:
+        raise RuntimeError("device status set during warm-up")
+    props = torch.cuda.get_device_properties(local)
+    clocks = Clocks(getattr(props, "uuid", None) and f"GPU-{props.uuid}")
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(args.steps):
+        step(args.warmup + s)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    clk = clocks.stop()
+    ms = max_over_ranks(ms, world)
+    value = world * args.steps * T / (ms / 1e3)
+
+    # end to end through the host-buffer entry point (pinned memory)
+    xh = torch.from_numpy(xs_host).pin_memory()
+    outh = torch.empty((T, cfg.H), dtype=torch.float32).pin_memory()
+    n_e2e = args.steps
+    torch.cuda.synchronize()
+    barrier(world)
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for s in range(n_e2e):
+        stack.decode_host(xh[s % n_in], outh, stream)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(e2.elapsed_time(e3), world)
+    if stack.status() != 0:
+        raise RuntimeError("device status set during the timed run")
+
+    # kernel durations: the same steps through the graph with event nodes around
+    # every route and FFN node (event nodes split the programmatic edges, so
+    # this graph is timed separately from the headline)
+    n_t = min(args.steps, 500)
+    for s in range(args.warmup):
+        tstack.x_in.copy_(xs[s % n_in], non_blocking=True)
+        tstack.decode(stream)
+    torch.cuda.synchronize()
+    e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    per_layer = []
+    e4.record(stream)
+    for s in range(n_t):
+        tstack.x_in.copy_(xs[(args.warmup + s) % n_in], non_blocking=True)
+        tstack.decode(stream)
+    e5.record(stream)
+    torch.cuda.synchronize()
+    route_ms, ffn_ms = tstack.layer_times()
+    ms_timing_graph = e4.elapsed_time(e5) / n_t
+    if tstack.status() != 0:
+        raise RuntimeError("device status set during the timing-graph run")
+
+    hbm, peak_kind = peaks()
+    idx = stack.idx.cpu().numpy()
+    uniq = [len(set(idx[l].ravel().tolist())) for l in range(cfg.L)]
+    ffn_bytes = [u * cfg.expert_bytes() for u in uniq]
+    ffn_mean_s = statistics.mean(ffn_ms) / 1e3
+    achieved = statistics.mean(b / (t / 1e3) for b, t in zip(ffn_bytes, ffn_ms)) / 1e9
+    expert_bytes_step = sum(ffn_bytes)
+    router_bytes_step = cfg.L * cfg.router_bytes()
+    step_s = ms / 1e3 / args.steps
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u8 codes x s8 activation limbs -> s32 (tensor core), f32 epilogue, f64 router",
+        "data": "synthetic (seeded SplitMix64 weights, Box-Muller activations)",
+        "config": dict(workload_desc(cfg, T), parallelism=f"replicas x{world}"),
+        "roofline": {"bound": "hbm", "kernel": "ffn_decode_kernel", "achieved": achieved, "peak": hbm,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": stored_traffic(args.workload),
+                     "algorithmic_bytes_per_launch": statistics.mean(ffn_bytes),
+                     "avg_launch_us": 1e6 * ffn_mean_s,
+                     "timing": "CUDA event nodes around every FFN node of a graph replayed over the same "
+                               "steps (per-layer durations of its last replay)"},
+        "stack": {"expert_bytes_per_step": expert_bytes_step, "router_bytes_per_step": router_bytes_step,
+                  "expert_GBps": expert_bytes_step / step_s / 1e9,
+                  "all_weight_GBps": (expert_bytes_step + router_bytes_step) / step_s / 1e9,
+                  "frac_all_weight_of_measured_hbm": (expert_bytes_step + router_bytes_step) / step_s / 1e9 / hbm,
+                  "frac_expert_of_8TBps": expert_bytes_step / step_s / 8e12,
+                  "route_us_mean": 1e3 * statistics.mean(route_ms), "ffn_us_mean": 1e3 * statistics.mean(ffn_ms),
+                  "ms_per_step_event_graph": ms_timing_graph,
+                  "unique_experts_per_layer_mean": statistics.mean(uniq),
+                  "reuse_pairs_per_unique_expert": T * cfg.k / statistics.mean(uniq)},
+        "e2e": {"value": world * n_e2e * T / (ms_e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * cfg.H * 4, "d2h_bytes_per_step": T * cfg.H * 4,
+                "path": "qmoe_stack_decode_host: pinned host x -> graph replay -> pinned host output"},
+        "clocks": clk,
+        "gpu_launches": args.steps * stack.kernels_per_replay,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, T)
+    stack.close()
+    tstack.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_layer(args, cfg):
+    """One decode layer per step (router + FFN, one token), L2 flushed between
+    steps so every step reads its experts from HBM; per-step CUDA events."""
+    import numpy as np
+    import torch
+
+    import quantised_expert_decode_b200 as q
+    from synth import gen
+    from synth.workload import device_layers
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    layers, routers, _ = device_layers(SEED, cfg, 1)
+    layer, Wr = layers[0], routers[0]
+    T = cfg.T
+    n_in = args.steps + args.warmup
+    xs = torch.from_numpy(np.stack([gen.tokens(SEED, cfg, s) for s in range(n_in)])).cuda()
+    idx = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
+    gate = torch.empty((T, cfg.k), dtype=torch.float32, device="cuda")
+    y = torch.empty((T, cfg.H), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rws = torch.zeros(q.qmoe_route_workspace_bytes(T, cfg.E), dtype=torch.uint8, device="cuda")
+    fws = torch.zeros(q.qmoe_decode_workspace_bytes(T, cfg.k, cfg.H, cfg.I), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    h = layer.handle()
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+
+    def step(s, e=None):
+        flush.fill_(s & 255)
+        if e:
+            e[0].record(stream)
+        q.qmoe_route(Wr, None, xs[s], q.F32, T, cfg.H, cfg.E, cfg.k, idx, gate, rws, st, stream)
+        if e:
+            e[1].record(stream)
+        q.qmoe_ffn_decode(h, xs[s], T, idx, gate, cfg.k, y, fws, st, stream)
+        if e:
+            e[2].record(stream)
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+    for s in range(args.steps):
+        step(args.warmup + s, ev[s])
+    torch.cuda.synchronize()
+    if q.qmoe_read_status(st) != 0:
+        raise RuntimeError("device status set")
+    route_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    ffn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    layer_s = (sum(route_ms) + sum(ffn_ms)) / 1e3
+    hbm, peak_kind = peaks()
+    ffn_bytes = cfg.k * cfg.expert_bytes()
+    achieved = ffn_bytes / (statistics.mean(ffn_ms) / 1e3) / 1e9
+    line = {"metric": "routed-MoE decode layer tokens/s (one layer); HBM GB/s on expert bytes vs peak",
+            "value": args.steps * T / layer_s, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * layer_s / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "u8 codes x s8 activation limbs -> s32 (tensor core), f32 epilogue, f64 router",
+            "data": "synthetic",
+            "config": {"workload": f"one decode layer: {cfg.E} Q{cfg.fmt} experts, hidden {cfg.H}, intermediate "
+                                   f"{cfg.I}, top-{cfg.k}, {T} token; L2 flushed (256 MB write) between steps"},
+            "roofline": {"bound": "hbm", "kernel": "ffn_decode_kernel", "achieved": achieved, "peak": hbm,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
+                         "traffic": stored_traffic(args.workload), "algorithmic_bytes_per_launch": ffn_bytes,
+                         "avg_launch_us": 1e3 * statistics.mean(ffn_ms),
+                         "median_launch_us": 1e3 * statistics.median(ffn_ms)},
+            "route_us_mean": 1e3 * statistics.mean(route_ms),
+            "gpu_launches": 2 * args.steps}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    from synth import configs
+    cfg = configs.get(WORKLOADS[args.workload])
+    if args.impl == "reference":
+        run_reference(args, cfg, cfg.T)
+    elif args.workload == "layer":
+        run_layer(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

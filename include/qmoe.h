@@ -1,0 +1,231 @@
+/*
+ * qmoe.h - C ABI of libqmoe, the B200 (sm_100a) routed mixture-of-experts FFN
+ * with 2-/4-bit block-quantised experts.
+ *
+ * Sources (web pages on the Strata engine; the method is defined by them and by
+ * the workload definitions of this library's synthetic configurations):
+ *   [P1] hexlives, "Commitment is a speedup" - one model whose 24,576 experts
+ *        are consulted about ten per token; the decode GEMV is bandwidth-bound
+ *        and a tensor-core variant lost on single-token shapes (fourth
+ *        paragraph).
+ *   [P3] pyshine, Strata source-tree tour - "Understanding the Architecture":
+ *        48 captured layer graphs fed through fixed-address device buffers; a
+ *        gate-weighted moe_combine summed on the device; wrong expert geometry
+ *        refused rather than mis-indexed; router_top10.cu routes each token to
+ *        ten experts; batched prefill in chunks of up to 8,192 tokens.
+ *
+ * Conventions shared by every call
+ *   - Every pointer argument is a DEVICE pointer unless its name ends in _host.
+ *     The caller owns all memory; no call allocates or frees device memory.
+ *   - Every device pointer must be 16-byte aligned, except route tables
+ *     (idx int32 [T,k], gate fp32 [T,k]), which need 4-byte alignment.
+ *   - Calls are asynchronous on the given stream (a cudaStream_t passed as
+ *     qmoe_stream_t; 0 = legacy default stream) and capturable into a CUDA
+ *     graph, except where stated.
+ *   - Host-side validation failures return an error code and launch nothing.
+ *   - Device-detected faults (an expert index outside [0, E), a repeated expert
+ *     within one token's route, a device wait that ran out of its time budget)
+ *     are written to the caller's int32 *dev_status (first error wins; 0 = ok)
+ *     and the kernel leaves without touching memory out of bounds. Read it with
+ *     qmoe_read_status() after synchronising the stream.
+ *   - No exception crosses this ABI.
+ */
+#ifndef QMOE_H_
+#define QMOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+#if defined(__GNUC__)
+#pragma GCC visibility push(default)
+#endif
+
+typedef struct CUstream_st *qmoe_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  QMOE_OK = 0,
+  QMOE_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, size out of range */
+  QMOE_ERR_GEOMETRY = 2,      /* tensor shapes disagree with the expert handle */
+  QMOE_ERR_UNSUPPORTED = 3,   /* valid request outside what this build supports */
+  QMOE_ERR_WORKSPACE = 4,     /* workspace smaller than *_workspace_bytes() */
+  QMOE_ERR_CUDA = 5,          /* a CUDA runtime call failed */
+  QMOE_ERR_TIMEOUT = 6,       /* a device-side wait exceeded its budget */
+  QMOE_ERR_DEVICE_STATUS = 7  /* invalid routed index seen on the device */
+} qmoe_status;
+
+enum { QMOE_Q2 = 2, QMOE_Q4 = 4 };        /* block formats (bits per code) */
+enum { QMOE_F32 = 0, QMOE_BF16 = 1 };     /* activation dtypes */
+enum { QMOE_GATE_UP = 0, QMOE_DOWN = 1 }; /* packed matrix kinds */
+
+/* One layer's experts, already packed by qmoe_pack().
+ *   gate_up: E experts x {gate [I,H], up [I,H]}   (reduction axis H)
+ *   down   : E experts x down [H,I]               (reduction axis I)
+ * gate_up_bytes / down_bytes are the sizes of the two buffers; a handle whose
+ * sizes differ from qmoe_packed_bytes() of its E/H/I/fmt is refused with
+ * QMOE_ERR_GEOMETRY ("a wrong expert geometry must be refused rather than
+ * mis-indexed", [P3] "Understanding the Architecture").
+ * Geometry limits: H and I multiples of 128; E <= 1024. */
+typedef struct {
+  int E, H, I, fmt;
+  const void *gate_up;
+  const void *down;
+  size_t gate_up_bytes;
+  size_t down_bytes;
+} qmoe_experts;
+
+/* ---------------------------------------------------------------- format --
+ * Self-defined block format: 32 consecutive weights along the reduction axis
+ * share fp16 scale d and fp16 min m, w = d*q + m, q a 2-bit (Q2) or 4-bit (Q4)
+ * code. (Strata loads third-party GGUF quant types - [P3] "How It Works" - whose
+ * specifications are not part of the method; this format takes their place.)
+ *
+ * Canonical input layout for qmoe_pack, per expert matrix [rows, K]:
+ *   codes  uint8  [E, rows, K*bits/8]: Q2 code j in byte j/4 bits 2*(j%4);
+ *                                     Q4 code j in byte j/2, low nibble = even j
+ *   scales uint16 [E, rows, K/32, 2]:  fp16 (d, m) per block
+ * For QMOE_GATE_UP the caller passes gate and up separately (rows = I, K = H);
+ * for QMOE_DOWN rows = H, K = I and the *_up pointers are NULL.
+ *
+ * Packed layout (this library's choice): 16-row tiles; inside a tile the codes
+ * are arranged so that lane l of a warp loads 16 contiguous bytes holding its
+ * tensor-core operand fragments, followed by the tile's (d, m) pairs.
+ * qmoe_packed_bytes() equals the canonical size (8 (Q2) or 16 (Q4) code bytes
+ * + 4 scale bytes per 32-weight block): packing adds no padding. */
+size_t qmoe_packed_bytes(int fmt, int kind, int E, int H, int I);
+
+/* Pack one layer's canonical matrices into dst (device, qmoe_packed_bytes()
+ * bytes). Errors: INVALID_ARG for null pointers or dst_bytes too small,
+ * UNSUPPORTED for H or I not multiples of 128 or fmt not Q2/Q4. */
+qmoe_status qmoe_pack(int fmt, int kind, int E, int H, int I,
+                      const uint8_t *codes_gate_or_down, const uint16_t *scales_gate_or_down,
+                      const uint8_t *codes_up, const uint16_t *scales_up,
+                      void *dst, size_t dst_bytes, qmoe_stream_t stream);
+
+/* ---------------------------------------------------------------- router --
+ * Router GEMV, softmax, top-k with renormalised gates ([P3] router_top10.cu,
+ * "Understanding the Architecture"; "the router names ten experts per token",
+ * [P3] end-to-end paragraph). For each token t:
+ *   l[t,e] = sum_h x[t,h] * Wr[e,h] (+ bias[e])     accumulated in float64
+ *   idx[t,:] = the k largest l[t,:], by value descending, ties to lower e
+ *   gate[t,j] = exp(l[t,idx[t,j]] - l[t,idx[t,0]]) / sum_j' exp(...)
+ * Inputs: Wr fp32 [E,H] row-major; bias fp32 [E] or NULL; x [T,H] fp32
+ * (x_dtype QMOE_F32) or bf16 (QMOE_BF16). Outputs: idx int32 [T,k] and
+ * gate fp32 [T,k]. Workspace: qmoe_route_workspace_bytes(T, E) bytes, zeroed
+ * once before first use (it is left zeroed by every completed call).
+ * Limits: 1 <= k <= 16, k <= E <= 1024, H multiple of 128, T >= 1.
+ * T <= 8 runs the single-pass decode router (float64 GEMV); larger T runs the
+ * prefill router (fp32 tiles with a per-token rounding bound; tokens whose
+ * ordering the bound cannot certify are recomputed in float64). */
+size_t qmoe_route_workspace_bytes(int T, int E);
+qmoe_status qmoe_route(const float *Wr, const float *bias, const void *x, int x_dtype,
+                       int T, int H, int E, int k, int32_t *idx, float *gate,
+                       void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                       qmoe_stream_t stream);
+
+/* Residual RMSNorm fused in front of the router (the residual stack every
+ * block reads and writes, [P3] "Understanding the Architecture"):
+ *   x_out[t,:] = z / sqrt(mean(z^2) + eps),  z = x_in[t,:] + y[t,:]
+ * then routes x_out exactly like qmoe_route (fp32 activations, T <= 8).
+ * x_out must not alias x_in or y. */
+qmoe_status qmoe_residual_route(const float *x_in, const float *y, float eps, float *x_out,
+                                const float *Wr, const float *bias, int T, int H, int E, int k,
+                                int32_t *idx, float *gate, void *workspace,
+                                size_t workspace_bytes, int32_t *dev_status,
+                                qmoe_stream_t stream);
+
+/* Standalone residual RMSNorm: x_out = RMSNorm(x_in + y), fp32 [T,H]. x_out
+ * may alias x_in. */
+qmoe_status qmoe_rmsnorm_residual(const float *x_in, const float *y, float eps, float *x_out,
+                                  int T, int H, qmoe_stream_t stream);
+
+/* -------------------------------------------------------------- decode FFN --
+ * Routed expert FFN with the gate-weighted combine on the device ([P3]
+ * moe_combine, native_moe.cu, "Understanding the Architecture"; [P1] the
+ * bandwidth-bound decode GEMV), for decode and speculative-verify batches:
+ *   for every token t and slot j, e = idx[t,j]:
+ *     h = silu(Wg_e x_t) * (Wu_e x_t),  silu(a) = a / (1 + exp(-a))
+ *   y[t,:] = sum_j gate[t,j] * (Wd_e h)        (summed in slot order)
+ * x fp32 [T,H]; idx int32 [T,k]; gate fp32 [T,k]; y fp32 [T,H] (overwritten).
+ * Limits: 1 <= T <= 8, 1 <= k <= 16. One cooperative grid of one CTA per SM:
+ * weights stream through shared memory with bulk asynchronous copies and are
+ * contracted on tensor cores (codes x 16-bit fixed-point activations, exact
+ * integer products, fp32 scaling per block).
+ * Workspace: qmoe_decode_workspace_bytes(T, k, H, I), zeroed once before first
+ * use (every completed call leaves its barrier words as it found them).
+ * Errors: GEOMETRY if the handle's H/I/E do not match; device status for an
+ * index outside [0, E) or a repeated expert in one token; TIMEOUT if a grid
+ * barrier waited longer than its budget (about one second). */
+size_t qmoe_decode_workspace_bytes(int T, int k, int H, int I);
+qmoe_status qmoe_ffn_decode(const qmoe_experts *experts, const float *x, int T,
+                            const int32_t *idx, const float *gate, int k, float *y,
+                            void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                            qmoe_stream_t stream);
+
+/* ------------------------------------------------------------ layer stack --
+ * L layers of route -> FFN -> residual RMSNorm captured once into one CUDA
+ * graph ([P3]: 48 captured layer graphs; "a graph bakes in its arguments, so
+ * per-token values arrive through fixed-address device buffers").
+ *   x_0 = input;  for l: (idx_l, gate_l) = route_l(x_l);  y_l = FFN_l(x_l);
+ *                       x_{l+1} = RMSNorm(x_l + y_l)
+ *   output = x_L
+ * The descriptor's arrays are host arrays of L entries (copied at create).
+ * The stack lives in caller workspace (qmoe_stack_workspace_bytes()); it keeps
+ * the input, output and every layer's idx/gate there at fixed addresses. */
+enum { QMOE_STACK_TIMING = 1 }; /* capture CUDA events around every route and FFN node */
+
+typedef struct {
+  int L, T, k;
+  float eps;
+  const float *const *Wr;      /* L device pointers, fp32 [E,H] */
+  const float *const *bias;    /* NULL or L device pointers (entries may be NULL) */
+  const qmoe_experts *layers;  /* L handles with identical E/H/I/fmt */
+  int flags;                   /* 0 or QMOE_STACK_TIMING */
+} qmoe_stack_desc;
+
+typedef struct qmoe_stack qmoe_stack;
+
+size_t qmoe_stack_workspace_bytes(const qmoe_stack_desc *desc);
+/* Builds and instantiates the graph (host allocation of graph objects only).
+ * Zeroes the workspace on `stream`. Not capturable. */
+qmoe_status qmoe_stack_create(const qmoe_stack_desc *desc, void *workspace, size_t workspace_bytes,
+                              qmoe_stream_t stream, qmoe_stack **out);
+qmoe_status qmoe_stack_destroy(qmoe_stack *stack);
+/* Fixed device buffers of the stack: input x [T,H], output x [T,H], idx [L,T,k],
+ * gate [L,T,k] and the device status word. Any argument may be NULL. */
+qmoe_status qmoe_stack_buffers(const qmoe_stack *stack, float **x_in, float **x_out,
+                               int32_t **idx, float **gate, int32_t **dev_status);
+/* Kernel launches in one replay of the stack's graph (2L + 1). */
+int qmoe_stack_kernels_per_replay(const qmoe_stack *stack);
+/* Per-layer durations (ms) of the most recent completed replay, measured by
+ * the event nodes of a QMOE_STACK_TIMING stack: route_ms[l] spans layer l's
+ * router (with its fused residual RMSNorm), ffn_ms[l] its FFN kernel. Host
+ * arrays of L floats (either may be NULL). Synchronous; UNSUPPORTED without
+ * the flag. */
+qmoe_status qmoe_stack_layer_times(const qmoe_stack *stack, float *route_ms, float *ffn_ms);
+/* One graph replay on `stream`: reads the stack's input buffer, writes its
+ * output buffer. */
+qmoe_status qmoe_stack_decode(qmoe_stack *stack, qmoe_stream_t stream);
+/* End to end from host memory: copies x_host (fp32 [T,H], ideally pinned) into
+ * the input buffer, replays the graph and copies the output to x_out_host.
+ * Asynchronous; synchronise `stream` before reading x_out_host. */
+qmoe_status qmoe_stack_decode_host(qmoe_stack *stack, const float *x_host, float *x_out_host,
+                                   qmoe_stream_t stream);
+
+/* ------------------------------------------------------------------- misc -- */
+/* Synchronous: copies *dev_status to the host and maps it to a status. */
+qmoe_status qmoe_read_status(const int32_t *dev_status);
+const char *qmoe_status_string(qmoe_status s);
+/* Number of this library's kernel launches issued since load (host counter). */
+uint64_t qmoe_launch_count(void);
+
+#if defined(__GNUC__)
+#pragma GCC visibility pop
+#endif
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QMOE_H_ */

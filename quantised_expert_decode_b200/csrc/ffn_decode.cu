@@ -1,0 +1,730 @@
+// Routed expert FFN + gate-weighted combine for decode / verify batches (T <= 8).
+//
+// One grid of one CTA per SM (all resident), three phases separated by grid barriers:
+//   phase 1  gate and up projections: items are (expert, gate|up, 16-row tile)
+//            over K = H; results a_g, a_u go to the workspace.
+//   phase 2  down projection: items are (expert, 32-row tile) over K = I on
+//            h = silu(a_g) * a_u; each result is scaled by its gate and stored
+//            per (token, slot).
+//   phase 3  y[t] = sum over slots j (in slot order) of the phase-2 results.
+// Weights stream HBM -> shared memory through bulk asynchronous copies issued by
+// one producer thread into a ring of slots (mbarrier full/empty pairs); the
+// copies of phase-2 tiles start as soon as ring slots free up, so they overlap
+// phase 1 and the first grid barrier.
+//
+// Contraction: activations of every 32-element block are quantised to 16-bit
+// fixed point with a per-block fp32 scale s (X = rint(v / s), |X| <= 32639) and
+// split into signed 8-bit limbs X = 256*hi + lo. The integer MMA m16n8k32
+// (u8 codes x s8 limbs, s32 accumulate) gives exact sum q*hi and sum q*lo per
+// block; the block's contribution is d * s * (256*Qhi + Qlo) + m * s * sum(X).
+// The eight MMA columns hold (hi, lo) pairs of up to four (token, block) pairs,
+// so even a single token keeps every lane busy in the fp32 epilogue.
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "layout.cuh"
+
+namespace qmoe {
+namespace {
+
+constexpr int NCW = 8;                     // consumer warps
+constexpr int FD_THREADS = 32 * (NCW + 1); // + one producer warp
+constexpr int FD_MAXT = 8;
+constexpr int FD_MAXK = 16;
+constexpr int FD_MAXP = FD_MAXT * FD_MAXK; // (token, slot) pairs
+constexpr int CONSUMER_BAR = 1;            // named barrier id for the consumer warps
+constexpr float QMAX = 32639.0f;           // keeps both limbs inside int8
+
+struct Plan {
+  int err;
+  int abort;
+  int U;
+  int ue[FD_MAXP];
+  int nt[FD_MAXP];
+  int pbase[FD_MAXP + 1];
+  int ptok[FD_MAXP];
+  int pslot[FD_MAXP];
+  float pgate[FD_MAXP];
+  int sidx[FD_MAXP];
+  float sgate[FD_MAXP];
+  unsigned bm[32];
+  int vids[NCW][FD_MAXT];  // per consumer warp: limb-region vectors of the current item
+};
+
+struct FfnArgs {
+  const uint8_t *gu;
+  const uint8_t *dn;
+  const float *x;
+  const int32_t *idx;
+  const float *gate;
+  float *y;
+  float *abuf;    // [P][2][I]
+  float *part;    // [T][k][H]
+  unsigned *bar;  // grid barrier counter
+  int32_t *status;
+  int T, k, E, H, I;
+  int slot_bytes, nslots;
+  int limb_bytes;  // activation-limb region
+  int lsc_count;   // float2 entries of the limb-scale table
+};
+
+// Shared-memory carve-up (byte offsets from the dynamic base), used by host and device.
+struct SmemLayout {
+  size_t bars, plan, limbs, lsc, total;
+};
+__host__ __device__ inline SmemLayout smem_layout(int nslots, int slot_bytes, int limb_bytes, int lsc_count) {
+  SmemLayout o;
+  o.bars = (size_t)nslots * slot_bytes;                       // slot_bytes is a multiple of 128
+  o.plan = (o.bars + (size_t)nslots * 16 + 15) & ~(size_t)15;
+  o.limbs = (o.plan + sizeof(Plan) + 127) & ~(size_t)127;
+  o.lsc = (o.limbs + (size_t)limb_bytes + 15) & ~(size_t)15;
+  o.total = o.lsc + (size_t)lsc_count * 8;
+  return o;
+}
+
+__device__ __forceinline__ float h2f(uint32_t bits16) { return __half2float(__ushort_as_half((unsigned short)bits16)); }
+
+// Quantise a 128-element chunk (4 blocks of 32) held one float4 per lane: lane
+// j carries elements 4j..4j+3, i.e. block j/8. Writes the int8 limbs of the
+// four blocks and (s, s * sum X) per block. The block's min term then uses the
+// same quantised values as its code term, so the whole block sees one
+// consistent activation s*X and the only error is that of quantising v,
+// carried through zero-mean weights.
+__device__ __forceinline__ int quant_one(float v, float inv) {
+  int X = __float2int_rn(v * inv);
+  return max(-32639, min(32639, X));
+}
+
+__device__ __forceinline__ void quant_chunk(float4 v, uint8_t *limbs_vec, float2 *lsc_vec, int chunk, int lane) {
+  float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
+  float s = 0.0f, inv = 0.0f;
+  if (a > 0.0f) {
+    s = a / QMAX;
+    inv = QMAX / a;
+  }
+  int X0 = quant_one(v.x, inv), X1 = quant_one(v.y, inv), X2 = quant_one(v.z, inv), X3 = quant_one(v.w, inv);
+  int h0 = (X0 + 128) >> 8, h1 = (X1 + 128) >> 8, h2 = (X2 + 128) >> 8, h3 = (X3 + 128) >> 8;
+  int l0 = X0 - (h0 << 8), l1 = X1 - (h1 << 8), l2 = X2 - (h2 << 8), l3 = X3 - (h3 << 8);
+  uint32_t hw = (uint32_t)(h0 & 0xff) | ((uint32_t)(h1 & 0xff) << 8) | ((uint32_t)(h2 & 0xff) << 16) |
+                ((uint32_t)(h3 & 0xff) << 24);
+  uint32_t lw = (uint32_t)(l0 & 0xff) | ((uint32_t)(l1 & 0xff) << 8) | ((uint32_t)(l2 & 0xff) << 16) |
+                ((uint32_t)(l3 & 0xff) << 24);
+  const int blk = chunk * 4 + (lane >> 3);
+  uint8_t *rec = limbs_vec + (size_t)blk * 64 + (lane & 7) * 4;
+  *reinterpret_cast<uint32_t *>(rec) = hw;
+  *reinterpret_cast<uint32_t *>(rec + 32) = lw;
+  int sx = X0 + X1 + X2 + X3;
+  sx += __shfl_xor_sync(0xffffffffu, sx, 1);
+  sx += __shfl_xor_sync(0xffffffffu, sx, 2);
+  sx += __shfl_xor_sync(0xffffffffu, sx, 4);   // |sx| < 2^24: exact in fp32
+  if ((lane & 7) == 0) lsc_vec[blk] = make_float2(s, s * (float)sx);
+}
+
+struct Acc {
+  float r0q0, r0q1, r1q0, r1q1;  // rows g / g+8 x column groups q = 0 / 1
+};
+
+// Dot products of one 16-row tile (K = 32 * nblk, nblk % 4 == 0) with n <= NP
+// activation vectors (vector ids vid[0..n)). Returns the lane's share; see the
+// file header for the column layout. Not inlined: phase 1 and phase 2 share one
+// copy of the code, which keeps the instruction footprint small.
+template <int BITS, int NP>
+__device__ __noinline__ Acc tile_dot(const uint8_t *tile, int nblk, const uint8_t *limbs, const float2 *lsc,
+                                     const int *vid, int n) {
+  constexpr int TS = NP <= 4 ? NP : 4;        // tokens per column set
+  constexpr int BS = NP <= 4 ? 4 / NP : 1;    // blocks per column set
+  constexpr int NQ = NP == 8 ? 2 : 1;         // column groups per block
+  constexpr int NSET = 4 / BS;                // column sets per 4-block chunk
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int pp = g >> 1, plimb = g & 1;
+  const int ptau = pp % TS, pbeta = pp / TS;
+  const int own_tau = t % TS, own_beta = t / TS;
+  const uint8_t *sbase = tile + 64 * nblk * BITS;   // scales follow the codes
+  float acc[2][NQ];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) acc[0][q] = acc[1][q] = 0.0f;
+  // vector ids of the B columns this lane provides / the D columns it reads
+  int pv[NQ], ov[NQ];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    const int ptq = (NP == 8) ? 4 * q + pp : ptau;
+    const int otq = (NP == 8) ? 4 * q + t : own_tau;
+    pv[q] = ptq < n ? vid[ptq] : -1;
+    ov[q] = otq < n ? vid[otq] : -1;
+  }
+
+#pragma unroll 1
+  for (int c = 0; c < (nblk >> 2); ++c) {
+    uint32_t w[8];
+    if (BITS == 2) {
+      const uint4 q = *reinterpret_cast<const uint4 *>(tile + c * 512 + lane * 16);
+      w[0] = q.x; w[1] = q.y; w[2] = q.z; w[3] = q.w;
+    } else {
+      const uint4 q0 = *reinterpret_cast<const uint4 *>(tile + (2 * c) * 512 + lane * 16);
+      const uint4 q1 = *reinterpret_cast<const uint4 *>(tile + (2 * c + 1) * 512 + lane * 16);
+      w[0] = q0.x; w[1] = q0.y; w[2] = q0.z; w[3] = q0.w;
+      w[4] = q1.x; w[5] = q1.y; w[6] = q1.z; w[7] = q1.w;
+    }
+#pragma unroll
+    for (int sb = 0; sb < NSET; ++sb) {
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        // B limbs this lane provides for this column set
+        uint32_t b0 = 0u, b1 = 0u;
+        if (pv[q] >= 0) {
+          const int blk = c * 4 + sb * BS + ((NP == 8) ? 0 : pbeta);
+          const uint8_t *lp = limbs + ((size_t)pv[q] * nblk + blk) * 64 + plimb * 32 + 4 * t;
+          b0 = *reinterpret_cast<const uint32_t *>(lp);
+          b1 = *reinterpret_cast<const uint32_t *>(lp + 16);
+        }
+        int d0 = 0, d1 = 0, d2 = 0, d3 = 0;
+#pragma unroll
+        for (int beta = 0; beta < BS; ++beta) {
+          const int bb = sb * BS + beta;
+          uint32_t a0, a1, a2, a3;
+          if (BITS == 2) {
+            const uint32_t x = w[bb];
+            a0 = x & 0x03030303u;
+            a1 = (x >> 2) & 0x03030303u;
+            a2 = (x >> 4) & 0x03030303u;
+            a3 = (x >> 6) & 0x03030303u;
+          } else {
+            const uint32_t x0 = w[2 * bb], x1 = w[2 * bb + 1];
+            a0 = x0 & 0x0F0F0F0Fu;
+            a1 = (x0 >> 4) & 0x0F0F0F0Fu;
+            a2 = x1 & 0x0F0F0F0Fu;
+            a3 = (x1 >> 4) & 0x0F0F0F0Fu;
+          }
+          const bool on = (NP == 8) || (pbeta == beta);
+          mma_u8s8(d0, d1, d2, d3, a0, a1, a2, a3, on ? b0 : 0u, on ? b1 : 0u);
+        }
+        if (ov[q] >= 0) {
+          const int bo = c * 4 + sb * BS + ((NP == 8) ? 0 : own_beta);
+          const float v0 = (float)(d0 * 256 + d1);
+          const float v1 = (float)(d2 * 256 + d3);
+          const float2 ss = lsc[(size_t)ov[q] * nblk + bo];
+          const uint2 dm = *reinterpret_cast<const uint2 *>(sbase + (bo * 8 + g) * 8);
+          acc[0][q] = fmaf(h2f(dm.x & 0xffffu), ss.x * v0, fmaf(h2f(dm.x >> 16), ss.y, acc[0][q]));
+          acc[1][q] = fmaf(h2f(dm.y & 0xffffu), ss.x * v1, fmaf(h2f(dm.y >> 16), ss.y, acc[1][q]));
+        }
+      }
+    }
+  }
+  if (NP == 1) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      acc[r][0] += __shfl_xor_sync(0xffffffffu, acc[r][0], 1);
+      acc[r][0] += __shfl_xor_sync(0xffffffffu, acc[r][0], 2);
+    }
+  } else if (NP == 2) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) acc[r][0] += __shfl_xor_sync(0xffffffffu, acc[r][0], 2);
+  }
+  Acc out;
+  out.r0q0 = acc[0][0];
+  out.r1q0 = acc[1][0];
+  out.r0q1 = NQ > 1 ? acc[0][NQ - 1] : 0.0f;
+  out.r1q1 = NQ > 1 ? acc[1][NQ - 1] : 0.0f;
+  return out;
+}
+
+// Token slot held by this lane for column group q after tile_dot (or -1).
+template <int NP>
+__device__ __forceinline__ int owner_tau(int t, int q) {
+  if (NP == 8) return 4 * q + t;
+  if (q != 0) return -1;
+  return t < NP ? t : -1;
+}
+
+template <int BITS>
+__device__ __forceinline__ int dispatch_dot(const uint8_t *tile, int nblk, const uint8_t *limbs, const float2 *lsc,
+                                            const int *vid, int n, Acc &acc) {
+  if (n <= 1) { acc = tile_dot<BITS, 1>(tile, nblk, limbs, lsc, vid, n); return 1; }
+  if (n <= 2) { acc = tile_dot<BITS, 2>(tile, nblk, limbs, lsc, vid, n); return 2; }
+  if (n <= 4) { acc = tile_dot<BITS, 4>(tile, nblk, limbs, lsc, vid, n); return 4; }
+  acc = tile_dot<BITS, 8>(tile, nblk, limbs, lsc, vid, n);
+  return 8;
+}
+
+__device__ __forceinline__ int owner(int np, int t, int q) {
+  switch (np) {
+    case 1: return owner_tau<1>(t, q);
+    case 2: return owner_tau<2>(t, q);
+    case 4: return owner_tau<4>(t, q);
+    default: return owner_tau<8>(t, q);
+  }
+}
+
+// Route table -> unique experts (ascending), their tokens (ascending) and slots.
+__device__ void build_plan(const FfnArgs &a, Plan *pl) {
+  const int lane = threadIdx.x & 31;
+  const int P = a.T * a.k;
+  pl->bm[lane] = 0u;
+  for (int p = lane; p < P; p += 32) {
+    pl->sidx[p] = a.idx[p];
+    pl->sgate[p] = a.gate[p];
+  }
+  __syncwarp();
+  int bad = 0;
+  for (int p = lane; p < P; p += 32) {
+    int e = pl->sidx[p];
+    if (e < 0 || e >= a.E) {
+      bad = DEV_BAD_INDEX;
+      continue;
+    }
+    int t = p / a.k, j = p % a.k;
+    for (int j2 = 0; j2 < j; ++j2)
+      if (pl->sidx[t * a.k + j2] == e) bad = DEV_DUP_INDEX;
+    atomicOr(&pl->bm[e >> 5], 1u << (e & 31));
+  }
+  unsigned badmask = __ballot_sync(0xffffffffu, bad != 0);
+  if (badmask) {
+    int first = __ffs(badmask) - 1;
+    int code = __shfl_sync(0xffffffffu, bad, first);
+    if (lane == 0) {
+      pl->err = code;
+      set_status(a.status, code);
+    }
+    return;
+  }
+  __syncwarp();
+  unsigned word = pl->bm[lane];
+  int cnt = __popc(word);
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  int wbase = incl - cnt;
+  int U = __shfl_sync(0xffffffffu, incl, 31);
+  {
+    unsigned w2 = word;
+    int r = wbase;
+    while (w2) {
+      int b = __ffs(w2) - 1;
+      w2 &= w2 - 1u;
+      pl->ue[r] = lane * 32 + b;
+      pl->nt[r] = 0;
+      ++r;
+    }
+  }
+  __syncwarp();
+  // per pair: expert rank u and position among the expert's tokens (token order)
+  int pu[FD_MAXP / 32], ppos[FD_MAXP / 32];
+#pragma unroll
+  for (int i = 0; i < FD_MAXP / 32; ++i) {
+    int p = lane + 32 * i;
+    pu[i] = -1;
+    if (p < P) {
+      int e = pl->sidx[p];
+      int wi = e >> 5;
+      unsigned wbits = pl->bm[wi];
+      int base = 0;  // experts in the bitmap words before wi
+      for (int q = 0; q < wi; ++q) base += __popc(pl->bm[q]);
+      pu[i] = base + __popc(wbits & ((1u << (e & 31)) - 1u));
+      int t = p / a.k;
+      int pos = 0;
+      for (int t2 = 0; t2 < t; ++t2)
+        for (int j2 = 0; j2 < a.k; ++j2) pos += (pl->sidx[t2 * a.k + j2] == e) ? 1 : 0;
+      ppos[i] = pos;
+      atomicAdd(&pl->nt[pu[i]], 1);
+    }
+  }
+  __syncwarp();
+  if (lane == 0) {
+    int s = 0;
+    for (int u = 0; u < U; ++u) {
+      pl->pbase[u] = s;
+      s += pl->nt[u];
+    }
+    pl->pbase[U] = s;
+    pl->U = U;
+    pl->err = 0;
+    pl->abort = 0;
+  }
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < FD_MAXP / 32; ++i) {
+    int p = lane + 32 * i;
+    if (p < P) {
+      int q = pl->pbase[pu[i]] + ppos[i];
+      pl->ptok[q] = p / a.k;
+      pl->pslot[q] = p % a.k;
+      pl->pgate[q] = pl->sgate[p];
+    }
+  }
+  __syncwarp();
+}
+
+// Quantise activation vectors of 128-element chunks; task = vec * nch + chunk.
+// Each warp first issues the loads of up to MB tasks, then quantises them, so a
+// warp pays one memory latency per MB tasks.
+template <int MB, typename Load>
+__device__ __forceinline__ void quant_tasks(int ntask, int nch, int nblk, uint8_t *limbs, float2 *lsc, int warp,
+                                            int lane, Load load) {
+  for (int base = warp; base < ntask; base += MB * NCW) {
+    float4 v[MB];
+#pragma unroll
+    for (int i = 0; i < MB; ++i) {
+      const int task = base + i * NCW;
+      if (task < ntask) v[i] = load(task / nch, task % nch);
+    }
+#pragma unroll
+    for (int i = 0; i < MB; ++i) {
+      const int task = base + i * NCW;
+      if (task < ntask) {
+        const int vec = task / nch;
+        quant_chunk(v[i], limbs + (size_t)vec * nblk * 64, lsc + (size_t)vec * nblk, task % nch, lane);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + expf(-a)); }
+
+template <int BITS>
+__global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int S = a.nslots;
+  const SmemLayout lay = smem_layout(S, a.slot_bytes, a.limb_bytes, a.lsc_count);
+  uint8_t *ring = smem;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.bars);
+  uint64_t *empty = full + S;
+  Plan *pl = reinterpret_cast<Plan *>(smem + lay.plan);
+  uint8_t *limbs = smem + lay.limbs;
+  float2 *lsc = reinterpret_cast<float2 *>(smem + lay.lsc);
+
+  const int H = a.H, I = a.I, k = a.k;
+  const int nblkH = H / 32, nblkI = I / 32;
+  const int I16 = I / 16, H16 = H / 16;
+  const int tgu = tile_bytes(BITS, H), tdn = tile_bytes(BITS, I);
+  const unsigned G = gridDim.x;
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    fence_mbar_init();
+  }
+  // Everything above overlaps the previous kernel; idx, gate and x are its outputs.
+  pdl_wait();
+  if (warp == 0) build_plan(a, pl);
+  __syncthreads();
+  if (pl->err) return;
+
+  const int U = pl->U;
+  const int N1 = 2 * U * I16, N2 = U * H16;
+  const int lo1 = (int)((long long)blockIdx.x * N1 / G), hi1 = (int)((long long)(blockIdx.x + 1) * N1 / G);
+  const int lo2 = (int)((long long)blockIdx.x * N2 / G), hi2 = (int)((long long)(blockIdx.x + 1) * N2 / G);
+  const int n1 = hi1 - lo1, ntot = n1 + (hi2 - lo2);
+
+  if (warp == NCW) {
+    // ------------------------------------------------------------ producer --
+    // Every lane issues copies (item n by lane n % 32): one thread's bulk copies
+    // are serviced one after another, several issuers keep more bytes in flight.
+    int my_last = -1;
+    bool aborted = false;
+    for (int n = lane; n < ntot; n += 32) {
+      const int s = n % S, it = n / S;
+      if (n >= S) {
+        const long long dl = clock64() + WAIT_BUDGET_CYCLES;
+        while (!mbar_try_wait(&empty[s], (uint32_t)((it - 1) & 1))) {
+          if (*(volatile int *)&pl->abort || clock64() > dl) {
+            aborted = true;
+            break;
+          }
+        }
+        if (aborted) break;
+      }
+      const uint8_t *src;
+      uint32_t bytes;
+      if (n < n1) {
+        const int i = lo1 + n;
+        const int u = i / (2 * I16), m = (i / I16) & 1, r = i % I16;
+        src = a.gu + (((size_t)pl->ue[u] * 2 + m) * I16 + r) * (size_t)tgu;
+        bytes = (uint32_t)tgu;
+      } else {
+        const int i = lo2 + (n - n1);
+        const int u = i / H16, r = i % H16;
+        src = a.dn + ((size_t)pl->ue[u] * H16 + r) * (size_t)tdn;
+        bytes = (uint32_t)tdn;
+      }
+      mbar_arrive_expect_tx(&full[s], bytes);
+      bulk_g2s(ring + (size_t)s * a.slot_bytes, src, bytes, &full[s]);
+      my_last = n;
+    }
+    // never leave with copies in flight: wait for this lane's copies whose slot
+    // was not reused (reuse implies the copy was consumed)
+    const long long dl = clock64() + WAIT_BUDGET_CYCLES;
+    for (int n = lane; n <= my_last; n += 32) {
+      if (!aborted && n + S < ntot) continue;
+      while (!mbar_try_wait(&full[n % S], (uint32_t)((n / S) & 1)))
+        if (clock64() > dl) break;
+    }
+    pdl_launch_dependents();
+    return;
+  }
+
+  // ---------------------------------------------------------------- consumers --
+  const int nth = NCW * 32;
+  // activation limbs of the T tokens
+  {
+    const int nch = H / 128;
+    const float *x = a.x;
+    quant_tasks<16>(a.T * nch, nch, nblkH, limbs, lsc, warp, lane, [&](int t, int c) {
+      return __ldcg(reinterpret_cast<const float4 *>(x + (size_t)t * H + c * 128) + lane);
+    });
+  }
+  named_barrier_sync(CONSUMER_BAR, nth);
+
+  auto wait_full = [&](int n) -> bool {
+    if (*(volatile int *)&pl->abort) return false;
+    long long dl = clock64() + WAIT_BUDGET_CYCLES;
+    if (!mbar_wait(&full[n % S], (uint32_t)((n / S) & 1), dl)) {
+      set_status(a.status, DEV_TIMEOUT);
+      *(volatile int *)&pl->abort = 1;
+      return false;
+    }
+    return true;
+  };
+  auto release = [&](int n) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[n % S]);
+  };
+  const int g = lane >> 2, t = lane & 3;
+
+  // phase 1: gate / up
+  for (int n = warp; n < n1; n += NCW) {
+    if (!wait_full(n)) break;
+    const int i = lo1 + n;
+    const int u = i / (2 * I16), m = (i / I16) & 1, r = i % I16;
+    const uint8_t *tile = ring + (size_t)(n % S) * a.slot_bytes;
+    const int nu = pl->nt[u], pb = pl->pbase[u];
+    Acc acc;
+    const int np = dispatch_dot<BITS>(tile, nblkH, limbs, lsc, &pl->ptok[pb], nu, acc);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int tau = owner(np, t, q);
+      if (tau >= 0 && tau < nu) {
+        float *dst = a.abuf + ((size_t)(pb + tau) * 2 + m) * I + r * 16;
+        dst[g] = q ? acc.r0q1 : acc.r0q0;
+        dst[g + 8] = q ? acc.r1q1 : acc.r1q0;
+      }
+    }
+    release(n);
+  }
+
+  // grid barrier 1: every a_g / a_u is written
+  named_barrier_sync(CONSUMER_BAR, nth);
+  if (tid == 0) {
+    if (!*(volatile int *)&pl->abort && !grid_barrier_one_thread(a.bar, G)) {
+      set_status(a.status, DEV_TIMEOUT);
+      *(volatile int *)&pl->abort = 1;
+    }
+    __threadfence();
+  }
+  named_barrier_sync(CONSUMER_BAR, nth);
+  // all CTAs of this grid are resident now; the next kernel may start its prologue
+  pdl_launch_dependents();
+  bool ok = !*(volatile int *)&pl->abort;
+
+  // phase 2: down projection, one expert chunk at a time
+  const int hmaxp = a.limb_bytes / (I * 2);
+  int item = lo2;
+  while (ok && item < hi2) {
+    const int u0 = item / H16;
+    const int ulast = (hi2 - 1) / H16;
+    int u1 = u0, pairs = 0;
+    while (u1 <= ulast && pairs + pl->nt[u1] <= hmaxp) {
+      pairs += pl->nt[u1];
+      ++u1;
+    }
+    if (u1 == u0) {  // cannot happen: hmaxp >= FD_MAXT >= any expert's token count
+      set_status(a.status, DEV_BAD_INDEX);
+      *(volatile int *)&pl->abort = 1;
+      break;
+    }
+    const int pb0 = pl->pbase[u0];
+    {
+      const int nch = I / 128;
+      const float *abuf = a.abuf;
+      quant_tasks<8>(pairs * nch, nch, nblkI, limbs, lsc, warp, lane, [&](int lv, int c) {
+        const float *ab = abuf + (size_t)(pb0 + lv) * 2 * I + c * 128;
+        float4 gv = __ldcg(reinterpret_cast<const float4 *>(ab) + lane);
+        float4 uv = __ldcg(reinterpret_cast<const float4 *>(ab + I) + lane);
+        return make_float4(silu_f(gv.x) * uv.x, silu_f(gv.y) * uv.y, silu_f(gv.z) * uv.z, silu_f(gv.w) * uv.w);
+      });
+    }
+    named_barrier_sync(CONSUMER_BAR, nth);
+    const int item_end = min(hi2, u1 * H16);
+    for (int it2 = item; it2 < item_end; ++it2) {
+      const int n = n1 + (it2 - lo2);
+      if (n % NCW != warp) continue;
+      if (!wait_full(n)) break;
+      const int u = it2 / H16, r = it2 % H16;
+      const int nu = pl->nt[u], pb = pl->pbase[u];
+      int *vid = pl->vids[warp];
+      if (lane < FD_MAXT) vid[lane] = pb - pb0 + lane;
+      __syncwarp();
+      const uint8_t *tile = ring + (size_t)(n % S) * a.slot_bytes;
+      Acc acc;
+      const int np = dispatch_dot<BITS>(tile, nblkI, limbs, lsc, vid, nu, acc);
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int tau = owner(np, t, q);
+        if (tau >= 0 && tau < nu) {
+          const int p = pb + tau;
+          const float gw = pl->pgate[p];
+          float *dst = a.part + ((size_t)pl->ptok[p] * k + pl->pslot[p]) * H + r * 16;
+          dst[g] = gw * (q ? acc.r0q1 : acc.r0q0);
+          dst[g + 8] = gw * (q ? acc.r1q1 : acc.r1q0);
+        }
+      }
+      release(n);
+    }
+    named_barrier_sync(CONSUMER_BAR, nth);
+    ok = !*(volatile int *)&pl->abort;
+    item = item_end;
+  }
+
+  // grid barrier 2: every gated expert output is written
+  named_barrier_sync(CONSUMER_BAR, nth);
+  if (tid == 0) {
+    if (!*(volatile int *)&pl->abort && !grid_barrier_one_thread(a.bar, G)) {
+      set_status(a.status, DEV_TIMEOUT);
+      *(volatile int *)&pl->abort = 1;
+    }
+    __threadfence();
+  }
+  named_barrier_sync(CONSUMER_BAR, nth);
+  if (*(volatile int *)&pl->abort) return;
+
+  // phase 3: y[t] = sum_j part[t][j] in slot order
+  const int H4 = H / 4;
+  const float4 *p4 = reinterpret_cast<const float4 *>(a.part);
+  float4 *y4 = reinterpret_cast<float4 *>(a.y);
+  for (int o = blockIdx.x * nth + tid; o < a.T * H4; o += G * nth) {
+    const int tt = o / H4, h = o % H4;
+    float4 v[FD_MAXK];
+#pragma unroll
+    for (int j = 0; j < FD_MAXK; ++j)
+      if (j < k) v[j] = __ldcg(p4 + ((size_t)tt * k + j) * H4 + h);
+    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < FD_MAXK; ++j)
+      if (j < k) {
+        sum.x += v[j].x; sum.y += v[j].y; sum.z += v[j].z; sum.w += v[j].w;
+      }
+    y4[o] = sum;
+  }
+}
+
+size_t ws_bar_bytes() { return 256; }
+size_t ws_abuf_bytes(int T, int k, int I) { return (((size_t)T * k * 2 * I * 4) + 255) & ~(size_t)255; }
+size_t ws_part_bytes(int T, int k, int H) { return (((size_t)T * k * H * 4) + 255) & ~(size_t)255; }
+
+}  // namespace
+}  // namespace qmoe
+
+namespace qmoe {
+qmoe_status ffn_decode_launch(const qmoe_experts *ex, const float *x, int T, const int32_t *idx, const float *gate,
+                              int k, float *y, void *ws, size_t ws_bytes, int32_t *status, cudaStream_t s,
+                              bool cooperative);
+}
+
+using namespace qmoe;
+
+extern "C" size_t qmoe_decode_workspace_bytes(int T, int k, int H, int I) {
+  if (T < 1 || k < 1 || H < 1 || I < 1) return 0;
+  return ws_bar_bytes() + ws_abuf_bytes(T, k, I) + ws_part_bytes(T, k, H);
+}
+
+qmoe_status qmoe::ffn_decode_launch(const qmoe_experts *ex, const float *x, int T, const int32_t *idx,
+                                    const float *gate, int k, float *y, void *workspace, size_t workspace_bytes,
+                                    int32_t *dev_status, cudaStream_t stream, bool cooperative) {
+  if (!ex || !x || !idx || !gate || !y || !workspace || !dev_status) return QMOE_ERR_INVALID_ARG;
+  if (!ex->gate_up || !ex->down) return QMOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(workspace) || !aligned16(ex->gate_up) || !aligned16(ex->down) ||
+      (reinterpret_cast<uintptr_t>(idx) & 3) || (reinterpret_cast<uintptr_t>(gate) & 3))
+    return QMOE_ERR_INVALID_ARG;
+  if (ex->fmt != QMOE_Q2 && ex->fmt != QMOE_Q4) return QMOE_ERR_GEOMETRY;
+  if (ex->E < 1 || ex->H < 128 || ex->I < 128 || ex->H % 128 || ex->I % 128 || ex->E > 1024) return QMOE_ERR_GEOMETRY;
+  if (ex->gate_up_bytes != qmoe_packed_bytes(ex->fmt, QMOE_GATE_UP, ex->E, ex->H, ex->I) ||
+      ex->down_bytes != qmoe_packed_bytes(ex->fmt, QMOE_DOWN, ex->E, ex->H, ex->I))
+    return QMOE_ERR_GEOMETRY;
+  if (T < 1 || T > FD_MAXT || k < 1 || k > FD_MAXK || k > ex->E) return QMOE_ERR_UNSUPPORTED;
+  if (workspace_bytes < qmoe_decode_workspace_bytes(T, k, ex->H, ex->I)) return QMOE_ERR_WORKSPACE;
+
+  const int bits = ex->fmt, H = ex->H, I = ex->I;
+  FfnArgs a{};
+  a.gu = static_cast<const uint8_t *>(ex->gate_up);
+  a.dn = static_cast<const uint8_t *>(ex->down);
+  a.x = x;
+  a.idx = idx;
+  a.gate = gate;
+  a.y = y;
+  char *ws = static_cast<char *>(workspace);
+  a.bar = reinterpret_cast<unsigned *>(ws);
+  a.abuf = reinterpret_cast<float *>(ws + ws_bar_bytes());
+  a.part = reinterpret_cast<float *>(ws + ws_bar_bytes() + ws_abuf_bytes(T, k, I));
+  a.status = dev_status;
+  a.T = T; a.k = k; a.E = ex->E; a.H = H; a.I = I;
+
+  const int tgu = tile_bytes(bits, H), tdn = tile_bytes(bits, I);
+  a.slot_bytes = ((tgu > tdn ? tgu : tdn) + 127) & ~127;
+  int limb_x = T * H * 2, limb_h = FD_MAXT * I * 2;
+  a.limb_bytes = ((limb_x > limb_h ? limb_x : limb_h) + 127) & ~127;
+  int lsc_x = T * (H / 32), lsc_h = (a.limb_bytes / (I * 2)) * (I / 32);
+  a.lsc_count = lsc_x > lsc_h ? lsc_x : lsc_h;
+  size_t cap = max_smem_optin();
+  int S = 16;
+  while (S >= 2 && smem_layout(S, a.slot_bytes, a.limb_bytes, a.lsc_count).total > cap) --S;
+  if (S < 2) return QMOE_ERR_UNSUPPORTED;
+  a.nslots = S;
+  size_t smem = smem_layout(S, a.slot_bytes, a.limb_bytes, a.lsc_count).total;
+
+  const void *fn = (bits == 2) ? (const void *)ffn_decode_kernel<2> : (const void *)ffn_decode_kernel<4>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return QMOE_ERR_CUDA;
+
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)num_sms());
+  cfg.blockDim = dim3(FD_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  // One CTA per SM (shared memory caps residency at one) and a grid of exactly
+  // the SM count, so every CTA is resident for the grid barriers; the
+  // programmatic-serialization attribute lets this grid launch while the
+  // previous kernel drains (the kernel waits for it before reading inputs).
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (cooperative) {
+    attr[na].id = cudaLaunchAttributeCooperative;
+    attr[na].val.cooperative = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  if (bits == 2)
+    e = cudaLaunchKernelEx(&cfg, ffn_decode_kernel<2>, a);
+  else
+    e = cudaLaunchKernelEx(&cfg, ffn_decode_kernel<4>, a);
+  note_launch();
+  return cuda_status(e);
+}
+
+extern "C" qmoe_status qmoe_ffn_decode(const qmoe_experts *ex, const float *x, int T, const int32_t *idx,
+                                       const float *gate, int k, float *y, void *workspace, size_t workspace_bytes,
+                                       int32_t *dev_status, qmoe_stream_t stream) {
+  return qmoe::ffn_decode_launch(ex, x, T, idx, gate, k, y, workspace, workspace_bytes, dev_status,
+                                 (cudaStream_t)stream, false);
+}

@@ -1,0 +1,141 @@
+// Warp-level top-k selection with renormalised gates over one token's float64
+// logits (used by the decode and prefill routers).
+//
+// Selection order: logit descending, expert index ascending on equal logits.
+// 1. Every logit gets an fp32 key (round-to-nearest of the float64 value, made
+//    order-preserving as an unsigned integer). Rounding is monotone, so the
+//    k largest float64 logits are among the k largest keys, counted with
+//    multiplicity.
+// 2. Rounds of warp max-reductions remove the largest remaining key (all its
+//    copies) until at least k keys are removed; the last removed key is the
+//    threshold and every key >= threshold is a candidate.
+// 3. Candidates are ranked exactly on their float64 logits (index breaks
+//    ties). Ranks below k give the slots.
+// 4. gate_j = exp(l_j - l_0) / sum_j' exp(l_j' - l_0) over the selected slots.
+#pragma once
+
+#include "common.cuh"
+
+namespace qmoe {
+
+constexpr int TOPK_MAX_K = 16;
+constexpr int TOPK_CAND = 64;
+
+struct TopkScratch {
+  int cand[TOPK_CAND];
+  double cand_v[TOPK_CAND];
+  int sel_e[TOPK_MAX_K];
+  double sel_v[TOPK_MAX_K];
+};
+
+__device__ __forceinline__ bool ranks_above(double va, int ea, double vb, int eb) {
+  return va > vb || (va == vb && ea < eb);
+}
+
+// One warp; `l` is the token's logits [E] in global memory (written by other
+// CTAs before a fence, read through L2). M = values per lane = ceil(E / 32).
+template <int M>
+__device__ inline void warp_topk_gates_m(const double *l, int E, int k, int32_t *idx_out, float *gate_out,
+                                         TopkScratch *sc) {
+  const int lane = threadIdx.x & 31;
+  double val[M];
+  unsigned key[M], rem[M];
+#pragma unroll
+  for (int j = 0; j < M; ++j) {
+    const int e = lane + 32 * j;
+    val[j] = e < E ? __ldcg(l + e) : 0.0;
+  }
+#pragma unroll
+  for (int j = 0; j < M; ++j) {
+    const int e = lane + 32 * j;
+    key[j] = e < E ? float_key(__double2float_rn(val[j])) : 0u;
+    rem[j] = key[j];
+  }
+  unsigned thr = 0;
+  int removed = 0;
+  while (removed < k) {
+    unsigned local = 0;
+#pragma unroll
+    for (int j = 0; j < M; ++j) local = max(local, rem[j]);
+    const unsigned mx = __reduce_max_sync(0xffffffffu, local);
+    if (mx == 0u) break;
+    int c = 0;
+#pragma unroll
+    for (int j = 0; j < M; ++j) {
+      if (rem[j] == mx) {
+        rem[j] = 0u;
+        ++c;
+      }
+    }
+    removed += (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
+    thr = mx;
+  }
+  // candidates: keys >= thr
+  int mine = 0;
+#pragma unroll
+  for (int j = 0; j < M; ++j) mine += (key[j] != 0u && key[j] >= thr) ? 1 : 0;
+  int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  if (total <= TOPK_CAND) {
+    int pos = incl - mine;
+#pragma unroll
+    for (int j = 0; j < M; ++j)
+      if (key[j] != 0u && key[j] >= thr) {
+        sc->cand[pos] = lane + 32 * j;
+        sc->cand_v[pos] = val[j];
+        ++pos;
+      }
+    __syncwarp();
+    for (int i = lane; i < total; i += 32) {
+      const int e = sc->cand[i];
+      const double v = sc->cand_v[i];
+      int rank = 0;
+      for (int i2 = 0; i2 < total; ++i2) rank += ranks_above(sc->cand_v[i2], sc->cand[i2], v, e) ? 1 : 0;
+      if (rank < k) {
+        sc->sel_e[rank] = e;
+        sc->sel_v[rank] = v;
+      }
+    }
+  } else {
+    // many equal fp32 keys (degenerate router): rank the candidates against all logits
+#pragma unroll
+    for (int j = 0; j < M; ++j) {
+      if (key[j] != 0u && key[j] >= thr) {
+        const int e = lane + 32 * j;
+        const double v = val[j];
+        int rank = 0;
+        for (int e2 = 0; e2 < E && rank < k; ++e2) rank += ranks_above(__ldcg(l + e2), e2, v, e) ? 1 : 0;
+        if (rank < k) {
+          sc->sel_e[rank] = e;
+          sc->sel_v[rank] = v;
+        }
+      }
+    }
+  }
+  __syncwarp();
+  float ex = 0.0f;
+  if (lane < k) ex = expf((float)(sc->sel_v[lane] - sc->sel_v[0]));
+  const float sum = warp_sum(ex);
+  if (lane < k) {
+    idx_out[lane] = sc->sel_e[lane];
+    gate_out[lane] = ex / sum;
+  }
+  __syncwarp();
+}
+
+__device__ inline void warp_topk_gates(const double *l, int E, int k, int32_t *idx_out, float *gate_out,
+                                       TopkScratch *sc) {
+  if (E <= 32) warp_topk_gates_m<1>(l, E, k, idx_out, gate_out, sc);
+  else if (E <= 64) warp_topk_gates_m<2>(l, E, k, idx_out, gate_out, sc);
+  else if (E <= 128) warp_topk_gates_m<4>(l, E, k, idx_out, gate_out, sc);
+  else if (E <= 256) warp_topk_gates_m<8>(l, E, k, idx_out, gate_out, sc);
+  else if (E <= 512) warp_topk_gates_m<16>(l, E, k, idx_out, gate_out, sc);
+  else warp_topk_gates_m<32>(l, E, k, idx_out, gate_out, sc);
+}
+
+}  // namespace qmoe

@@ -1,0 +1,246 @@
+// Layer stack: L x (route -> decode FFN) + residual RMSNorm, captured once into
+// one CUDA graph whose arguments are fixed-address buffers in caller workspace.
+#include <new>
+#include <vector>
+
+#include "common.cuh"
+
+namespace qmoe {
+qmoe_status ffn_decode_launch(const qmoe_experts *ex, const float *x, int T, const int32_t *idx, const float *gate,
+                              int k, float *y, void *ws, size_t ws_bytes, int32_t *status, cudaStream_t s,
+                              bool cooperative);
+}
+
+struct qmoe_stack {
+  int L, T, k, E, H, I, fmt;
+  float eps;
+  std::vector<const float *> Wr, bias;
+  std::vector<qmoe_experts> layers;
+  float *x_in, *x_out, *xa, *xb, *y;
+  int32_t *idx;
+  float *gate;
+  int32_t *status;
+  void *route_ws;
+  size_t route_ws_bytes;
+  void *ffn_ws;
+  size_t ffn_ws_bytes;
+  cudaGraph_t graph;
+  cudaGraphExec_t exec;
+  int kernels;
+  int flags;
+  std::vector<cudaEvent_t> events;  // 2L + 1 when timing
+};
+
+namespace {
+
+size_t al(size_t b) { return (b + 255) & ~(size_t)255; }
+
+struct Layout {
+  size_t x, idx, gate, status, route, ffn, total;
+};
+
+Layout layout_of(const qmoe_stack_desc *d) {
+  const qmoe_experts &e = d->layers[0];
+  Layout l;
+  l.x = al((size_t)d->T * e.H * 4);
+  l.idx = al((size_t)d->L * d->T * d->k * 4);
+  l.gate = l.idx;
+  l.status = 256;
+  l.route = al(qmoe_route_workspace_bytes(d->T, e.E));
+  l.ffn = al(qmoe_decode_workspace_bytes(d->T, d->k, e.H, e.I));
+  l.total = 5 * l.x + l.idx + l.gate + l.status + l.route + l.ffn;
+  return l;
+}
+
+qmoe_status check_desc(const qmoe_stack_desc *d) {
+  if (!d || d->L < 1 || d->T < 1 || d->T > 8 || d->k < 1 || !d->Wr || !d->layers) return QMOE_ERR_INVALID_ARG;
+  if (!(d->eps >= 0.0f)) return QMOE_ERR_INVALID_ARG;
+  const qmoe_experts &e0 = d->layers[0];
+  for (int l = 0; l < d->L; ++l) {
+    const qmoe_experts &e = d->layers[l];
+    if (e.E != e0.E || e.H != e0.H || e.I != e0.I || e.fmt != e0.fmt) return QMOE_ERR_GEOMETRY;
+    if (e.gate_up_bytes != qmoe_packed_bytes(e.fmt, QMOE_GATE_UP, e.E, e.H, e.I) ||
+        e.down_bytes != qmoe_packed_bytes(e.fmt, QMOE_DOWN, e.E, e.H, e.I))
+      return QMOE_ERR_GEOMETRY;
+    if (!e.gate_up || !e.down || !d->Wr[l]) return QMOE_ERR_INVALID_ARG;
+  }
+  return QMOE_OK;
+}
+
+qmoe_status record(qmoe_stack *s, cudaStream_t cs, bool coop) {
+  qmoe_status st;
+  const float *x_prev = s->x_in;
+  const bool timing = !s->events.empty();
+  if (timing && cudaEventRecordWithFlags(s->events[0], cs, cudaEventRecordExternal) != cudaSuccess) return QMOE_ERR_CUDA;
+  for (int l = 0; l < s->L; ++l) {
+    int32_t *idx = s->idx + (size_t)l * s->T * s->k;
+    float *gate = s->gate + (size_t)l * s->T * s->k;
+    const float *bias = s->bias[l];
+    const float *x_cur;
+    if (l == 0) {
+      st = qmoe_route(s->Wr[l], bias, s->x_in, QMOE_F32, s->T, s->H, s->E, s->k, idx, gate, s->route_ws,
+                      s->route_ws_bytes, s->status, (qmoe_stream_t)cs);
+      x_cur = s->x_in;
+    } else {
+      float *xo = (l & 1) ? s->xa : s->xb;
+      st = qmoe_residual_route(x_prev, s->y, s->eps, xo, s->Wr[l], bias, s->T, s->H, s->E, s->k, idx, gate,
+                               s->route_ws, s->route_ws_bytes, s->status, (qmoe_stream_t)cs);
+      x_cur = xo;
+    }
+    if (st != QMOE_OK) return st;
+    if (timing && cudaEventRecordWithFlags(s->events[2 * l + 1], cs, cudaEventRecordExternal) != cudaSuccess) return QMOE_ERR_CUDA;
+    st = qmoe::ffn_decode_launch(&s->layers[l], x_cur, s->T, idx, gate, s->k, s->y, s->ffn_ws, s->ffn_ws_bytes,
+                                 s->status, cs, coop);
+    if (st != QMOE_OK) return st;
+    if (timing && cudaEventRecordWithFlags(s->events[2 * l + 2], cs, cudaEventRecordExternal) != cudaSuccess) return QMOE_ERR_CUDA;
+    x_prev = x_cur;
+  }
+  st = qmoe_rmsnorm_residual(x_prev, s->y, s->eps, s->x_out, s->T, s->H, (qmoe_stream_t)cs);
+  s->kernels = 2 * s->L + 1;
+  return st;
+}
+
+qmoe_status capture(qmoe_stack *s, bool coop) {
+  cudaStream_t cs;
+  if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return QMOE_ERR_CUDA;
+  qmoe_status st = QMOE_OK;
+  cudaGraph_t g = nullptr;
+  if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    cudaStreamDestroy(cs);
+    return QMOE_ERR_CUDA;
+  }
+  qmoe_status rs = record(s, cs, coop);
+  cudaError_t e = cudaStreamEndCapture(cs, &g);
+  if (rs != QMOE_OK) st = rs;
+  else if (e != cudaSuccess) st = QMOE_ERR_CUDA;
+  cudaGraphExec_t ex = nullptr;
+  if (st == QMOE_OK && cudaGraphInstantiate(&ex, g, 0) != cudaSuccess) st = QMOE_ERR_CUDA;
+  if (st == QMOE_OK) {
+    s->graph = g;
+    s->exec = ex;
+  } else {
+    if (g) cudaGraphDestroy(g);
+    cudaGetLastError();
+  }
+  cudaStreamDestroy(cs);
+  return st;
+}
+
+}  // namespace
+
+extern "C" size_t qmoe_stack_workspace_bytes(const qmoe_stack_desc *d) {
+  if (check_desc(d) != QMOE_OK) return 0;
+  return layout_of(d).total;
+}
+
+extern "C" qmoe_status qmoe_stack_create(const qmoe_stack_desc *d, void *workspace, size_t workspace_bytes,
+                                         qmoe_stream_t stream, qmoe_stack **out) {
+  if (!out) return QMOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  qmoe_status st = check_desc(d);
+  if (st != QMOE_OK) return st;
+  if (!workspace || !qmoe::aligned16(workspace)) return QMOE_ERR_INVALID_ARG;
+  Layout lo = layout_of(d);
+  if (workspace_bytes < lo.total) return QMOE_ERR_WORKSPACE;
+  qmoe_stack *s = new (std::nothrow) qmoe_stack();
+  if (!s) return QMOE_ERR_CUDA;
+  const qmoe_experts &e0 = d->layers[0];
+  s->L = d->L; s->T = d->T; s->k = d->k; s->E = e0.E; s->H = e0.H; s->I = e0.I; s->fmt = e0.fmt;
+  s->eps = d->eps;
+  s->Wr.assign(d->Wr, d->Wr + d->L);
+  s->bias.assign(d->L, nullptr);
+  if (d->bias)
+    for (int l = 0; l < d->L; ++l) s->bias[l] = d->bias[l];
+  s->layers.assign(d->layers, d->layers + d->L);
+  s->flags = d->flags;
+  if (d->flags & QMOE_STACK_TIMING) {
+    s->events.assign(2 * d->L + 1, nullptr);
+    for (auto &e : s->events)
+      if (cudaEventCreate(&e) != cudaSuccess) {
+        for (auto &e2 : s->events)
+          if (e2) cudaEventDestroy(e2);
+        delete s;
+        return QMOE_ERR_CUDA;
+      }
+  }
+  char *p = static_cast<char *>(workspace);
+  s->x_in = reinterpret_cast<float *>(p); p += lo.x;
+  s->x_out = reinterpret_cast<float *>(p); p += lo.x;
+  s->xa = reinterpret_cast<float *>(p); p += lo.x;
+  s->xb = reinterpret_cast<float *>(p); p += lo.x;
+  s->y = reinterpret_cast<float *>(p); p += lo.x;
+  s->idx = reinterpret_cast<int32_t *>(p); p += lo.idx;
+  s->gate = reinterpret_cast<float *>(p); p += lo.gate;
+  s->status = reinterpret_cast<int32_t *>(p); p += lo.status;
+  s->route_ws = p; s->route_ws_bytes = lo.route; p += lo.route;
+  s->ffn_ws = p; s->ffn_ws_bytes = lo.ffn;
+  if (cudaMemsetAsync(workspace, 0, lo.total, (cudaStream_t)stream) != cudaSuccess ||
+      cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) {
+    delete s;
+    return QMOE_ERR_CUDA;
+  }
+  st = capture(s, false);
+  if (st != QMOE_OK) {
+    for (auto &e : s->events) cudaEventDestroy(e);
+    delete s;
+    return st;
+  }
+  *out = s;
+  return QMOE_OK;
+}
+
+extern "C" qmoe_status qmoe_stack_destroy(qmoe_stack *s) {
+  if (!s) return QMOE_ERR_INVALID_ARG;
+  if (s->exec) cudaGraphExecDestroy(s->exec);
+  if (s->graph) cudaGraphDestroy(s->graph);
+  for (auto &e : s->events) cudaEventDestroy(e);
+  delete s;
+  return QMOE_OK;
+}
+
+extern "C" qmoe_status qmoe_stack_buffers(const qmoe_stack *s, float **x_in, float **x_out, int32_t **idx,
+                                          float **gate, int32_t **dev_status) {
+  if (!s) return QMOE_ERR_INVALID_ARG;
+  if (x_in) *x_in = s->x_in;
+  if (x_out) *x_out = s->x_out;
+  if (idx) *idx = s->idx;
+  if (gate) *gate = s->gate;
+  if (dev_status) *dev_status = s->status;
+  return QMOE_OK;
+}
+
+extern "C" int qmoe_stack_kernels_per_replay(const qmoe_stack *s) { return s ? s->kernels : 0; }
+
+extern "C" qmoe_status qmoe_stack_decode(qmoe_stack *s, qmoe_stream_t stream) {
+  if (!s || !s->exec) return QMOE_ERR_INVALID_ARG;
+  cudaError_t e = cudaGraphLaunch(s->exec, (cudaStream_t)stream);
+  qmoe::note_launch(s->kernels);
+  return qmoe::cuda_status(e);
+}
+
+extern "C" qmoe_status qmoe_stack_decode_host(qmoe_stack *s, const float *x_host, float *x_out_host,
+                                              qmoe_stream_t stream) {
+  if (!s || !s->exec || !x_host || !x_out_host) return QMOE_ERR_INVALID_ARG;
+  size_t bytes = (size_t)s->T * s->H * sizeof(float);
+  cudaStream_t cs = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(s->x_in, x_host, bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess) return QMOE_ERR_CUDA;
+  if (cudaGraphLaunch(s->exec, cs) != cudaSuccess) return QMOE_ERR_CUDA;
+  qmoe::note_launch(s->kernels);
+  if (cudaMemcpyAsync(x_out_host, s->x_out, bytes, cudaMemcpyDeviceToHost, cs) != cudaSuccess) return QMOE_ERR_CUDA;
+  return QMOE_OK;
+}
+
+extern "C" qmoe_status qmoe_stack_layer_times(const qmoe_stack *s, float *route_ms, float *ffn_ms) {
+  if (!s) return QMOE_ERR_INVALID_ARG;
+  if (s->events.empty()) return QMOE_ERR_UNSUPPORTED;
+  if (cudaEventSynchronize(s->events.back()) != cudaSuccess) return QMOE_ERR_CUDA;
+  for (int l = 0; l < s->L; ++l) {
+    float a = 0.f, b = 0.f;
+    if (cudaEventElapsedTime(&a, s->events[2 * l], s->events[2 * l + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&b, s->events[2 * l + 1], s->events[2 * l + 2]) != cudaSuccess)
+      return QMOE_ERR_CUDA;
+    if (route_ms) route_ms[l] = a;
+    if (ffn_ms) ffn_ms[l] = b;
+  }
+  return QMOE_OK;
+}

@@ -1,0 +1,101 @@
+"""GPU parity of the captured layer stack (route -> FFN -> residual RMSNorm per
+layer, one CUDA graph) against the float64 oracle run free from the same x_0."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe
+from oracle import workload as W
+from quantised_expert_decode_b200.model import DecodeStack
+from synth import configs, gen
+from synth.workload import device_layers
+from tests.gpu_util import DECODE_TOL, GATE_TOL, gap_report, to_np
+
+pytestmark = pytest.mark.gpu
+SEED = 0
+
+
+# Beyond the first layer the GPU and the oracle route slightly different
+# activations (fp32 vs float64 arithmetic, 16-bit activation limbs), so two
+# logits closer than this may legitimately order differently. A differing
+# expert SET is accepted only as a reported near-tie below this gap.
+NEAR_TIE = 1e-4
+
+
+def _compare(cfg, stack, x0_np, n_layers):
+    xo, recs = W.run_stack(SEED, cfg, x0_np.astype(np.float64), n_layers)
+    idx = to_np(stack.idx)
+    gate = to_np(stack.gate)
+    for l, (x_in, oi, og, _) in enumerate(recs):
+        if np.array_equal(idx[l], oi):
+            assert np.max(np.abs(gate[l] - og)) < 50 * GATE_TOL, l
+            continue
+        L_ = W.Layer(SEED, cfg, l)
+        lg = moe.logits(x_in, L_.Wr, L_.bias, cfg.k)
+        for t in range(cfg.T):
+            if set(idx[l, t].tolist()) != set(oi[t].tolist()):
+                gap = gap_report(lg[t], cfg.k)
+                if gap < NEAR_TIE:
+                    pytest.xfail(f"layer {l} token {t}: near-tie route flip, oracle top-k gap {gap:.3g}")
+                pytest.fail(f"layer {l} token {t}: expert sets differ; oracle top-k gap {gap:.3g}")
+            for a, b in zip(idx[l, t], oi[t]):
+                if a != b:
+                    assert abs(lg[t, a] - lg[t, b]) < NEAR_TIE, (l, t, a, b)
+            gm = dict(zip(idx[l, t].tolist(), gate[l, t].tolist()))
+            for e, gv in zip(oi[t].tolist(), og[t].tolist()):
+                assert abs(gm[e] - gv) < 50 * GATE_TOL, (l, t, e)
+    err = moe.rel_rms(to_np(stack.x_out), xo)
+    assert err < DECODE_TOL, err
+    return err
+
+
+def _run(cfg, n_layers, step=0):
+    layers, routers, biases = device_layers(SEED, cfg, n_layers)
+    stack = DecodeStack(layers, routers, biases, cfg.T, cfg.k, cfg.eps)
+    x0 = gen.tokens(SEED, cfg, step)
+    stack.x_in.copy_(torch.from_numpy(x0))
+    stack.decode()
+    torch.cuda.synchronize()
+    assert stack.status() == 0
+    return stack, x0, layers
+
+
+def test_stack_small_geometry():
+    cfg = configs.get(0).with_(L=6, residual=True)
+    stack, x0, _ = _run(cfg, 6)
+    _compare(cfg, stack, x0, 6)
+    assert stack.kernels_per_replay == 13
+    # host-buffer entry point gives the same answer as the device-buffer replay
+    xh = torch.from_numpy(x0).pin_memory()
+    out = torch.empty_like(xh).pin_memory()
+    ref = stack.x_out.clone()
+    stack.decode_host(xh, out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref.cpu())
+    stack.close()
+
+
+def test_stack_48_layers_q2_single_token():
+    cfg = configs.get(2)
+    stack, x0, layers = _run(cfg, cfg.L)
+    assert sum(l.nbytes for l in layers) == cfg.L * cfg.E * cfg.expert_bytes()
+    _compare(cfg, stack, x0, cfg.L)
+    # replays are deterministic
+    first = stack.x_out.clone()
+    stack.decode()
+    torch.cuda.synchronize()
+    assert torch.equal(first, stack.x_out)
+    # a second token through the same graph
+    x1 = gen.tokens(SEED, cfg, 1)
+    stack.x_in.copy_(torch.from_numpy(x1))
+    stack.decode()
+    torch.cuda.synchronize()
+    _compare(cfg, stack, x1, cfg.L)
+    stack.close()
+
+
+def test_stack_48_layers_q4_verify_batch():
+    cfg = configs.get(3)
+    stack, x0, _ = _run(cfg, cfg.L)
+    _compare(cfg, stack, x0, cfg.L)
+    stack.close()
