@@ -1,0 +1,243 @@
+// Decode tile primitives shared by the per-layer FFN kernel and the fused
+// layer-stack kernel: activation quantisation into int8 limbs and the integer
+// tensor-core dot product of one packed 16-row weight tile.
+//
+// Contraction: activations of every 32-element block are quantised to 24-bit
+// fixed point with a per-block fp32 scale s (X = rint(v / s), |X| <= 8355711)
+// and split into three signed 8-bit limbs X = 65536*l2 + 256*l1 + l0. The
+// integer MMA m16n8k32 (u8 codes x s8 limbs, s32 accumulate) gives the exact
+// sums Q_i = sum q*l_i per block; the block's contribution is
+// d * s * (65536*Q2 + 256*Q1 + Q0) + m * s * sum(X). A (token, block) pair
+// occupies four MMA columns (l2, l1, 0, l0): lane 2P reads (l2, l1) and lane
+// 2P+1 reads (0, l0), so each lane finishes its share in fp32 on its own and
+// two pairs share one accumulator tile.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "layout.cuh"
+
+namespace qmoe {
+namespace tile {
+namespace {  // internal linkage: each translation unit keeps its own copy
+
+constexpr float QMAX = 8355711.0f;         // 127*65536 + 127*256 + 127: three int8 limbs
+constexpr int LIMB_REC = 96;               // bytes per (vector, block): l2 | l1 | l0
+
+__device__ __forceinline__ float h2f(uint32_t bits16) { return __half2float(__ushort_as_half((unsigned short)bits16)); }
+
+// Quantise a 128-element chunk (4 blocks of 32) held one float4 per lane: lane
+// j carries elements 4j..4j+3, i.e. block j/8. Writes the three int8 limbs of
+// the four blocks and (s, s * sum X) per block. The block's min term uses the
+// same quantised values as its code term, so the whole block sees one
+// consistent activation s*X and the only error is that of quantising v.
+__device__ __forceinline__ int quant_one(float v, float inv) {
+  const int X = __float2int_rn(v * inv);
+  return max(-8355711, min(8355711, X));
+}
+
+// balanced base-256 digits of |X| <= 8355711, each in [-128, 127]
+__device__ __forceinline__ void limbs3(int X, int &l2, int &l1, int &l0) {
+  l0 = ((X + 128) & 255) - 128;
+  const int X1 = (X - l0) >> 8;
+  l1 = ((X1 + 128) & 255) - 128;
+  l2 = (X1 - l1) >> 8;
+}
+
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
+  return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8) | ((uint32_t)(c & 0xff) << 16) |
+         ((uint32_t)(d & 0xff) << 24);
+}
+
+__device__ __noinline__ void quant_chunk(float4 v, uint8_t *limbs_vec, float2 *lsc_vec, int chunk, int lane) {
+  float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
+  float s = 0.0f, inv = 0.0f;
+  if (a > 0.0f) {
+    s = a / QMAX;
+    inv = QMAX / a;
+  }
+  const int X0 = quant_one(v.x, inv), X1 = quant_one(v.y, inv), X2 = quant_one(v.z, inv), X3 = quant_one(v.w, inv);
+  int a2, a1, a0, b2, b1, b0, c2, c1, c0, d2, d1, d0;
+  limbs3(X0, a2, a1, a0);
+  limbs3(X1, b2, b1, b0);
+  limbs3(X2, c2, c1, c0);
+  limbs3(X3, d2, d1, d0);
+  const int blk = chunk * 4 + (lane >> 3);
+  uint8_t *rec = limbs_vec + (size_t)blk * LIMB_REC + (lane & 7) * 4;
+  *reinterpret_cast<uint32_t *>(rec) = pack4(a2, b2, c2, d2);
+  *reinterpret_cast<uint32_t *>(rec + 32) = pack4(a1, b1, c1, d1);
+  *reinterpret_cast<uint32_t *>(rec + 64) = pack4(a0, b0, c0, d0);
+  int sx = X0 + X1 + X2 + X3;                  // |sum over the block| < 2^31
+  sx += __shfl_xor_sync(0xffffffffu, sx, 1);
+  sx += __shfl_xor_sync(0xffffffffu, sx, 2);
+  sx += __shfl_xor_sync(0xffffffffu, sx, 4);
+  if ((lane & 7) == 0) lsc_vec[blk] = make_float2(s, s * (float)sx);
+}
+
+struct Acc {
+  float r0[4], r1[4];  // rows g / g+8 x column groups q
+};
+
+// Dot products of one 16-row tile (K = 32 * nblk, nblk % 4 == 0) with n <= NP
+// activation vectors (vector ids vid[0..n)). Returns the lane's share; see the
+// file header for the column layout. Not inlined: phase 1 and phase 2 share one
+// copy of the code, which keeps the instruction footprint small.
+//   NP = 1: one accumulator tile holds 2 blocks of the token (2 tiles per chunk)
+//   NP >= 2: one tile holds 2 tokens of one block; NQ = NP/2 tiles per block
+template <int BITS, int NP>
+__device__ __noinline__ Acc tile_dot(const uint8_t *tile, int nblk, const uint8_t *limbs, const float2 *lsc,
+                                     const int *vid, int n) {
+  constexpr int TS = NP == 1 ? 1 : 2;     // tokens per accumulator tile
+  constexpr int BS = 2 / TS;              // blocks per accumulator tile
+  constexpr int NQ = NP == 1 ? 1 : NP / 2;
+  constexpr int NSET = 4 / BS;            // tiles per 4-block chunk and column group
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  // B columns this lane provides: column g -> pair g>>2, limb slot g&3 (l2, l1, zero, l0)
+  const int pP = g >> 2, pslot = g & 3;
+  const int ploff = pslot == 0 ? 0 : (pslot == 1 ? 32 : 64);
+  // D columns this lane reads: (2t, 2t+1) -> pair t>>1, half t&1
+  const int oP = t >> 1, ohalf = t & 1;
+  const float wgt = ohalf ? 1.0f : 256.0f;
+  const uint8_t *sbase = tile + 64 * nblk * BITS;   // scales follow the codes
+  float acc[2][NQ];
+  int pv[NQ], ov[NQ];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    acc[0][q] = acc[1][q] = 0.0f;
+    const int ptq = (NP == 1) ? 0 : 2 * q + pP;
+    const int otq = (NP == 1) ? 0 : 2 * q + oP;
+    pv[q] = (ptq < n && pslot != 2) ? vid[ptq] : -1;
+    ov[q] = otq < n ? vid[otq] : -1;
+  }
+  const int pbeta = (NP == 1) ? pP : 0;
+  const int obeta = (NP == 1) ? oP : 0;
+
+#pragma unroll 1
+  for (int c = 0; c < (nblk >> 2); ++c) {
+    uint32_t w[8];
+    if (BITS == 2) {
+      const uint4 q = *reinterpret_cast<const uint4 *>(tile + c * 512 + lane * 16);
+      w[0] = q.x; w[1] = q.y; w[2] = q.z; w[3] = q.w;
+    } else {
+      const uint4 q0 = *reinterpret_cast<const uint4 *>(tile + (2 * c) * 512 + lane * 16);
+      const uint4 q1 = *reinterpret_cast<const uint4 *>(tile + (2 * c + 1) * 512 + lane * 16);
+      w[0] = q0.x; w[1] = q0.y; w[2] = q0.z; w[3] = q0.w;
+      w[4] = q1.x; w[5] = q1.y; w[6] = q1.z; w[7] = q1.w;
+    }
+#pragma unroll
+    for (int sb = 0; sb < NSET; ++sb) {
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        uint32_t b0 = 0u, b1 = 0u;
+        if (pv[q] >= 0) {
+          const int blk = c * 4 + sb * BS + pbeta;
+          const uint8_t *lp = limbs + ((size_t)pv[q] * nblk + blk) * LIMB_REC + ploff + 4 * t;
+          b0 = *reinterpret_cast<const uint32_t *>(lp);
+          b1 = *reinterpret_cast<const uint32_t *>(lp + 16);
+        }
+        int d0 = 0, d1 = 0, d2 = 0, d3 = 0;
+#pragma unroll
+        for (int beta = 0; beta < BS; ++beta) {
+          const int bb = sb * BS + beta;
+          uint32_t a0, a1, a2, a3;
+          if (BITS == 2) {
+            const uint32_t x = w[bb];
+            a0 = x & 0x03030303u;
+            a1 = (x >> 2) & 0x03030303u;
+            a2 = (x >> 4) & 0x03030303u;
+            a3 = (x >> 6) & 0x03030303u;
+          } else {
+            const uint32_t x0 = w[2 * bb], x1 = w[2 * bb + 1];
+            a0 = x0 & 0x0F0F0F0Fu;
+            a1 = (x0 >> 4) & 0x0F0F0F0Fu;
+            a2 = x1 & 0x0F0F0F0Fu;
+            a3 = (x1 >> 4) & 0x0F0F0F0Fu;
+          }
+          const bool on = (pbeta == beta);
+          mma_u8s8(d0, d1, d2, d3, a0, a1, a2, a3, on ? b0 : 0u, on ? b1 : 0u);
+        }
+        if (ov[q] >= 0) {
+          const int bo = c * 4 + sb * BS + obeta;
+          const float v0 = (float)(d0 * 256 + d1);
+          const float v1 = (float)(d2 * 256 + d3);
+          const float2 ss = lsc[(size_t)ov[q] * nblk + bo];
+          const uint2 dm = *reinterpret_cast<const uint2 *>(sbase + (bo * 8 + g) * 8);
+          const float sw = ss.x * wgt;
+          const float mt = ohalf ? 0.0f : ss.y;    // the min term once per pair
+          acc[0][q] = fmaf(h2f(dm.x & 0xffffu), sw * v0, fmaf(h2f(dm.x >> 16), mt, acc[0][q]));
+          acc[1][q] = fmaf(h2f(dm.y & 0xffffu), sw * v1, fmaf(h2f(dm.y >> 16), mt, acc[1][q]));
+        }
+      }
+    }
+  }
+  // combine the lanes that share a token: the two halves of a pair, and for
+  // NP == 1 also the two pairs (two blocks of the same token)
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      acc[r][q] += __shfl_xor_sync(0xffffffffu, acc[r][q], 1);
+      if (NP == 1) acc[r][q] += __shfl_xor_sync(0xffffffffu, acc[r][q], 2);
+    }
+  }
+  Acc out;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    out.r0[q] = q < NQ ? acc[0][q < NQ ? q : 0] : 0.0f;
+    out.r1[q] = q < NQ ? acc[1][q < NQ ? q : 0] : 0.0f;
+  }
+  return out;
+}
+
+template <int BITS>
+__device__ __forceinline__ int dispatch_dot(const uint8_t *tile, int nblk, const uint8_t *limbs, const float2 *lsc,
+                                            const int *vid, int n, Acc &acc) {
+  if (n <= 1) { acc = tile_dot<BITS, 1>(tile, nblk, limbs, lsc, vid, n); return 1; }
+  if (n <= 2) { acc = tile_dot<BITS, 2>(tile, nblk, limbs, lsc, vid, n); return 2; }
+  if (n <= 4) { acc = tile_dot<BITS, 4>(tile, nblk, limbs, lsc, vid, n); return 4; }
+  acc = tile_dot<BITS, 8>(tile, nblk, limbs, lsc, vid, n);
+  return 8;
+}
+
+// Token held by lane t in column group q after tile_dot (or -1): lane 0 for
+// NP == 1; for NP >= 2 lanes 0 and 2 hold tokens 2q and 2q + 1.
+__device__ __forceinline__ int owner(int np, int t, int q) {
+  if (np == 1) return (t == 0 && q == 0) ? 0 : -1;
+  if (t & 1) return -1;
+  return q < np / 2 ? 2 * q + (t >> 1) : -1;
+}
+
+// Quantise activation vectors of 128-element chunks; task = vec * nch + chunk.
+// Each warp first issues the loads of up to MB tasks, then quantises them, so a
+// warp pays one memory latency per MB tasks.
+template <int NW, int MB, typename Load>
+__device__ __forceinline__ void quant_tasks(int ntask, int nch, int nblk, uint8_t *limbs, float2 *lsc, int warp,
+                                            int lane, Load load) {
+  for (int base = warp; base < ntask; base += MB * NW) {
+    float4 v[MB];
+#pragma unroll
+    for (int i = 0; i < MB; ++i) {
+      const int task = base + i * NW;
+      if (task < ntask) v[i] = load(task / nch, task % nch);
+    }
+#pragma unroll
+    for (int i = 0; i < MB; ++i) {
+      const int task = base + i * NW;
+      if (task < ntask) {
+        const int vec = task / nch;
+        quant_chunk(v[i], limbs + (size_t)vec * nblk * LIMB_REC, lsc + (size_t)vec * nblk, task % nch, lane);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + expf(-a)); }
+
+
+}  // namespace
+}  // namespace tile
+}  // namespace qmoe

@@ -12,20 +12,17 @@
 // copies of phase-2 tiles start as soon as ring slots free up, so they overlap
 // phase 1 and the first grid barrier.
 //
-// Contraction: activations of every 32-element block are quantised to 16-bit
-// fixed point with a per-block fp32 scale s (X = rint(v / s), |X| <= 32639) and
-// split into signed 8-bit limbs X = 256*hi + lo. The integer MMA m16n8k32
-// (u8 codes x s8 limbs, s32 accumulate) gives exact sum q*hi and sum q*lo per
-// block; the block's contribution is d * s * (256*Qhi + Qlo) + m * s * sum(X).
-// The eight MMA columns hold (hi, lo) pairs of up to four (token, block) pairs,
-// so even a single token keeps every lane busy in the fp32 epilogue.
+// The contraction itself (limb quantisation, integer MMA tiles) lives in
+// decode_tile.cuh, shared with the fused layer-stack kernel.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "decode_tile.cuh"
 #include "layout.cuh"
 
 namespace qmoe {
 namespace {
+using namespace tile;
 
 constexpr int NCW = 8;                     // consumer warps
 constexpr int FD_THREADS = 32 * (NCW + 1); // + one producer warp
@@ -33,11 +30,10 @@ constexpr int FD_MAXT = 8;
 constexpr int FD_MAXK = 16;
 constexpr int FD_MAXP = FD_MAXT * FD_MAXK; // (token, slot) pairs
 constexpr int CONSUMER_BAR = 1;            // named barrier id for the consumer warps
-constexpr float QMAX = 32639.0f;           // keeps both limbs inside int8
-
 struct Plan {
   int err;
   int abort;
+  int turn;  // next ring item whose arrival a consumer warp may wait for
   int U;
   int ue[FD_MAXP];
   int nt[FD_MAXP];
@@ -80,182 +76,6 @@ __host__ __device__ inline SmemLayout smem_layout(int nslots, int slot_bytes, in
   o.lsc = (o.limbs + (size_t)limb_bytes + 15) & ~(size_t)15;
   o.total = o.lsc + (size_t)lsc_count * 8;
   return o;
-}
-
-__device__ __forceinline__ float h2f(uint32_t bits16) { return __half2float(__ushort_as_half((unsigned short)bits16)); }
-
-// Quantise a 128-element chunk (4 blocks of 32) held one float4 per lane: lane
-// j carries elements 4j..4j+3, i.e. block j/8. Writes the int8 limbs of the
-// four blocks and (s, s * sum X) per block. The block's min term then uses the
-// same quantised values as its code term, so the whole block sees one
-// consistent activation s*X and the only error is that of quantising v,
-// carried through zero-mean weights.
-__device__ __forceinline__ int quant_one(float v, float inv) {
-  int X = __float2int_rn(v * inv);
-  return max(-32639, min(32639, X));
-}
-
-__device__ __forceinline__ void quant_chunk(float4 v, uint8_t *limbs_vec, float2 *lsc_vec, int chunk, int lane) {
-  float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
-  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
-  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
-  float s = 0.0f, inv = 0.0f;
-  if (a > 0.0f) {
-    s = a / QMAX;
-    inv = QMAX / a;
-  }
-  int X0 = quant_one(v.x, inv), X1 = quant_one(v.y, inv), X2 = quant_one(v.z, inv), X3 = quant_one(v.w, inv);
-  int h0 = (X0 + 128) >> 8, h1 = (X1 + 128) >> 8, h2 = (X2 + 128) >> 8, h3 = (X3 + 128) >> 8;
-  int l0 = X0 - (h0 << 8), l1 = X1 - (h1 << 8), l2 = X2 - (h2 << 8), l3 = X3 - (h3 << 8);
-  uint32_t hw = (uint32_t)(h0 & 0xff) | ((uint32_t)(h1 & 0xff) << 8) | ((uint32_t)(h2 & 0xff) << 16) |
-                ((uint32_t)(h3 & 0xff) << 24);
-  uint32_t lw = (uint32_t)(l0 & 0xff) | ((uint32_t)(l1 & 0xff) << 8) | ((uint32_t)(l2 & 0xff) << 16) |
-                ((uint32_t)(l3 & 0xff) << 24);
-  const int blk = chunk * 4 + (lane >> 3);
-  uint8_t *rec = limbs_vec + (size_t)blk * 64 + (lane & 7) * 4;
-  *reinterpret_cast<uint32_t *>(rec) = hw;
-  *reinterpret_cast<uint32_t *>(rec + 32) = lw;
-  int sx = X0 + X1 + X2 + X3;
-  sx += __shfl_xor_sync(0xffffffffu, sx, 1);
-  sx += __shfl_xor_sync(0xffffffffu, sx, 2);
-  sx += __shfl_xor_sync(0xffffffffu, sx, 4);   // |sx| < 2^24: exact in fp32
-  if ((lane & 7) == 0) lsc_vec[blk] = make_float2(s, s * (float)sx);
-}
-
-struct Acc {
-  float r0q0, r0q1, r1q0, r1q1;  // rows g / g+8 x column groups q = 0 / 1
-};
-
-// Dot products of one 16-row tile (K = 32 * nblk, nblk % 4 == 0) with n <= NP
-// activation vectors (vector ids vid[0..n)). Returns the lane's share; see the
-// file header for the column layout. Not inlined: phase 1 and phase 2 share one
-// copy of the code, which keeps the instruction footprint small.
-template <int BITS, int NP>
-__device__ __noinline__ Acc tile_dot(const uint8_t *tile, int nblk, const uint8_t *limbs, const float2 *lsc,
-                                     const int *vid, int n) {
-  constexpr int TS = NP <= 4 ? NP : 4;        // tokens per column set
-  constexpr int BS = NP <= 4 ? 4 / NP : 1;    // blocks per column set
-  constexpr int NQ = NP == 8 ? 2 : 1;         // column groups per block
-  constexpr int NSET = 4 / BS;                // column sets per 4-block chunk
-  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int pp = g >> 1, plimb = g & 1;
-  const int ptau = pp % TS, pbeta = pp / TS;
-  const int own_tau = t % TS, own_beta = t / TS;
-  const uint8_t *sbase = tile + 64 * nblk * BITS;   // scales follow the codes
-  float acc[2][NQ];
-#pragma unroll
-  for (int q = 0; q < NQ; ++q) acc[0][q] = acc[1][q] = 0.0f;
-  // vector ids of the B columns this lane provides / the D columns it reads
-  int pv[NQ], ov[NQ];
-#pragma unroll
-  for (int q = 0; q < NQ; ++q) {
-    const int ptq = (NP == 8) ? 4 * q + pp : ptau;
-    const int otq = (NP == 8) ? 4 * q + t : own_tau;
-    pv[q] = ptq < n ? vid[ptq] : -1;
-    ov[q] = otq < n ? vid[otq] : -1;
-  }
-
-#pragma unroll 1
-  for (int c = 0; c < (nblk >> 2); ++c) {
-    uint32_t w[8];
-    if (BITS == 2) {
-      const uint4 q = *reinterpret_cast<const uint4 *>(tile + c * 512 + lane * 16);
-      w[0] = q.x; w[1] = q.y; w[2] = q.z; w[3] = q.w;
-    } else {
-      const uint4 q0 = *reinterpret_cast<const uint4 *>(tile + (2 * c) * 512 + lane * 16);
-      const uint4 q1 = *reinterpret_cast<const uint4 *>(tile + (2 * c + 1) * 512 + lane * 16);
-      w[0] = q0.x; w[1] = q0.y; w[2] = q0.z; w[3] = q0.w;
-      w[4] = q1.x; w[5] = q1.y; w[6] = q1.z; w[7] = q1.w;
-    }
-#pragma unroll
-    for (int sb = 0; sb < NSET; ++sb) {
-#pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        // B limbs this lane provides for this column set
-        uint32_t b0 = 0u, b1 = 0u;
-        if (pv[q] >= 0) {
-          const int blk = c * 4 + sb * BS + ((NP == 8) ? 0 : pbeta);
-          const uint8_t *lp = limbs + ((size_t)pv[q] * nblk + blk) * 64 + plimb * 32 + 4 * t;
-          b0 = *reinterpret_cast<const uint32_t *>(lp);
-          b1 = *reinterpret_cast<const uint32_t *>(lp + 16);
-        }
-        int d0 = 0, d1 = 0, d2 = 0, d3 = 0;
-#pragma unroll
-        for (int beta = 0; beta < BS; ++beta) {
-          const int bb = sb * BS + beta;
-          uint32_t a0, a1, a2, a3;
-          if (BITS == 2) {
-            const uint32_t x = w[bb];
-            a0 = x & 0x03030303u;
-            a1 = (x >> 2) & 0x03030303u;
-            a2 = (x >> 4) & 0x03030303u;
-            a3 = (x >> 6) & 0x03030303u;
-          } else {
-            const uint32_t x0 = w[2 * bb], x1 = w[2 * bb + 1];
-            a0 = x0 & 0x0F0F0F0Fu;
-            a1 = (x0 >> 4) & 0x0F0F0F0Fu;
-            a2 = x1 & 0x0F0F0F0Fu;
-            a3 = (x1 >> 4) & 0x0F0F0F0Fu;
-          }
-          const bool on = (NP == 8) || (pbeta == beta);
-          mma_u8s8(d0, d1, d2, d3, a0, a1, a2, a3, on ? b0 : 0u, on ? b1 : 0u);
-        }
-        if (ov[q] >= 0) {
-          const int bo = c * 4 + sb * BS + ((NP == 8) ? 0 : own_beta);
-          const float v0 = (float)(d0 * 256 + d1);
-          const float v1 = (float)(d2 * 256 + d3);
-          const float2 ss = lsc[(size_t)ov[q] * nblk + bo];
-          const uint2 dm = *reinterpret_cast<const uint2 *>(sbase + (bo * 8 + g) * 8);
-          acc[0][q] = fmaf(h2f(dm.x & 0xffffu), ss.x * v0, fmaf(h2f(dm.x >> 16), ss.y, acc[0][q]));
-          acc[1][q] = fmaf(h2f(dm.y & 0xffffu), ss.x * v1, fmaf(h2f(dm.y >> 16), ss.y, acc[1][q]));
-        }
-      }
-    }
-  }
-  if (NP == 1) {
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      acc[r][0] += __shfl_xor_sync(0xffffffffu, acc[r][0], 1);
-      acc[r][0] += __shfl_xor_sync(0xffffffffu, acc[r][0], 2);
-    }
-  } else if (NP == 2) {
-#pragma unroll
-    for (int r = 0; r < 2; ++r) acc[r][0] += __shfl_xor_sync(0xffffffffu, acc[r][0], 2);
-  }
-  Acc out;
-  out.r0q0 = acc[0][0];
-  out.r1q0 = acc[1][0];
-  out.r0q1 = NQ > 1 ? acc[0][NQ - 1] : 0.0f;
-  out.r1q1 = NQ > 1 ? acc[1][NQ - 1] : 0.0f;
-  return out;
-}
-
-// Token slot held by this lane for column group q after tile_dot (or -1).
-template <int NP>
-__device__ __forceinline__ int owner_tau(int t, int q) {
-  if (NP == 8) return 4 * q + t;
-  if (q != 0) return -1;
-  return t < NP ? t : -1;
-}
-
-template <int BITS>
-__device__ __forceinline__ int dispatch_dot(const uint8_t *tile, int nblk, const uint8_t *limbs, const float2 *lsc,
-                                            const int *vid, int n, Acc &acc) {
-  if (n <= 1) { acc = tile_dot<BITS, 1>(tile, nblk, limbs, lsc, vid, n); return 1; }
-  if (n <= 2) { acc = tile_dot<BITS, 2>(tile, nblk, limbs, lsc, vid, n); return 2; }
-  if (n <= 4) { acc = tile_dot<BITS, 4>(tile, nblk, limbs, lsc, vid, n); return 4; }
-  acc = tile_dot<BITS, 8>(tile, nblk, limbs, lsc, vid, n);
-  return 8;
-}
-
-__device__ __forceinline__ int owner(int np, int t, int q) {
-  switch (np) {
-    case 1: return owner_tau<1>(t, q);
-    case 2: return owner_tau<2>(t, q);
-    case 4: return owner_tau<4>(t, q);
-    default: return owner_tau<8>(t, q);
-  }
 }
 
 // Route table -> unique experts (ascending), their tokens (ascending) and slots.
@@ -345,6 +165,7 @@ __device__ void build_plan(const FfnArgs &a, Plan *pl) {
     pl->U = U;
     pl->err = 0;
     pl->abort = 0;
+    pl->turn = 0;
   }
   __syncwarp();
 #pragma unroll
@@ -359,32 +180,6 @@ __device__ void build_plan(const FfnArgs &a, Plan *pl) {
   }
   __syncwarp();
 }
-
-// Quantise activation vectors of 128-element chunks; task = vec * nch + chunk.
-// Each warp first issues the loads of up to MB tasks, then quantises them, so a
-// warp pays one memory latency per MB tasks.
-template <int MB, typename Load>
-__device__ __forceinline__ void quant_tasks(int ntask, int nch, int nblk, uint8_t *limbs, float2 *lsc, int warp,
-                                            int lane, Load load) {
-  for (int base = warp; base < ntask; base += MB * NCW) {
-    float4 v[MB];
-#pragma unroll
-    for (int i = 0; i < MB; ++i) {
-      const int task = base + i * NCW;
-      if (task < ntask) v[i] = load(task / nch, task % nch);
-    }
-#pragma unroll
-    for (int i = 0; i < MB; ++i) {
-      const int task = base + i * NCW;
-      if (task < ntask) {
-        const int vec = task / nch;
-        quant_chunk(v[i], limbs + (size_t)vec * nblk * 64, lsc + (size_t)vec * nblk, task % nch, lane);
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + expf(-a)); }
 
 template <int BITS>
 __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
@@ -426,11 +221,14 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
 
   if (warp == NCW) {
     // ------------------------------------------------------------ producer --
-    // Every lane issues copies (item n by lane n % 32): one thread's bulk copies
-    // are serviced one after another, several issuers keep more bytes in flight.
+    // Lane s issues every copy into ring slot s, in item order (item n goes to
+    // slot n % S). One thread's bulk copies are serviced one after another, so
+    // several issuers keep more bytes in flight; keeping each slot's copies on
+    // one lane and in order means each wait below is at most one phase behind
+    // its barrier, which is what a parity wait can tell apart.
     int my_last = -1;
     bool aborted = false;
-    for (int n = lane; n < ntot; n += 32) {
+    for (int n = lane; lane < S && n < ntot; n += S) {
       const int s = n % S, it = n / S;
       if (n >= S) {
         const long long dl = clock64() + WAIT_BUDGET_CYCLES;
@@ -462,7 +260,7 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
     // never leave with copies in flight: wait for this lane's copies whose slot
     // was not reused (reuse implies the copy was consumed)
     const long long dl = clock64() + WAIT_BUDGET_CYCLES;
-    for (int n = lane; n <= my_last; n += 32) {
+    for (int n = lane; n <= my_last; n += S) {
       if (!aborted && n + S < ntot) continue;
       while (!mbar_try_wait(&full[n % S], (uint32_t)((n / S) & 1)))
         if (clock64() > dl) break;
@@ -477,19 +275,35 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
   {
     const int nch = H / 128;
     const float *x = a.x;
-    quant_tasks<16>(a.T * nch, nch, nblkH, limbs, lsc, warp, lane, [&](int t, int c) {
+    quant_tasks<NCW, 16>(a.T * nch, nch, nblkH, limbs, lsc, warp, lane, [&](int t, int c) {
       return __ldcg(reinterpret_cast<const float4 *>(x + (size_t)t * H + c * 128) + lane);
     });
   }
   named_barrier_sync(CONSUMER_BAR, nth);
 
+  // Waits for ring item n. Consumer warps take these waits in item order (the
+  // turn counter): when item n is awaited every earlier item has arrived, so
+  // its slot's barrier is at most one phase behind and the parity is exact.
   auto wait_full = [&](int n) -> bool {
-    if (*(volatile int *)&pl->abort) return false;
-    long long dl = clock64() + WAIT_BUDGET_CYCLES;
-    if (!mbar_wait(&full[n % S], (uint32_t)((n / S) & 1), dl)) {
+    const long long dl = clock64() + WAIT_BUDGET_CYCLES;
+    bool ok = true;
+    while (*(volatile int *)&pl->turn != n) {
+      if (*(volatile int *)&pl->abort) return false;
+      if (clock64() > dl) {
+        ok = false;
+        break;
+      }
+    }
+    if (ok) ok = mbar_wait(&full[n % S], (uint32_t)((n / S) & 1), dl);
+    if (!ok) {
       set_status(a.status, DEV_TIMEOUT);
       *(volatile int *)&pl->abort = 1;
       return false;
+    }
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence_block();
+      *(volatile int *)&pl->turn = n + 1;
     }
     return true;
   };
@@ -509,12 +323,12 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
     Acc acc;
     const int np = dispatch_dot<BITS>(tile, nblkH, limbs, lsc, &pl->ptok[pb], nu, acc);
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
+    for (int q = 0; q < 4; ++q) {
       const int tau = owner(np, t, q);
       if (tau >= 0 && tau < nu) {
         float *dst = a.abuf + ((size_t)(pb + tau) * 2 + m) * I + r * 16;
-        dst[g] = q ? acc.r0q1 : acc.r0q0;
-        dst[g + 8] = q ? acc.r1q1 : acc.r1q0;
+        dst[g] = acc.r0[q];
+        dst[g + 8] = acc.r1[q];
       }
     }
     release(n);
@@ -535,7 +349,7 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
   bool ok = !*(volatile int *)&pl->abort;
 
   // phase 2: down projection, one expert chunk at a time
-  const int hmaxp = a.limb_bytes / (I * 2);
+  const int hmaxp = a.limb_bytes / (I * 3);
   int item = lo2;
   while (ok && item < hi2) {
     const int u0 = item / H16;
@@ -554,7 +368,7 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
     {
       const int nch = I / 128;
       const float *abuf = a.abuf;
-      quant_tasks<8>(pairs * nch, nch, nblkI, limbs, lsc, warp, lane, [&](int lv, int c) {
+      quant_tasks<NCW, 8>(pairs * nch, nch, nblkI, limbs, lsc, warp, lane, [&](int lv, int c) {
         const float *ab = abuf + (size_t)(pb0 + lv) * 2 * I + c * 128;
         float4 gv = __ldcg(reinterpret_cast<const float4 *>(ab) + lane);
         float4 uv = __ldcg(reinterpret_cast<const float4 *>(ab + I) + lane);
@@ -576,14 +390,14 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
       Acc acc;
       const int np = dispatch_dot<BITS>(tile, nblkI, limbs, lsc, vid, nu, acc);
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
+      for (int q = 0; q < 4; ++q) {
         const int tau = owner(np, t, q);
         if (tau >= 0 && tau < nu) {
           const int p = pb + tau;
           const float gw = pl->pgate[p];
           float *dst = a.part + ((size_t)pl->ptok[p] * k + pl->pslot[p]) * H + r * 16;
-          dst[g] = gw * (q ? acc.r0q1 : acc.r0q0);
-          dst[g + 8] = gw * (q ? acc.r1q1 : acc.r1q0);
+          dst[g] = gw * acc.r0[q];
+          dst[g + 8] = gw * acc.r1[q];
         }
       }
       release(n);
@@ -678,9 +492,9 @@ qmoe_status qmoe::ffn_decode_launch(const qmoe_experts *ex, const float *x, int 
 
   const int tgu = tile_bytes(bits, H), tdn = tile_bytes(bits, I);
   a.slot_bytes = ((tgu > tdn ? tgu : tdn) + 127) & ~127;
-  int limb_x = T * H * 2, limb_h = FD_MAXT * I * 2;
+  int limb_x = T * H * 3, limb_h = FD_MAXT * I * 3;
   a.limb_bytes = ((limb_x > limb_h ? limb_x : limb_h) + 127) & ~127;
-  int lsc_x = T * (H / 32), lsc_h = (a.limb_bytes / (I * 2)) * (I / 32);
+  int lsc_x = T * (H / 32), lsc_h = (a.limb_bytes / (I * 3)) * (I / 32);
   a.lsc_count = lsc_x > lsc_h ? lsc_x : lsc_h;
   size_t cap = max_smem_optin();
   int S = 16;

@@ -32,10 +32,11 @@ __device__ __forceinline__ bool ranks_above(double va, int ea, double vb, int eb
   return va > vb || (va == vb && ea < eb);
 }
 
-// One warp; `l` is the token's logits [E] in global memory (written by other
-// CTAs before a fence, read through L2). M = values per lane = ceil(E / 32).
-template <int M>
-__device__ inline void warp_topk_gates_m(const double *l, int E, int k, int32_t *idx_out, float *gate_out,
+// One warp; get(e) returns the token's float64 logit of expert e (global
+// memory written by other CTAs and read through L2, or shared memory).
+// M = values per lane = ceil(E / 32).
+template <int M, typename Get>
+__device__ inline void warp_topk_gates_m(Get get, int E, int k, int32_t *idx_out, float *gate_out,
                                          TopkScratch *sc) {
   const int lane = threadIdx.x & 31;
   double val[M];
@@ -43,7 +44,7 @@ __device__ inline void warp_topk_gates_m(const double *l, int E, int k, int32_t 
 #pragma unroll
   for (int j = 0; j < M; ++j) {
     const int e = lane + 32 * j;
-    val[j] = e < E ? __ldcg(l + e) : 0.0;
+    val[j] = e < E ? get(e) : 0.0;
   }
 #pragma unroll
   for (int j = 0; j < M; ++j) {
@@ -109,7 +110,7 @@ __device__ inline void warp_topk_gates_m(const double *l, int E, int k, int32_t 
         const int e = lane + 32 * j;
         const double v = val[j];
         int rank = 0;
-        for (int e2 = 0; e2 < E && rank < k; ++e2) rank += ranks_above(__ldcg(l + e2), e2, v, e) ? 1 : 0;
+        for (int e2 = 0; e2 < E && rank < k; ++e2) rank += ranks_above(get(e2), e2, v, e) ? 1 : 0;
         if (rank < k) {
           sc->sel_e[rank] = e;
           sc->sel_v[rank] = v;
@@ -128,14 +129,21 @@ __device__ inline void warp_topk_gates_m(const double *l, int E, int k, int32_t 
   __syncwarp();
 }
 
+template <typename Get>
+__device__ inline void warp_topk_gates_get(Get get, int E, int k, int32_t *idx_out, float *gate_out,
+                                           TopkScratch *sc) {
+  if (E <= 32) warp_topk_gates_m<1>(get, E, k, idx_out, gate_out, sc);
+  else if (E <= 64) warp_topk_gates_m<2>(get, E, k, idx_out, gate_out, sc);
+  else if (E <= 128) warp_topk_gates_m<4>(get, E, k, idx_out, gate_out, sc);
+  else if (E <= 256) warp_topk_gates_m<8>(get, E, k, idx_out, gate_out, sc);
+  else if (E <= 512) warp_topk_gates_m<16>(get, E, k, idx_out, gate_out, sc);
+  else warp_topk_gates_m<32>(get, E, k, idx_out, gate_out, sc);
+}
+
+// Logits in global memory, written by other CTAs of this grid before a fence.
 __device__ inline void warp_topk_gates(const double *l, int E, int k, int32_t *idx_out, float *gate_out,
                                        TopkScratch *sc) {
-  if (E <= 32) warp_topk_gates_m<1>(l, E, k, idx_out, gate_out, sc);
-  else if (E <= 64) warp_topk_gates_m<2>(l, E, k, idx_out, gate_out, sc);
-  else if (E <= 128) warp_topk_gates_m<4>(l, E, k, idx_out, gate_out, sc);
-  else if (E <= 256) warp_topk_gates_m<8>(l, E, k, idx_out, gate_out, sc);
-  else if (E <= 512) warp_topk_gates_m<16>(l, E, k, idx_out, gate_out, sc);
-  else warp_topk_gates_m<32>(l, E, k, idx_out, gate_out, sc);
+  warp_topk_gates_get([&](int e) { return __ldcg(l + e); }, E, k, idx_out, gate_out, sc);
 }
 
 }  // namespace qmoe
