@@ -174,7 +174,11 @@ qmoe_status qmoe_ffn_decode(const qmoe_experts *experts, const float *x, int T,
  * The descriptor's arrays are host arrays of L entries (copied at create).
  * The stack lives in caller workspace (qmoe_stack_workspace_bytes()); it keeps
  * the input, output and every layer's idx/gate there at fixed addresses. */
-enum { QMOE_STACK_TIMING = 1 }; /* capture CUDA events around every route and FFN node */
+enum {
+  QMOE_STACK_TIMING = 1,    /* capture CUDA events around every route and FFN node */
+  QMOE_STACK_LAYERWISE = 2  /* use the per-layer kernel graph even where the fused kernel applies */
+};
+enum { QMOE_PATH_LAYERWISE = 0, QMOE_PATH_FUSED = 1 };
 
 typedef struct {
   int L, T, k;
@@ -197,13 +201,22 @@ qmoe_status qmoe_stack_destroy(qmoe_stack *stack);
  * gate [L,T,k] and the device status word. Any argument may be NULL. */
 qmoe_status qmoe_stack_buffers(const qmoe_stack *stack, float **x_in, float **x_out,
                                int32_t **idx, float **gate, int32_t **dev_status);
-/* Kernel launches in one replay of the stack's graph (2L + 1). */
+/* Kernel launches in one replay of the stack's graph: 2L + 1 on the per-layer
+ * path, 1 on the fused path. */
 int qmoe_stack_kernels_per_replay(const qmoe_stack *stack);
+/* Which path the stack runs. QMOE_PATH_FUSED (single-token stacks whose
+ * geometry fits one SM's shared memory): one persistent kernel runs all L
+ * layers with two grid barriers per layer; router logits there are formed from
+ * exact fixed-point partial sums (resolution 2^-40 per partial) instead of one
+ * float64 dot product per expert. QMOE_PATH_LAYERWISE: qmoe_residual_route and
+ * qmoe_ffn_decode per layer, chained with programmatic dependent launch. */
+int qmoe_stack_path(const qmoe_stack *stack);
 /* Per-layer durations (ms) of the most recent completed replay, measured by
  * the event nodes of a QMOE_STACK_TIMING stack: route_ms[l] spans layer l's
  * router (with its fused residual RMSNorm), ffn_ms[l] its FFN kernel. Host
  * arrays of L floats (either may be NULL). Synchronous; UNSUPPORTED without
- * the flag. */
+ * the flag. On the fused path the single kernel's duration is split evenly:
+ * route_ms[l] = 0 and ffn_ms[l] = kernel / L. */
 qmoe_status qmoe_stack_layer_times(const qmoe_stack *stack, float *route_ms, float *ffn_ms);
 /* One graph replay on `stream`: reads the stack's input buffer, writes its
  * output buffer. */

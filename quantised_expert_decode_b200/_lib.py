@@ -18,6 +18,8 @@ Q2, Q4 = 2, 4
 F32, BF16 = 0, 1
 GATE_UP, DOWN = 0, 1
 STACK_TIMING = 1
+STACK_LAYERWISE = 2
+PATH_LAYERWISE, PATH_FUSED = 0, 1
 
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "GEOMETRY", 3: "UNSUPPORTED", 4: "WORKSPACE",
                 5: "CUDA", 6: "TIMEOUT", 7: "DEVICE_STATUS"}
@@ -57,6 +59,7 @@ _SIGS = {
     "qmoe_stack_buffers": (_I, [_VP, ctypes.POINTER(_VP), ctypes.POINTER(_VP), ctypes.POINTER(_VP),
                                 ctypes.POINTER(_VP), ctypes.POINTER(_VP)]),
     "qmoe_stack_kernels_per_replay": (_I, [_VP]),
+    "qmoe_stack_path": (_I, [_VP]),
     "qmoe_stack_decode": (_I, [_VP, _VP]),
     "qmoe_stack_layer_times": (_I, [_VP, _VP, _VP]),
     "qmoe_stack_decode_host": (_I, [_VP, _VP, _VP, _VP]),
@@ -177,6 +180,10 @@ def qmoe_stack_buffers(stack: int) -> dict:
 
 def qmoe_stack_kernels_per_replay(stack: int) -> int:
     return lib().qmoe_stack_kernels_per_replay(stack)
+
+
+def qmoe_stack_path(stack: int) -> int:
+    return lib().qmoe_stack_path(stack)
 
 
 def qmoe_stack_layer_times(stack: int, L: int):

@@ -94,6 +94,10 @@ __device__ __forceinline__ void mma_u8s8(int &d0, int &d1, int &d2, int &d3, uin
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Orders this thread's generic-proxy memory accesses (and those it has
+// synchronised with) before its subsequent async-proxy (bulk copy) accesses.
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async;" ::: "memory"); }
+
 // Programmatic dependent launch: wait for the preceding grid's completion (and
 // its memory) / allow the next grid on the stream to start launching.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

@@ -25,6 +25,12 @@ namespace {  // internal linkage: each translation unit keeps its own copy
 constexpr float QMAX = 8355711.0f;         // 127*65536 + 127*256 + 127: three int8 limbs
 constexpr int LIMB_REC = 96;               // bytes per (vector, block): l2 | l1 | l0
 
+// Exact int -> float for |v| < 2^22: add into the mantissa of 1.5 * 2^23 and
+// subtract it again (two full-rate operations instead of a conversion).
+__device__ __forceinline__ float i2f_small(int v) {
+  return __int_as_float(0x4B400000 + v) - 12582912.0f;
+}
+
 __device__ __forceinline__ float h2f(uint32_t bits16) { return __half2float(__ushort_as_half((unsigned short)bits16)); }
 
 // Quantise a 128-element chunk (4 blocks of 32) held one float4 per lane: lane
@@ -209,6 +215,141 @@ __device__ __forceinline__ int owner(int np, int t, int q) {
   if (np == 1) return (t == 0 && q == 0) ? 0 : -1;
   if (t & 1) return -1;
   return q < np / 2 ? 2 * q + (t >> 1) : -1;
+}
+
+// Single-vector variant of tile_dot (NP == 1) with NCH 4-block chunks in flight,
+// so that independent MMAs and shared-memory loads overlap. Returns the tile's
+// rows (g, g+8) dot products; every lane of a quad holds them after the final
+// reduction. `limbs` / `lsc` point at the activation vector's own records.
+template <int BITS, int NCH = 2>
+__device__ __noinline__ float2 tile_dot1(const uint8_t *tile, int nblk, const uint8_t *limbs, const float2 *lsc) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int pP = g >> 2, pslot = g & 3;
+  const int ploff = pslot == 0 ? 0 : (pslot == 1 ? 32 : 64);
+  const bool pon = pslot != 2;
+  const int oP = t >> 1, ohalf = t & 1;
+  const float wgt = ohalf ? 1.0f : 256.0f;
+  const uint8_t *sbase = tile + 64 * nblk * BITS;
+  const int nchunks = nblk >> 2;
+  float acc0 = 0.0f, acc1 = 0.0f;
+  for (int c0 = 0; c0 < nchunks; c0 += NCH) {
+    uint32_t w[NCH][8];
+    uint32_t bv[NCH][2][2];
+#pragma unroll
+    for (int ch = 0; ch < NCH; ++ch) {
+      const int c = c0 + ch;
+      if (c < nchunks) {
+        if (BITS == 2) {
+          const uint4 q = *reinterpret_cast<const uint4 *>(tile + c * 512 + lane * 16);
+          w[ch][0] = q.x; w[ch][1] = q.y; w[ch][2] = q.z; w[ch][3] = q.w;
+        } else {
+          const uint4 q0 = *reinterpret_cast<const uint4 *>(tile + (2 * c) * 512 + lane * 16);
+          const uint4 q1 = *reinterpret_cast<const uint4 *>(tile + (2 * c + 1) * 512 + lane * 16);
+          w[ch][0] = q0.x; w[ch][1] = q0.y; w[ch][2] = q0.z; w[ch][3] = q0.w;
+          w[ch][4] = q1.x; w[ch][5] = q1.y; w[ch][6] = q1.z; w[ch][7] = q1.w;
+        }
+#pragma unroll
+        for (int sb = 0; sb < 2; ++sb) {
+          bv[ch][sb][0] = bv[ch][sb][1] = 0u;
+          if (pon) {
+            const uint8_t *lp = limbs + (size_t)(c * 4 + sb * 2 + pP) * LIMB_REC + ploff + 4 * t;
+            bv[ch][sb][0] = *reinterpret_cast<const uint32_t *>(lp);
+            bv[ch][sb][1] = *reinterpret_cast<const uint32_t *>(lp + 16);
+          }
+        }
+      }
+    }
+    int D[NCH][2][4];
+#pragma unroll
+    for (int ch = 0; ch < NCH; ++ch)
+#pragma unroll
+      for (int sb = 0; sb < 2; ++sb) D[ch][sb][0] = D[ch][sb][1] = D[ch][sb][2] = D[ch][sb][3] = 0;
+#pragma unroll
+    for (int beta = 0; beta < 2; ++beta) {
+#pragma unroll
+      for (int ch = 0; ch < NCH; ++ch) {
+        if (c0 + ch < nchunks) {
+#pragma unroll
+          for (int sb = 0; sb < 2; ++sb) {
+            const int bb = sb * 2 + beta;
+            uint32_t a0, a1, a2, a3;
+            if (BITS == 2) {
+              const uint32_t x = w[ch][bb];
+              a0 = x & 0x03030303u;
+              a1 = (x >> 2) & 0x03030303u;
+              a2 = (x >> 4) & 0x03030303u;
+              a3 = (x >> 6) & 0x03030303u;
+            } else {
+              const uint32_t x0 = w[ch][2 * bb], x1 = w[ch][2 * bb + 1];
+              a0 = x0 & 0x0F0F0F0Fu;
+              a1 = (x0 >> 4) & 0x0F0F0F0Fu;
+              a2 = x1 & 0x0F0F0F0Fu;
+              a3 = (x1 >> 4) & 0x0F0F0F0Fu;
+            }
+            const bool on = pP == beta;
+            mma_u8s8(D[ch][sb][0], D[ch][sb][1], D[ch][sb][2], D[ch][sb][3], a0, a1, a2, a3,
+                     on ? bv[ch][sb][0] : 0u, on ? bv[ch][sb][1] : 0u);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int ch = 0; ch < NCH; ++ch) {
+      if (c0 + ch < nchunks) {
+#pragma unroll
+        for (int sb = 0; sb < 2; ++sb) {
+          const int bo = (c0 + ch) * 4 + sb * 2 + oP;
+          // |v| <= 32*3*128*257 < 2^22 for 2-bit codes; 4-bit codes need the conversion
+          const int i0 = D[ch][sb][0] * 256 + D[ch][sb][1], i1 = D[ch][sb][2] * 256 + D[ch][sb][3];
+          const float v0 = BITS == 2 ? i2f_small(i0) : (float)i0;
+          const float v1 = BITS == 2 ? i2f_small(i1) : (float)i1;
+          const float2 ss = lsc[bo];
+          const uint2 dm = *reinterpret_cast<const uint2 *>(sbase + (bo * 8 + g) * 8);
+          const float sw = ss.x * wgt;
+          const float mt = ohalf ? 0.0f : ss.y;
+          acc0 = fmaf(h2f(dm.x & 0xffffu), sw * v0, fmaf(h2f(dm.x >> 16), mt, acc0));
+          acc1 = fmaf(h2f(dm.y & 0xffffu), sw * v1, fmaf(h2f(dm.y >> 16), mt, acc1));
+        }
+      }
+    }
+  }
+  acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
+  acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
+  acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
+  acc1 += __shfl_xor_sync(0xffffffffu, acc1, 2);
+  return make_float2(acc0, acc1);
+}
+
+// Inline form of quant_chunk with a reciprocal in place of the divisions, for
+// loops whose iterations the compiler may interleave. s and inv need not be
+// exact inverses: the contraction uses s itself, so s * X still tracks v to
+// within rounding of the quantisation.
+__device__ __forceinline__ void quant_chunk_inl(float4 v, uint8_t *limbs_vec, float2 *lsc_vec, int chunk, int lane) {
+  float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
+  float s = 0.0f, inv = 0.0f;
+  if (a > 0.0f) {
+    s = a * (1.0f / QMAX);
+    inv = __frcp_rn(s);
+  }
+  const int X0 = quant_one(v.x, inv), X1 = quant_one(v.y, inv), X2 = quant_one(v.z, inv), X3 = quant_one(v.w, inv);
+  int a2, a1, a0, b2, b1, b0, c2, c1, c0, d2, d1, d0;
+  limbs3(X0, a2, a1, a0);
+  limbs3(X1, b2, b1, b0);
+  limbs3(X2, c2, c1, c0);
+  limbs3(X3, d2, d1, d0);
+  const int blk = chunk * 4 + (lane >> 3);
+  uint8_t *rec = limbs_vec + (size_t)blk * LIMB_REC + (lane & 7) * 4;
+  *reinterpret_cast<uint32_t *>(rec) = pack4(a2, b2, c2, d2);
+  *reinterpret_cast<uint32_t *>(rec + 32) = pack4(a1, b1, c1, d1);
+  *reinterpret_cast<uint32_t *>(rec + 64) = pack4(a0, b0, c0, d0);
+  int sx = X0 + X1 + X2 + X3;
+  sx += __shfl_xor_sync(0xffffffffu, sx, 1);
+  sx += __shfl_xor_sync(0xffffffffu, sx, 2);
+  sx += __shfl_xor_sync(0xffffffffu, sx, 4);
+  if ((lane & 7) == 0) lsc_vec[blk] = make_float2(s, s * (float)sx);
 }
 
 // Quantise activation vectors of 128-element chunks; task = vec * nch + chunk.

@@ -6,6 +6,26 @@
 #include "common.cuh"
 
 namespace qmoe {
+struct FusedPlan {
+  size_t smem;
+  int nslots, slot_bytes;
+};
+struct FusedBufs {
+  float *wrt;
+  unsigned long long *lacc, *ssacc;
+  float *zbuf, *hbuf;
+  unsigned *bar;
+  const uint8_t **gu, **dn;
+  const float **bias;
+};
+bool fused_stack_plan(int fmt, int E, int H, int I, int k, FusedPlan *p);
+size_t fused_stack_ws_bytes(int L, int E, int H, int I, int k);
+FusedBufs fused_carve(void *ws, int L, int E, int H, int I, int k);
+qmoe_status fused_prepare(const FusedBufs &b, int L, int E, int H, const float *const *Wr,
+                          const qmoe_experts *layers, const float *const *bias, cudaStream_t s);
+qmoe_status fused_launch(const FusedBufs &b, const FusedPlan &p, int fmt, int L, int E, int H, int I, int k, float eps,
+                         const float *x_in, float *x_out, int32_t *idx_rec, float *gate_rec, int32_t *status,
+                         cudaStream_t s, bool cooperative);
 qmoe_status ffn_decode_launch(const qmoe_experts *ex, const float *x, int T, const int32_t *idx, const float *gate,
                               int k, float *y, void *ws, size_t ws_bytes, int32_t *status, cudaStream_t s,
                               bool cooperative);
@@ -28,6 +48,9 @@ struct qmoe_stack {
   cudaGraphExec_t exec;
   int kernels;
   int flags;
+  int path;
+  qmoe::FusedPlan fplan;
+  qmoe::FusedBufs fbufs;
   std::vector<cudaEvent_t> events;  // 2L + 1 when timing
 };
 
@@ -36,19 +59,24 @@ namespace {
 size_t al(size_t b) { return (b + 255) & ~(size_t)255; }
 
 struct Layout {
-  size_t x, idx, gate, status, route, ffn, total;
+  size_t x, idx, gate, status, route, ffn, fused, total;
+  bool use_fused;
+  qmoe::FusedPlan fplan;
 };
 
 Layout layout_of(const qmoe_stack_desc *d) {
   const qmoe_experts &e = d->layers[0];
   Layout l;
+  l.use_fused = d->T == 1 && !(d->flags & QMOE_STACK_LAYERWISE) &&
+                qmoe::fused_stack_plan(e.fmt, e.E, e.H, e.I, d->k, &l.fplan);
+  l.fused = l.use_fused ? al(qmoe::fused_stack_ws_bytes(d->L, e.E, e.H, e.I, d->k)) : 0;
   l.x = al((size_t)d->T * e.H * 4);
   l.idx = al((size_t)d->L * d->T * d->k * 4);
   l.gate = l.idx;
   l.status = 256;
   l.route = al(qmoe_route_workspace_bytes(d->T, e.E));
   l.ffn = al(qmoe_decode_workspace_bytes(d->T, d->k, e.H, e.I));
-  l.total = 5 * l.x + l.idx + l.gate + l.status + l.route + l.ffn;
+  l.total = 5 * l.x + l.idx + l.gate + l.status + l.route + l.ffn + l.fused;
   return l;
 }
 
@@ -100,6 +128,17 @@ qmoe_status record(qmoe_stack *s, cudaStream_t cs, bool coop) {
   return st;
 }
 
+qmoe_status record_fused(qmoe_stack *s, cudaStream_t cs, bool coop) {
+  const bool timing = !s->events.empty();
+  if (timing && cudaEventRecordWithFlags(s->events[0], cs, cudaEventRecordExternal) != cudaSuccess) return QMOE_ERR_CUDA;
+  qmoe_status st = qmoe::fused_launch(s->fbufs, s->fplan, s->fmt, s->L, s->E, s->H, s->I, s->k, s->eps, s->x_in,
+                                      s->x_out, s->idx, s->gate, s->status, cs, coop);
+  if (st != QMOE_OK) return st;
+  if (timing && cudaEventRecordWithFlags(s->events[1], cs, cudaEventRecordExternal) != cudaSuccess) return QMOE_ERR_CUDA;
+  s->kernels = 1;
+  return QMOE_OK;
+}
+
 qmoe_status capture(qmoe_stack *s, bool coop) {
   cudaStream_t cs;
   if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return QMOE_ERR_CUDA;
@@ -109,7 +148,7 @@ qmoe_status capture(qmoe_stack *s, bool coop) {
     cudaStreamDestroy(cs);
     return QMOE_ERR_CUDA;
   }
-  qmoe_status rs = record(s, cs, coop);
+  qmoe_status rs = s->path == QMOE_PATH_FUSED ? record_fused(s, cs, coop) : record(s, cs, coop);
   cudaError_t e = cudaStreamEndCapture(cs, &g);
   if (rs != QMOE_OK) st = rs;
   else if (e != cudaSuccess) st = QMOE_ERR_CUDA;
@@ -173,13 +212,24 @@ extern "C" qmoe_status qmoe_stack_create(const qmoe_stack_desc *d, void *workspa
   s->gate = reinterpret_cast<float *>(p); p += lo.gate;
   s->status = reinterpret_cast<int32_t *>(p); p += lo.status;
   s->route_ws = p; s->route_ws_bytes = lo.route; p += lo.route;
-  s->ffn_ws = p; s->ffn_ws_bytes = lo.ffn;
+  s->ffn_ws = p; s->ffn_ws_bytes = lo.ffn; p += lo.ffn;
+  s->path = lo.use_fused ? QMOE_PATH_FUSED : QMOE_PATH_LAYERWISE;
+  s->fplan = lo.fplan;
+  if (lo.use_fused) s->fbufs = qmoe::fused_carve(p, d->L, s->E, s->H, s->I, s->k);
   if (cudaMemsetAsync(workspace, 0, lo.total, (cudaStream_t)stream) != cudaSuccess ||
       cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) {
     delete s;
     return QMOE_ERR_CUDA;
   }
-  st = capture(s, false);
+  if (s->path == QMOE_PATH_FUSED) {
+    st = qmoe::fused_prepare(s->fbufs, s->L, s->E, s->H, d->Wr, d->layers, d->bias, (cudaStream_t)stream);
+    if (st == QMOE_OK) {
+      st = capture(s, true);                        // cooperative launch: all CTAs resident
+      if (st == QMOE_ERR_CUDA) st = capture(s, false);
+    }
+  } else {
+    st = capture(s, false);
+  }
   if (st != QMOE_OK) {
     for (auto &e : s->events) cudaEventDestroy(e);
     delete s;
@@ -211,6 +261,8 @@ extern "C" qmoe_status qmoe_stack_buffers(const qmoe_stack *s, float **x_in, flo
 
 extern "C" int qmoe_stack_kernels_per_replay(const qmoe_stack *s) { return s ? s->kernels : 0; }
 
+extern "C" int qmoe_stack_path(const qmoe_stack *s) { return s ? s->path : -1; }
+
 extern "C" qmoe_status qmoe_stack_decode(qmoe_stack *s, qmoe_stream_t stream) {
   if (!s || !s->exec) return QMOE_ERR_INVALID_ARG;
   cudaError_t e = cudaGraphLaunch(s->exec, (cudaStream_t)stream);
@@ -233,6 +285,17 @@ extern "C" qmoe_status qmoe_stack_decode_host(qmoe_stack *s, const float *x_host
 extern "C" qmoe_status qmoe_stack_layer_times(const qmoe_stack *s, float *route_ms, float *ffn_ms) {
   if (!s) return QMOE_ERR_INVALID_ARG;
   if (s->events.empty()) return QMOE_ERR_UNSUPPORTED;
+  if (s->path == QMOE_PATH_FUSED) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(s->events[1]) != cudaSuccess ||
+        cudaEventElapsedTime(&ms, s->events[0], s->events[1]) != cudaSuccess)
+      return QMOE_ERR_CUDA;
+    for (int l = 0; l < s->L; ++l) {
+      if (route_ms) route_ms[l] = 0.f;
+      if (ffn_ms) ffn_ms[l] = ms / s->L;
+    }
+    return QMOE_OK;
+  }
   if (cudaEventSynchronize(s->events.back()) != cudaSuccess) return QMOE_ERR_CUDA;
   for (int l = 0; l < s->L; ++l) {
     float a = 0.f, b = 0.f;

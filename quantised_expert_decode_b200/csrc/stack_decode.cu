@@ -1,0 +1,599 @@
+// Fused single-token decode stack: all L layers of router -> expert FFN ->
+// gate-weighted combine -> residual RMSNorm in ONE persistent kernel (one CTA
+// per SM, every CTA resident), so the instruction stream, the shared-memory
+// carve-up and the bulk-copy ring stay warm across layers and a layer costs two
+// grid barriers instead of several kernel boundaries.
+//
+// Work split per layer l (G CTAs; CTA c < H/16 owns output rows R_c = 16c..16c+15):
+//   A  every CTA: x_l = z_l / rms_l from the z slices and the exact sum of
+//      squares of the previous layer; router logits from the exact partial sums
+//      of the previous layer (divided by rms_l, plus the bias); top-k with
+//      renormalised gates (one warp, identical in every CTA); then the producer
+//      warp issues this layer's weight copies.
+//   C  gate/up tiles (selected expert j, 16-row tile r, gate or up), one ring
+//      item each: a_g = Wg x or a_u = Wu x for those 16 rows -> global
+//      ---- grid barrier (h complete) ----
+//   D  row owners: h_j = silu(a_g) * a_u, quantise all h_j, down tiles of rows R_c for every selected
+//      expert (prefetched during C), y[R_c] = sum_j g_j * (Wd_j h_j)[R_c] in
+//      slot order, z_{l+1}[R_c] = x_l[R_c] + y[R_c]; then, from the rows
+//      R_c of the next layer's transposed router (prefetched), partial logits
+//      sum_{h in R_c} Wr_{l+1}[e][h] z[h] for every expert and the partial sum of
+//      squares of z, both added as fixed-point integers (scale 2^40) so the
+//      totals are exact and independent of the order of the additions.
+//      ---- grid barrier (z, logit and norm partials complete) ----
+// The router logit of the next layer is Wr (z / rms) = (Wr z) / rms, which is
+// why the partial logits can be formed before the norm is known. Layer 0 uses
+// the raw input (no norm); after the last layer x_out = z_L / rms_L.
+#include <vector>
+
+#include "common.cuh"
+#include "decode_tile.cuh"
+#include "layout.cuh"
+#include "route_common.cuh"
+
+namespace qmoe {
+namespace {
+using namespace tile;
+
+constexpr int SK_NCW = 7;  // consumer warps; with the producer 256 threads, so up to 255 registers
+constexpr int SK_THREADS = 32 * (SK_NCW + 1);
+constexpr int SK_MAXK = 16;
+constexpr int CONS_BAR = 1;
+constexpr double FIX_SCALE = 1099511627776.0;  // 2^40
+constexpr double FIX_INV = 1.0 / 1099511627776.0;
+
+struct StackArgs {
+  int L, E, H, I, k;
+  float eps;
+  const uint8_t *const *gu;   // [L] packed gate/up tiles per layer
+  const uint8_t *const *dn;   // [L] packed down tiles per layer
+  const float *const *bias;   // [L], entries may be null
+  const float *wrt;           // [L][H][E] routers, transposed
+  const float *x_in;          // [H]
+  float *x_out;               // [H]
+  int32_t *idx_rec;           // [L][k]
+  float *gate_rec;            // [L][k]
+  float *zbuf;                // [2][H]
+  unsigned long long *lacc;   // [2][E] fixed-point partial-logit sums (two's complement)
+  unsigned long long *ssacc;  // [2] fixed-point sum of squares
+  float *hbuf;                // [2][k][I]: a_g, a_u
+  unsigned *bar;
+  int32_t *status;
+  int nslots, slot_bytes;
+  int w_rows, w_free;         // gate/up work weights of CTAs with / without output rows
+};
+
+struct SkState {
+  int abort;
+  int turn;  // next ring item whose arrival a consumer warp may wait for
+  int idx[SK_MAXK];
+  float gate[SK_MAXK];
+  float ztmp[16];
+  int vid[SK_MAXK];  // vector ids 0..k-1 of the limb region
+  TopkScratch tks;
+};
+
+struct SkLayout {
+  size_t ring, dnbuf, wrtbuf, xs, limbs, lsc, logits, ytmp, bars, state, total;
+};
+
+__host__ __device__ inline size_t al128(size_t v) { return (v + 127) & ~(size_t)127; }
+
+__host__ __device__ inline SkLayout sk_layout(int bits, int E, int H, int I, int k, int nslots, int slot_bytes) {
+  SkLayout o;
+  const size_t tdn = (size_t)tile_bytes(bits, I);
+  const size_t vecs = (size_t)((H / 32) > k * (I / 32) ? (H / 32) : k * (I / 32));  // limb records
+  o.ring = 0;
+  o.dnbuf = al128(o.ring + (size_t)nslots * slot_bytes);
+  o.wrtbuf = al128(o.dnbuf + (size_t)k * tdn);
+  o.xs = al128(o.wrtbuf + (size_t)16 * E * 4);
+  o.limbs = al128(o.xs + (size_t)H * 4);
+  o.lsc = al128(o.limbs + vecs * LIMB_REC);
+  o.logits = al128(o.lsc + vecs * 8);
+  o.ytmp = al128(o.logits + (size_t)E * 8);
+  o.bars = al128(o.ytmp + (size_t)k * 16 * 4);
+  o.state = al128(o.bars + (size_t)(2 * nslots + 3) * 8);
+  o.total = o.state + sizeof(SkState);
+  return o;
+}
+
+__device__ __forceinline__ unsigned long long to_fixed(double v) {
+  return (unsigned long long)__double2ll_rn(v * FIX_SCALE);
+}
+__device__ __forceinline__ double from_fixed(unsigned long long v) { return (double)(long long)v * FIX_INV; }
+
+// Consumer-side grid barrier: the 256 consumer threads meet, one thread joins
+// the grid, the consumers meet again. Returns false once the CTA has aborted.
+__device__ __forceinline__ bool cons_grid_barrier(const StackArgs &a, SkState *st, int tid) {
+  named_barrier_sync(CONS_BAR, SK_NCW * 32);
+  if (tid == 0) {
+    if (!*(volatile int *)&st->abort && !grid_barrier_one_thread(a.bar, gridDim.x)) {
+      set_status(a.status, DEV_TIMEOUT);
+      *(volatile int *)&st->abort = 1;
+    }
+    __threadfence();
+  }
+  named_barrier_sync(CONS_BAR, SK_NCW * 32);
+  return !*(volatile int *)&st->abort;
+}
+
+// Top-k of logits held in shared memory (kept out of line: it runs once per
+// layer and would otherwise add its registers to the kernel body's).
+__device__ __noinline__ void topk_smem(const double *logits, int E, int k, int32_t *idx, float *gate, TopkScratch *sc) {
+  warp_topk_gates_get([&](int e) { return logits[e]; }, E, k, idx, gate, sc);
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int S = a.nslots;
+  const int H = a.H, I = a.I, E = a.E, k = a.k, L = a.L;
+  const SkLayout lay = sk_layout(BITS, E, H, I, k, S, a.slot_bytes);
+  uint8_t *ring = smem + lay.ring;
+  uint8_t *dnbuf = smem + lay.dnbuf;
+  float *wrtbuf = reinterpret_cast<float *>(smem + lay.wrtbuf);
+  float *xs = reinterpret_cast<float *>(smem + lay.xs);
+  uint8_t *limbs = smem + lay.limbs;
+  float2 *lsc = reinterpret_cast<float2 *>(smem + lay.lsc);
+  double *logits = reinterpret_cast<double *>(smem + lay.logits);
+  float *ytmp = reinterpret_cast<float *>(smem + lay.ytmp);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.bars);
+  uint64_t *empty = full + S;
+  uint64_t *dnbar = empty + S;
+  uint64_t *wrtbar = dnbar + 1;
+  uint64_t *hbar = wrtbar + 1;
+  SkState *st = reinterpret_cast<SkState *>(smem + lay.state);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nblkH = H / 32, nblkI = I / 32, I16 = I / 16, H16 = H / 16;
+  const int tgu = tile_bytes(BITS, H), tdn = tile_bytes(BITS, I);
+  const int G = (int)gridDim.x, c = blockIdx.x;
+  const bool rows = c < H16;
+  const int r0 = 16 * c;
+  // gate/up units (selected expert j, 16-row tile r) of this CTA, balanced by bytes
+  auto wcum = [&](int cc) -> long long {
+    const int nr = cc < H16 ? cc : H16;
+    return (long long)nr * a.w_rows + (long long)(cc - nr) * a.w_free;
+  };
+  const int NU = k * I16;
+  const long long WT = wcum(G);
+  const int ulo = (int)(wcum(c) * NU / WT), uhi = (int)(wcum(c + 1) * NU / WT);
+  const int nunits = uhi - ulo;
+  const int nth = SK_NCW * 32;
+  const bool producer = warp == SK_NCW;
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(dnbar, 1);
+    mbar_init(wrtbar, 1);
+    mbar_init(hbar, 1);
+    fence_mbar_init();
+    st->abort = 0;
+    st->turn = 0;
+    for (int j = 0; j < SK_MAXK; ++j) st->vid[j] = j;
+  }
+  __syncthreads();
+
+  // ------------------------------------------ prologue: layer-0 logit partials
+  if (producer && lane == 0 && rows) {
+    mbar_arrive_expect_tx(wrtbar, (uint32_t)(16 * E * 4));
+    bulk_g2s(wrtbuf, a.wrt + (size_t)r0 * E, (uint32_t)(16 * E * 4), wrtbar);
+  }
+  if (!producer && rows) {
+    if (tid < 16) {
+      const float z = a.x_in[r0 + tid];
+      st->ztmp[tid] = z;
+      a.zbuf[r0 + tid] = z;
+    }
+    named_barrier_sync(CONS_BAR, nth);
+    if (!mbar_wait(wrtbar, 0u, clock64() + WAIT_BUDGET_CYCLES)) {
+      set_status(a.status, DEV_TIMEOUT);
+      st->abort = 1;
+    } else {
+      for (int e = tid; e < E; e += nth) {
+        double p = 0.0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) p = fma((double)wrtbuf[i * E + e], (double)st->ztmp[i], p);
+        atomicAdd(&a.lacc[e], to_fixed(p));
+      }
+    }
+  }
+  if (!producer) cons_grid_barrier(a, st, tid);
+
+  // Ring bookkeeping shared by producer and consumers (same sequence of items).
+  int nring = 0;
+  // Consumers take arrival waits in ring order; see the per-layer FFN kernel.
+  auto wait_full = [&](int n) -> bool {
+    const long long dl = clock64() + WAIT_BUDGET_CYCLES;
+    bool ok = true;
+    while (*(volatile int *)&st->turn != n) {
+      if (*(volatile int *)&st->abort) return false;
+      if (clock64() > dl) {
+        ok = false;
+        break;
+      }
+    }
+    if (ok) ok = mbar_wait(&full[n % S], (uint32_t)((n / S) & 1), dl);
+    if (!ok) {
+      set_status(a.status, DEV_TIMEOUT);
+      *(volatile int *)&st->abort = 1;
+      return false;
+    }
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence_block();
+      *(volatile int *)&st->turn = n + 1;
+    }
+    return true;
+  };
+
+  for (int l = 0; l < L; ++l) {
+    const int par = l & 1;
+    // ------------------------------------------------------------------ A --
+    if (!producer && !*(volatile int *)&st->abort) {
+      // one batch of loads: sum of squares, z, partial logits, bias
+      const float4 *zb = reinterpret_cast<const float4 *>(a.zbuf + (size_t)par * H);
+      const float *b = a.bias[l];
+      const unsigned long long *la = a.lacc + (size_t)par * E;
+      const unsigned long long ssv = __ldcg(&a.ssacc[par]);
+      float4 zv[4];
+      unsigned long long lv[4];
+      float bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int q = tid + i * nth;
+        if (q < H / 4) zv[i] = __ldcg(zb + q);
+        if (q < E) {
+          lv[i] = __ldcg(la + q);
+          bv[i] = b ? __ldg(b + q) : 0.0f;
+        }
+      }
+      const double rms = l > 0 ? sqrt(from_fixed(ssv) / (double)H + (double)a.eps) : 1.0;
+      const double rinv = 1.0 / rms;
+      const float inv = (float)rinv;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int q = tid + i * nth;
+        if (q < H / 4) {
+          float4 v = zv[i];
+          if (l > 0) {
+            v.x *= inv; v.y *= inv; v.z *= inv; v.w *= inv;
+          }
+          reinterpret_cast<float4 *>(xs)[q] = v;
+        }
+        if (q < E) logits[q] = from_fixed(lv[i]) * rinv + (double)bv[i];
+      }
+      for (int q = tid + 4 * nth; q < H / 4; q += nth) {   // larger geometries only
+        float4 v = __ldcg(zb + q);
+        if (l > 0) {
+          v.x *= inv; v.y *= inv; v.z *= inv; v.w *= inv;
+        }
+        reinterpret_cast<float4 *>(xs)[q] = v;
+      }
+      for (int q = tid + 4 * nth; q < E; q += nth) logits[q] = from_fixed(__ldcg(la + q)) * rinv + (b ? (double)b[q] : 0.0);
+      // clear the other parity's accumulators for the next layer (read last by
+      // every CTA before the previous barriers)
+      unsigned long long *lz = a.lacc + (size_t)(par ^ 1) * E;
+      for (int e = c * nth + tid; e < E; e += G * nth) lz[e] = 0ull;
+      if (c == 0 && tid == 0) a.ssacc[par ^ 1] = 0ull;
+      named_barrier_sync(CONS_BAR, nth);
+      if (warp == 0) {
+        topk_smem(logits, E, k, st->idx, st->gate, &st->tks);
+        if (c == 0 && lane < k) {
+          a.idx_rec[l * k + lane] = st->idx[lane];
+          a.gate_rec[l * k + lane] = st->gate[lane];
+        }
+      } else {
+        // quantise x_l (all 7 other warps)
+        const int nch = H / 128;
+        for (int task = warp - 1; task < nch; task += SK_NCW - 1) {
+          const float4 v = reinterpret_cast<const float4 *>(xs + task * 128)[lane];
+          quant_chunk_inl(v, limbs, lsc, task, lane);
+        }
+      }
+    }
+    // plan ready (includes the producer warp); every thread sees one abort value
+    if (__syncthreads_or(*(volatile int *)&st->abort)) break;
+
+    if (producer) {
+      // -------------------------------------------------------------- B --
+      // lane s < S: ring slot s (gate/up tiles, in item order); lane 31: this
+      // CTA's down tiles; lane 30: next layer's router rows.
+      fence_proxy_async();   // ring memory was last read with ordinary loads
+      const uint8_t *gu = a.gu[l];
+      const int first = nring + ((lane - nring % S) % S + S) % S;  // first item of slot `lane`
+      for (int n = first; lane < S && n < nring + 2 * nunits; n += S) {
+        const int s = n % S;
+        if (n >= S) {
+          const long long dl = clock64() + WAIT_BUDGET_CYCLES;
+          bool ok = true;
+          while (!mbar_try_wait(&empty[s], (uint32_t)(((n / S) - 1) & 1))) {
+            if (*(volatile int *)&st->abort || clock64() > dl) {
+              ok = false;
+              break;
+            }
+          }
+          if (!ok) break;
+        }
+        const int m = (n - nring) >> 1, mat = (n - nring) & 1;
+        const int u = ulo + m, j = u / I16, r = u % I16;
+        const uint8_t *src = gu + (((size_t)st->idx[j] * 2 + mat) * I16 + r) * (size_t)tgu;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)tgu);
+        bulk_g2s(ring + (size_t)s * a.slot_bytes, src, (uint32_t)tgu, &full[s]);
+      }
+      if (lane == 31 && rows) {
+        const uint8_t *dn = a.dn[l];
+        mbar_arrive_expect_tx(dnbar, (uint32_t)(k * tdn));
+        for (int j = 0; j < k; ++j)
+          bulk_g2s(dnbuf + (size_t)j * tdn, dn + ((size_t)st->idx[j] * H16 + c) * (size_t)tdn, (uint32_t)tdn, dnbar);
+      }
+      if (lane == 30 && rows && l + 1 < L) {
+        mbar_arrive_expect_tx(wrtbar, (uint32_t)(16 * E * 4));
+        bulk_g2s(wrtbuf, a.wrt + ((size_t)(l + 1) * H + r0) * E, (uint32_t)(16 * E * 4), wrtbar);
+      }
+      nring += 2 * nunits;
+      continue;
+    }
+
+    // -------------------------------------------------------------------- C --
+    for (int m = warp; m < 2 * nunits; m += SK_NCW) {
+      const int n = nring + m;
+      if (!wait_full(n)) break;
+      const int u = ulo + (m >> 1), mat = m & 1, j = u / I16, r = u % I16;
+      const float2 o = tile_dot1<BITS, 4>(ring + (size_t)(n % S) * a.slot_bytes, nblkH, limbs, lsc);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[n % S]);
+      if ((lane & 3) == 0) {   // lanes of quad g hold rows g and g+8 of the tile
+        const int g = lane >> 2;
+        float *dst = a.hbuf + ((size_t)mat * k + j) * I + r * 16;
+        dst[g] = o.x;
+        dst[g + 8] = o.y;
+      }
+    }
+    nring += 2 * nunits;
+    if (!cons_grid_barrier(a, st, tid)) continue;
+
+    // -------------------------------------------------------------------- D --
+    if (rows) {
+      {
+        const int nch = I / 128;
+        // a_g and a_u of every selected expert arrive in one bulk copy into
+        // the ring (all of this layer's ring items were consumed before the
+        // barrier), then quantise from shared memory
+        float *hs = reinterpret_cast<float *>(ring);
+        const uint32_t hbytes = (uint32_t)(2 * k * I * 4);
+        if (tid == 0) {
+          fence_proxy_async();   // h was written by ordinary stores; the ring was read by ordinary loads
+          mbar_arrive_expect_tx(hbar, hbytes);
+          bulk_g2s(hs, a.hbuf, hbytes, hbar);
+        }
+        const bool hok = mbar_wait(hbar, (uint32_t)(l & 1), clock64() + WAIT_BUDGET_CYCLES);
+        if (!hok) {
+          set_status(a.status, DEV_TIMEOUT);
+          *(volatile int *)&st->abort = 1;
+        }
+        const float *hg = hs, *hu = hs + (size_t)k * I;
+        const int ntask = hok ? k * nch : 0;
+        // three chunks per pass so that their independent chains interleave
+        for (int base = warp; base < ntask; base += 3 * SK_NCW) {
+          float4 h[3];
+#pragma unroll
+          for (int i = 0; i < 3; ++i) {
+            const int task = base + i * SK_NCW;
+            if (task < ntask) {
+              const size_t off = (size_t)(task / nch) * I + (task % nch) * 128;
+              const float4 gv = reinterpret_cast<const float4 *>(hg + off)[lane];
+              const float4 uv = reinterpret_cast<const float4 *>(hu + off)[lane];
+              h[i] = make_float4(silu_f(gv.x) * uv.x, silu_f(gv.y) * uv.y, silu_f(gv.z) * uv.z, silu_f(gv.w) * uv.w);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 3; ++i) {
+            const int task = base + i * SK_NCW;
+            if (task < ntask) {
+              const int j = task / nch;
+              quant_chunk_inl(h[i], limbs + (size_t)j * nblkI * LIMB_REC, lsc + (size_t)j * nblkI, task % nch, lane);
+            }
+          }
+        }
+      }
+      named_barrier_sync(CONS_BAR, nth);
+      bool ok = mbar_wait(dnbar, (uint32_t)(l & 1), clock64() + WAIT_BUDGET_CYCLES);
+      if (ok) {
+        for (int j = warp; j < k; j += SK_NCW) {
+          const float2 o = tile_dot1<BITS, 4>(dnbuf + (size_t)j * tdn, nblkI, limbs + (size_t)j * nblkI * LIMB_REC,
+                                           lsc + (size_t)j * nblkI);
+          if ((lane & 3) == 0) {
+            const int g = lane >> 2;
+            ytmp[j * 16 + g] = o.x;
+            ytmp[j * 16 + g + 8] = o.y;
+          }
+        }
+      } else {
+        set_status(a.status, DEV_TIMEOUT);
+        *(volatile int *)&st->abort = 1;
+      }
+      named_barrier_sync(CONS_BAR, nth);
+      if (ok && warp == 0) {
+        double ssp = 0.0;
+        if (lane < 16) {
+          float y = 0.0f;
+          for (int j = 0; j < k; ++j) y = fmaf(st->gate[j], ytmp[j * 16 + lane], y);  // slot order
+          const float z = xs[r0 + lane] + y;
+          st->ztmp[lane] = z;
+          a.zbuf[(size_t)(par ^ 1) * H + r0 + lane] = z;
+          ssp = (double)z * (double)z;
+        }
+        ssp = warp_sum_d(ssp);
+        if (lane == 0) atomicAdd(&a.ssacc[par ^ 1], to_fixed(ssp));
+      }
+      named_barrier_sync(CONS_BAR, nth);
+      if (ok && l + 1 < L) {
+        if (mbar_wait(wrtbar, (uint32_t)((l + 1) & 1), clock64() + WAIT_BUDGET_CYCLES)) {
+          unsigned long long *la = a.lacc + (size_t)(par ^ 1) * E;
+          for (int e = tid; e < E; e += nth) {
+            double p = 0.0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) p = fma((double)wrtbuf[i * E + e], (double)st->ztmp[i], p);
+            atomicAdd(la + e, to_fixed(p));
+          }
+        } else {
+          set_status(a.status, DEV_TIMEOUT);
+          *(volatile int *)&st->abort = 1;
+        }
+      }
+    }
+    cons_grid_barrier(a, st, tid);
+  }
+
+  if (producer) {
+    // never leave with copies in flight (only after an abort can any remain)
+    if (lane < S && *(volatile int *)&st->abort) {
+      const long long dl = clock64() + WAIT_BUDGET_CYCLES;
+      for (int n = nring + lane - S; n < nring; n += S)
+        if (n >= 0)
+          while (!mbar_try_wait(&full[n % S], (uint32_t)((n / S) & 1)))
+            if (clock64() > dl) break;
+    }
+    return;
+  }
+  if (*(volatile int *)&st->abort) return;
+  // ---------------------------------------------------------------- output --
+  if (rows && tid < 16) {
+    const double ss = from_fixed(__ldcg(&a.ssacc[L & 1]));
+    const float inv = (float)(1.0 / sqrt(ss / (double)H + (double)a.eps));
+    a.x_out[r0 + tid] = __ldcg(a.zbuf + (size_t)(L & 1) * H + r0 + tid) * inv;
+  }
+  // leave lacc[0] clear for the next launch's layer-0 partials (its last
+  // reader finished long before the last barrier)
+  for (int e = c * nth + tid; e < E; e += G * nth) a.lacc[e] = 0ull;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- host side --
+struct FusedPlan {
+  size_t smem;
+  int nslots, slot_bytes;
+};
+
+// Can the fused kernel run this stack? Fills the launch plan when it can.
+bool fused_stack_plan(int fmt, int E, int H, int I, int k, FusedPlan *p) {
+  if (k > SK_MAXK || E > 1024 || H / 16 > num_sms() || H % 128 || I % 128) return false;
+  const int slot = (int)al128((size_t)tile_bytes(fmt, H));
+  const size_t cap = max_smem_optin();
+  for (int S = 12; S >= 4; --S) {
+    const SkLayout o = sk_layout(fmt, E, H, I, k, S, slot);
+    if (o.total <= cap && (size_t)2 * k * I * 4 <= (size_t)S * slot) {  // D stages a_g, a_u in the ring
+      p->smem = o.total;
+      p->nslots = S;
+      p->slot_bytes = slot;
+      return true;
+    }
+  }
+  return false;
+}
+
+size_t fused_stack_ws_bytes(int L, int E, int H, int I, int k) {
+  auto a = [](size_t v) { return (v + 255) & ~(size_t)255; };
+  return a((size_t)L * H * E * 4) + a(2 * (size_t)E * 8) + 256 + a(2 * (size_t)H * 4) + a(2 * (size_t)k * I * 4) + 256 +
+         3 * a((size_t)L * 8);
+}
+
+struct FusedBufs {
+  float *wrt;
+  unsigned long long *lacc, *ssacc;
+  float *zbuf, *hbuf;
+  unsigned *bar;
+  const uint8_t **gu, **dn;
+  const float **bias;
+};
+
+FusedBufs fused_carve(void *ws, int L, int E, int H, int I, int k) {
+  auto a = [](size_t v) { return (v + 255) & ~(size_t)255; };
+  char *p = static_cast<char *>(ws);
+  FusedBufs b;
+  b.wrt = reinterpret_cast<float *>(p); p += a((size_t)L * H * E * 4);
+  b.lacc = reinterpret_cast<unsigned long long *>(p); p += a(2 * (size_t)E * 8);
+  b.ssacc = reinterpret_cast<unsigned long long *>(p); p += 256;
+  b.zbuf = reinterpret_cast<float *>(p); p += a(2 * (size_t)H * 4);
+  b.hbuf = reinterpret_cast<float *>(p); p += a(2 * (size_t)k * I * 4);
+  b.bar = reinterpret_cast<unsigned *>(p); p += 256;
+  b.gu = reinterpret_cast<const uint8_t **>(p); p += a((size_t)L * 8);
+  b.dn = reinterpret_cast<const uint8_t **>(p); p += a((size_t)L * 8);
+  b.bias = reinterpret_cast<const float **>(p);
+  return b;
+}
+
+namespace {
+__global__ void transpose_router(const float *Wr, float *WrT, int E, int H) {
+  __shared__ float t[32][33];
+  const int e0 = blockIdx.y * 32, h0 = blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y)
+    if (e0 + i < E) t[i][threadIdx.x] = Wr[(size_t)(e0 + i) * H + h0 + threadIdx.x];
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y)
+    if (e0 + threadIdx.x < E) WrT[(size_t)(h0 + i) * E + e0 + threadIdx.x] = t[threadIdx.x][i];
+}
+}  // namespace
+
+// Prepare the fused buffers (transposed routers, pointer tables); called once
+// at stack creation on `s`.
+qmoe_status fused_prepare(const FusedBufs &b, int L, int E, int H, const float *const *Wr,
+                          const qmoe_experts *layers, const float *const *bias, cudaStream_t s) {
+  for (int l = 0; l < L; ++l) {
+    transpose_router<<<dim3(H / 32, (E + 31) / 32), dim3(32, 8), 0, s>>>(Wr[l], b.wrt + (size_t)l * H * E, E, H);
+    note_launch();
+  }
+  std::vector<const void *> gu(L), dn(L), bi(L);
+  for (int l = 0; l < L; ++l) {
+    gu[l] = layers[l].gate_up;
+    dn[l] = layers[l].down;
+    bi[l] = bias ? bias[l] : nullptr;
+  }
+  if (cudaMemcpyAsync((void *)b.gu, gu.data(), L * 8, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync((void *)b.dn, dn.data(), L * 8, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync((void *)b.bias, bi.data(), L * 8, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return QMOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return QMOE_ERR_CUDA;
+  return cuda_status(cudaGetLastError());
+}
+
+qmoe_status fused_launch(const FusedBufs &b, const FusedPlan &p, int fmt, int L, int E, int H, int I, int k, float eps,
+                         const float *x_in, float *x_out, int32_t *idx_rec, float *gate_rec, int32_t *status,
+                         cudaStream_t s, bool cooperative) {
+  StackArgs a{};
+  a.L = L; a.E = E; a.H = H; a.I = I; a.k = k; a.eps = eps;
+  a.gu = b.gu; a.dn = b.dn; a.bias = b.bias; a.wrt = b.wrt;
+  a.x_in = x_in; a.x_out = x_out; a.idx_rec = idx_rec; a.gate_rec = gate_rec;
+  a.zbuf = b.zbuf; a.lacc = b.lacc; a.ssacc = b.ssacc; a.hbuf = b.hbuf; a.bar = b.bar; a.status = status;
+  a.nslots = p.nslots; a.slot_bytes = p.slot_bytes;
+  // Gate/up units are split evenly: the h barrier waits for the slowest CTA's
+  // gate/up tiles, while the row owners' down tiles and router rows are only
+  // needed after it and stream in behind the gate/up work.
+  const int G = num_sms();
+  a.w_rows = 1;
+  a.w_free = 1;
+  const void *fn = fmt == 2 ? (const void *)stack_decode_kernel<2> : (const void *)stack_decode_kernel<4>;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) != cudaSuccess)
+    return QMOE_ERR_CUDA;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)G);
+  cfg.blockDim = dim3(SK_THREADS);
+  cfg.dynamicSmemBytes = p.smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = cooperative ? 1 : 0;
+  cudaError_t e = fmt == 2 ? cudaLaunchKernelEx(&cfg, stack_decode_kernel<2>, a)
+                           : cudaLaunchKernelEx(&cfg, stack_decode_kernel<4>, a);
+  note_launch();
+  return cuda_status(e);
+}
+
+}  // namespace qmoe

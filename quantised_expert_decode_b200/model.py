@@ -40,7 +40,8 @@ class PackedLayer:
 class DecodeStack:
     """L layers of route -> FFN -> residual RMSNorm as one CUDA graph."""
 
-    def __init__(self, layers, routers, biases, T: int, k: int, eps: float, stream=None, timing: bool = False):
+    def __init__(self, layers, routers, biases, T: int, k: int, eps: float, stream=None, timing: bool = False,
+                 layerwise: bool = False):
         self.layers, self.routers, self.biases = list(layers), list(routers), biases
         self.L, self.T, self.k = len(self.layers), T, k
         self.H = self.layers[0].H
@@ -51,7 +52,7 @@ class DecodeStack:
         else:
             self._bias = None
         self.desc = L.qmoe_stack_desc(self.L, T, k, eps, self._wr, self._bias, self._handles,
-                                      L.STACK_TIMING if timing else 0)
+                                      (L.STACK_TIMING if timing else 0) | (L.STACK_LAYERWISE if layerwise else 0))
         nbytes = L.qmoe_stack_workspace_bytes(self.desc)
         if nbytes == 0:
             raise L.QmoeError("qmoe_stack_workspace_bytes", 1)
@@ -73,6 +74,7 @@ class DecodeStack:
         self.gate = view(bufs["gate"], self.L * T * k, torch.float32).view(self.L, T, k)
         self.dev_status = view(bufs["dev_status"], 1, torch.int32)
         self.kernels_per_replay = L.qmoe_stack_kernels_per_replay(self.handle)
+        self.path = L.qmoe_stack_path(self.handle)
 
     def decode(self, stream=None) -> None:
         L.qmoe_stack_decode(self.handle, stream)

@@ -49,9 +49,9 @@ def _compare(cfg, stack, x0_np, n_layers):
     return err
 
 
-def _run(cfg, n_layers, step=0):
-    layers, routers, biases = device_layers(SEED, cfg, n_layers)
-    stack = DecodeStack(layers, routers, biases, cfg.T, cfg.k, cfg.eps)
+def _run(cfg, n_layers, step=0, layerwise=False, built=None):
+    layers, routers, biases = built if built else device_layers(SEED, cfg, n_layers)
+    stack = DecodeStack(layers, routers, biases, cfg.T, cfg.k, cfg.eps, layerwise=layerwise)
     x0 = gen.tokens(SEED, cfg, step)
     stack.x_in.copy_(torch.from_numpy(x0))
     stack.decode()
@@ -60,11 +60,13 @@ def _run(cfg, n_layers, step=0):
     return stack, x0, layers
 
 
-def test_stack_small_geometry():
+@pytest.mark.parametrize("layerwise", [False, True])
+def test_stack_small_geometry(layerwise):
     cfg = configs.get(0).with_(L=6, residual=True)
-    stack, x0, _ = _run(cfg, 6)
+    stack, x0, _ = _run(cfg, 6, layerwise=layerwise)
     _compare(cfg, stack, x0, 6)
-    assert stack.kernels_per_replay == 13
+    assert stack.path == (0 if layerwise else 1)
+    assert stack.kernels_per_replay == (13 if layerwise else 1)
     # host-buffer entry point gives the same answer as the device-buffer replay
     xh = torch.from_numpy(x0).pin_memory()
     out = torch.empty_like(xh).pin_memory()
@@ -91,6 +93,15 @@ def test_stack_48_layers_q2_single_token():
     stack.decode()
     torch.cuda.synchronize()
     _compare(cfg, stack, x1, cfg.L)
+    # the per-layer kernel path routes identically and agrees to fp32 roundoff
+    lw = DecodeStack(layers, stack.routers, None, cfg.T, cfg.k, cfg.eps, layerwise=True)
+    lw.x_in.copy_(torch.from_numpy(x1))
+    lw.decode()
+    torch.cuda.synchronize()
+    assert stack.path == 1 and lw.path == 0
+    assert torch.equal(lw.idx, stack.idx)
+    assert moe.rel_rms(to_np(lw.x_out), to_np(stack.x_out)) < 1e-5
+    lw.close()
     stack.close()
 
 
