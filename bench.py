@@ -27,8 +27,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE decode tokens/s over 48 layers; HBM GB/s on weight bytes vs peak"
+PREFILL_METRIC = "MoE prefill tokens/s (4096-token bf16 chunk, one 512-expert Q4 layer); tensor TFLOP/s vs peak"
 SEED = 0
-WORKLOADS = {"decode48": 2, "verify48": 3, "layer": 1}
+WORKLOADS = {"decode48": 2, "verify48": 3, "layer": 1, "prefill": 4}
 
 
 def parse():
@@ -49,6 +50,16 @@ def peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def tensor_peak():
+    """Dense bf16 TFLOP/s: the sustained figure (kernels timed inside a long loop)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured (sustained)"
+    return 1400.0, "fallback (sustained)"
 
 
 def workload_desc(cfg, T):
@@ -477,12 +488,212 @@ def run_layer(args, cfg):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- prefill --
+def prefill_desc(cfg):
+    return {"workload": f"prefill chunk: {cfg.T} bf16 tokens through one {cfg.E}-expert layer, hidden {cfg.H}, "
+                        f"intermediate {cfg.I}, top-{cfg.k}, Q{cfg.fmt} blocks, biased router",
+            "tokens_per_step": cfg.T, "experts": cfg.E, "hidden": cfg.H, "intermediate": cfg.I, "top_k": cfg.k,
+            "format": f"Q{cfg.fmt}", "seed": SEED,
+            "l2": "no flush: each step streams the ~1 GB of Q4 weights of its active experts (> 126 MB L2); "
+                  "4 distinct activation draws rotate between steps"}
+
+
+def prefill_flops(cfg, pairs):
+    return 2.0 * 3 * cfg.H * cfg.I * pairs, 2.0 * 2 * cfg.H * cfg.I * pairs   # layer, GEMM 1
+
+
+def oracle_prefill_time(cfg, n_tok):
+    """Seconds per token of the float64 oracle: routing of the whole chunk
+    (charged per token) plus expert FFNs and combine of n_tok tokens."""
+    import numpy as np
+    from oracle import moe
+    from oracle import workload as W
+    x = W.x_float(SEED, cfg)
+    Wr, b = gen_router_bias(cfg)
+    t0 = time.perf_counter()
+    idx, g, _ = moe.route(x, Wr, b, cfg.k)
+    t_route = time.perf_counter() - t0
+    from synth import gen
+    rows = np.arange(n_tok)
+    raw = {int(e): gen.expert(SEED, cfg, 0, int(e)) for e in set(idx[rows].ravel().tolist())}
+    bits = cfg.format.bits
+    t0 = time.perf_counter()
+
+    def get(e):
+        r = raw[e]
+        return tuple(moe.dequantize(r[n + "_codes"], r[n + "_scales"], bits) for n in ("gate", "up", "down"))
+    moe.moe_layer(x[rows], idx[rows], g[rows], get)
+    t_ffn = time.perf_counter() - t0
+    return t_route / cfg.T + t_ffn / n_tok, t_route, t_ffn
+
+
+def gen_router_bias(cfg):
+    from synth import gen
+    return gen.router(SEED, cfg, 0), gen.bias(SEED, cfg, 0)
+
+
+def run_prefill_reference(args, cfg):
+    """The oracle as the reference arm: each step runs it on a bounded sample of
+    the chunk (routing of all tokens, FFNs of 8 tokens), scaled per token; at
+    most 2 timed steps and 1 warm-up step so the run stays within minutes."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    n_tok, steps, warm = 8, max(1, min(args.steps, 2)), min(args.warmup, 1)
+    for _ in range(warm):
+        oracle_prefill_time(cfg, n_tok)
+    per = [oracle_prefill_time(cfg, n_tok)[0] for _ in range(steps)]
+    per_tok = statistics.mean(per)
+    value = 1.0 / per_tok
+    line = {"impl": "reference", "metric": PREFILL_METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": steps, "warmup": warm, "ms_per_step": 1e3 * per_tok * cfg.T,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": prefill_desc(cfg),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"per step: routing of all {cfg.T} tokens (charged per token) + expert FFNs "
+                                       f"and combine of {n_tok} tokens; weight generation excluded"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_prefill(args, cfg):
+    import numpy as np
+    import torch
+
+    import quantised_expert_decode_b200 as q
+    from quantised_expert_decode_b200 import _lib as L
+    from synth import gen
+    from synth.workload import device_layers
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+    T, k, E, H, I = cfg.T, cfg.k, cfg.E, cfg.H, cfg.I
+    layers, routers, biases = device_layers(SEED, cfg, 1)
+    layer, Wr, bias = layers[0], routers[0], biases[0]
+    n_in = 4
+    xs_host = [gen.tokens(SEED + 1000 * rank, cfg, s).view(np.int16) for s in range(n_in)]
+    xs = [torch.from_numpy(a).cuda().view(torch.bfloat16) for a in xs_host]
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    gate = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    y = torch.empty((T, H), dtype=torch.float32, device="cuda")
+    rws = torch.zeros(q.qmoe_route_workspace_bytes(T, E), dtype=torch.uint8, device="cuda")
+    pws = torch.empty(q.qmoe_prefill_workspace_bytes(T, k, E, H, I), dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for es in ev:
+        for e in es:
+            e.record(stream)
+    h = layer.handle()
+
+    def step(s, events=None):
+        x = xs[s % n_in]
+        q.qmoe_route(Wr, bias, x, L.BF16, T, H, E, k, idx, gate, rws, st, stream)
+        if events is None:
+            q.qmoe_ffn_prefill(h, x, T, idx, gate, k, y, pws, st, stream)
+        else:
+            q.qmoe_ffn_prefill_timed(h, x, T, idx, gate, k, y, pws, st, events, stream)
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError("device status set during warm-up")
+    props = torch.cuda.get_device_properties(local)
+    clocks = Clocks(getattr(props, "uuid", None) and f"GPU-{props.uuid}")
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = q.qmoe_launch_count()
+    e0.record(stream)
+    for s in range(args.steps):
+        step(args.warmup + s, ev[s])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = q.qmoe_launch_count() - n0
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    clk = clocks.stop()
+    if int(st.item()) != 0:
+        raise RuntimeError("device status set during the timed run")
+    g1_ms = [es[0].elapsed_time(es[1]) for es in ev]
+    g2_ms = [es[1].elapsed_time(es[2]) for es in ev]
+    value = world * args.steps * T / (ms / 1e3)
+
+    # end to end: pinned bf16 x -> device, route + FFN, y -> pinned host
+    xh = [torch.from_numpy(a).pin_memory() for a in xs_host]
+    yh = torch.empty((T, H), dtype=torch.float32).pin_memory()
+    xdev = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    torch.cuda.synchronize()
+    barrier(world)
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for s in range(args.steps):
+        xdev.copy_(xh[s % n_in], non_blocking=True)
+        xb = xdev.view(torch.bfloat16)
+        q.qmoe_route(Wr, bias, xb, L.BF16, T, H, E, k, idx, gate, rws, st, stream)
+        q.qmoe_ffn_prefill(h, xb, T, idx, gate, k, y, pws, st, stream)
+        yh.copy_(y, non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(e2.elapsed_time(e3), world)
+
+    peak, peak_kind = tensor_peak()
+    pairs = T * k
+    f_layer, f_g1 = prefill_flops(cfg, pairs)
+    f_g2 = f_layer - f_g1
+    t1, t2 = statistics.mean(g1_ms) / 1e3, statistics.mean(g2_ms) / 1e3
+    counts = np.bincount(idx.cpu().numpy().ravel(), minlength=E)
+    padded = int(sum((c + 15) // 16 * 16 for c in counts))
+    a1 = f_g1 / t1 / 1e12
+    line = {
+        "metric": PREFILL_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 x bf16 -> f32 (tcgen05, Q4 weights dequantised in shared memory), f64 router",
+        "data": "synthetic (seeded SplitMix64 weights, Box-Muller bf16 activations, N(0,1) router bias)",
+        "config": dict(prefill_desc(cfg), parallelism=f"replicas x{world}"),
+        "roofline": {"bound": "tensor", "kernel": "pf_gemm_kernel (grouped GEMM 1: gate/up + SiLU*up epilogue)",
+                     "achieved": a1, "peak": peak, "peak_kind": peak_kind, "unit": "TFLOP/s", "frac": a1 / peak,
+                     "traffic": None, "algorithmic_flops_per_launch": f_g1, "avg_launch_us": 1e6 * t1,
+                     "timing": "CUDA events recorded on the launching stream around each GEMM launch"},
+        "prefill": {"gemm2_TFLOPs": f_g2 / t2 / 1e12, "gemm2_frac": f_g2 / t2 / 1e12 / peak,
+                    "gemm2_us": 1e6 * t2, "ffn_gemms_frac": f_layer / (t1 + t2) / 1e12 / peak,
+                    "layer_TFLOPs_per_step": f_layer / (ms / 1e3 / args.steps) / 1e12,
+                    "pairs": pairs, "active_experts": int((counts > 0).sum()), "max_expert_load": int(counts.max()),
+                    "mma_columns_padded_over_pairs": padded / pairs},
+        "e2e": {"value": world * args.steps * T / (ms_e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 4,
+                "path": "pinned bf16 x -> device, qmoe_route + qmoe_ffn_prefill, y -> pinned host"},
+        "clocks": clk,
+        "gpu_launches": launches,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        per_tok, tr, tf = oracle_prefill_time(cfg, 16)
+        line["cpu_baseline"] = {"value": 1.0 / per_tok, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"routing of all {T} tokens ({tr:.1f} s, charged per token) + expert FFNs "
+                                          f"and combine of 16 tokens ({tf:.1f} s); weight generation excluded"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     from synth import configs
     cfg = configs.get(WORKLOADS[args.workload])
-    if args.impl == "reference":
+    if args.impl == "reference" and args.workload == "prefill":
+        run_prefill_reference(args, cfg)
+    elif args.impl == "reference":
         run_reference(args, cfg, cfg.T)
+    elif args.workload == "prefill":
+        run_prefill(args, cfg)
     elif args.workload == "layer":
         run_layer(args, cfg)
     else:

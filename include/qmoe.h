@@ -116,9 +116,10 @@ qmoe_status qmoe_pack(int fmt, int kind, int E, int H, int I,
  * gate fp32 [T,k]. Workspace: qmoe_route_workspace_bytes(T, E) bytes, zeroed
  * once before first use (it is left zeroed by every completed call).
  * Limits: 1 <= k <= 16, k <= E <= 1024, H multiple of 128, T >= 1.
- * T <= 8 runs the single-pass decode router (float64 GEMV); larger T runs the
- * prefill router (fp32 tiles with a per-token rounding bound; tokens whose
- * ordering the bound cannot certify are recomputed in float64). */
+ * T <= 8 with fp32 x runs the single-pass decode router (float64 GEMV); larger
+ * T or bf16 x runs the prefill router (a float64 logit GEMM over register
+ * tiles into the workspace, then one warp per token for the selection). Both
+ * form every product exactly in float64 and sum in float64. */
 size_t qmoe_route_workspace_bytes(int T, int E);
 qmoe_status qmoe_route(const float *Wr, const float *bias, const void *x, int x_dtype,
                        int T, int H, int E, int k, int32_t *idx, float *gate,
@@ -163,6 +164,50 @@ qmoe_status qmoe_ffn_decode(const qmoe_experts *experts, const float *x, int T,
                             const int32_t *idx, const float *gate, int k, float *y,
                             void *workspace, size_t workspace_bytes, int32_t *dev_status,
                             qmoe_stream_t stream);
+
+/* -------------------------------------------------------------- bucketing --
+ * Token -> expert bucketing of a route (the routed pairs regrouped per expert
+ * so each expert's weights are read once per chunk; [P3] batched prefill,
+ * "Understanding the Architecture"). Pairs are numbered p = t*k + j. A stable
+ * counting sort orders them by (expert, t, j):
+ *   offsets int32 [E+1]: offsets[e] = number of pairs routed to experts < e
+ *   perm    int32 [T*k]: perm[offsets[e] + i] = i-th pair (in pair order) of e
+ *   active  int32 [E] or NULL: experts with at least one pair, ascending
+ *   nactive int32 [1] or NULL: their count
+ * Limits: E <= 1024, T*k <= 2^30. One CTA; an index outside [0, E) sets the
+ * device status and leaves the outputs unwritten. */
+qmoe_status qmoe_bucket(const int32_t *idx, int T, int k, int E, int32_t *offsets, int32_t *perm,
+                        int32_t *active, int32_t *nactive, int32_t *dev_status, qmoe_stream_t stream);
+
+/* ------------------------------------------------------------- prefill FFN --
+ * Routed expert FFN for prefill chunks of many tokens ([P3] batched prefill in
+ * chunks of up to 8,192 tokens, "Understanding the Architecture"), computing
+ * the same function as qmoe_ffn_decode on bf16 activations:
+ *   y[t,:] = sum_j gate[t,j] * Wd_e (silu(Wg_e x_t) * (Wu_e x_t)),  e = idx[t,j]
+ * x bf16 [T,H]; idx int32 [T,k]; gate fp32 [T,k]; y fp32 [T,H] (overwritten).
+ * Steps (all on `stream`): bucketing by expert, a tile plan, then two grouped
+ * GEMMs on the tcgen05 tensor cores - bf16 operands (Q4 weights dequantised
+ * to bf16 in shared memory, w = bf16(d)*q + bf16(m) rounded once), fp32
+ * accumulation in tensor memory; the intermediate silu(g)*u is rounded to
+ * bf16 between the two GEMMs; the gate-weighted combine is a sum of fp32
+ * atomic additions, so its order (and the last bits of y) may vary between
+ * runs. Expected relative error against exact arithmetic: about 1e-3.
+ * Limits: fmt Q4, H a multiple of 256, I a multiple of 128, k <= E <= 1024,
+ * T*k <= 2^28. Workspace: qmoe_prefill_workspace_bytes(T, k, E, H, I) bytes,
+ * no initialisation needed. *dev_status must be 0 on entry (a nonzero value
+ * skips the GEMMs); an index outside [0, E) or an expert repeated within one
+ * token's route sets it. */
+size_t qmoe_prefill_workspace_bytes(int T, int k, int E, int H, int I);
+qmoe_status qmoe_ffn_prefill(const qmoe_experts *experts, const void *x, int T, const int32_t *idx,
+                             const float *gate, int k, float *y, void *workspace, size_t workspace_bytes,
+                             int32_t *dev_status, qmoe_stream_t stream);
+/* qmoe_ffn_prefill with kernel timing: events is a host array of three
+ * cudaEvent_t (created by the caller, timing enabled) recorded on `stream`
+ * right before the first grouped GEMM, between the two, and after the second;
+ * cudaEventElapsedTime of consecutive pairs gives the two GEMM durations. */
+qmoe_status qmoe_ffn_prefill_timed(const qmoe_experts *experts, const void *x, int T, const int32_t *idx,
+                                   const float *gate, int k, float *y, void *workspace, size_t workspace_bytes,
+                                   int32_t *dev_status, qmoe_stream_t stream, void *const *events);
 
 /* ------------------------------------------------------------ layer stack --
  * L layers of route -> FFN -> residual RMSNorm captured once into one CUDA

@@ -53,6 +53,11 @@ _SIGS = {
     "qmoe_rmsnorm_residual": (_I, [_VP, _VP, _F, _VP, _I, _I, _VP]),
     "qmoe_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "qmoe_ffn_decode": (_I, [ctypes.POINTER(qmoe_experts), _VP, _I, _VP, _VP, _I, _VP, _VP, _SZ, _VP, _VP]),
+    "qmoe_bucket": (_I, [_VP, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "qmoe_prefill_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
+    "qmoe_ffn_prefill": (_I, [ctypes.POINTER(qmoe_experts), _VP, _I, _VP, _VP, _I, _VP, _VP, _SZ, _VP, _VP]),
+    "qmoe_ffn_prefill_timed": (_I, [ctypes.POINTER(qmoe_experts), _VP, _I, _VP, _VP, _I, _VP, _VP, _SZ, _VP, _VP,
+                                    ctypes.POINTER(_VP)]),
     "qmoe_stack_workspace_bytes": (_SZ, [ctypes.POINTER(qmoe_stack_desc)]),
     "qmoe_stack_create": (_I, [ctypes.POINTER(qmoe_stack_desc), _VP, _SZ, _VP, ctypes.POINTER(_VP)]),
     "qmoe_stack_destroy": (_I, [_VP]),
@@ -154,6 +159,30 @@ def qmoe_ffn_decode(experts: qmoe_experts, x, T, idx, gate, k, y, workspace, dev
     _check("qmoe_ffn_decode", lib().qmoe_ffn_decode(
         ctypes.byref(experts), _p(x), T, _p(idx), _p(gate), k, _p(y), _p(workspace),
         workspace.numel() * workspace.element_size(), _p(dev_status), _s(stream)))
+
+
+def qmoe_bucket(idx, T, k, E, offsets, perm, active, nactive, dev_status, stream=None) -> None:
+    _check("qmoe_bucket", lib().qmoe_bucket(_p(idx), T, k, E, _p(offsets), _p(perm), _p(active), _p(nactive),
+                                            _p(dev_status), _s(stream)))
+
+
+def qmoe_prefill_workspace_bytes(T: int, k: int, E: int, H: int, I: int) -> int:
+    return lib().qmoe_prefill_workspace_bytes(T, k, E, H, I)
+
+
+def qmoe_ffn_prefill(experts: qmoe_experts, x, T, idx, gate, k, y, workspace, dev_status, stream=None) -> None:
+    _check("qmoe_ffn_prefill", lib().qmoe_ffn_prefill(
+        ctypes.byref(experts), _p(x), T, _p(idx), _p(gate), k, _p(y), _p(workspace),
+        workspace.numel() * workspace.element_size(), _p(dev_status), _s(stream)))
+
+
+def qmoe_ffn_prefill_timed(experts: qmoe_experts, x, T, idx, gate, k, y, workspace, dev_status, events,
+                           stream=None) -> None:
+    """``events``: three torch.cuda.Event(enable_timing=True) objects."""
+    arr = (_VP * 3)(*[e.cuda_event for e in events])
+    _check("qmoe_ffn_prefill_timed", lib().qmoe_ffn_prefill_timed(
+        ctypes.byref(experts), _p(x), T, _p(idx), _p(gate), k, _p(y), _p(workspace),
+        workspace.numel() * workspace.element_size(), _p(dev_status), _s(stream), arr))
 
 
 def qmoe_stack_workspace_bytes(desc: qmoe_stack_desc) -> int:

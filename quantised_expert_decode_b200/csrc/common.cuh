@@ -141,6 +141,22 @@ __device__ __forceinline__ double warp_sum_d(double v) {
   return v;
 }
 
+// Inclusive warp scan of three counters at once.
+__device__ __forceinline__ void warp_scan3(int &a, int &b, int &c) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, a, o);
+    const int y = __shfl_up_sync(0xffffffffu, b, o);
+    const int z = __shfl_up_sync(0xffffffffu, c, o);
+    if (lane >= o) {
+      a += x;
+      b += y;
+      c += z;
+    }
+  }
+}
+
 // Orderable unsigned key of a float (larger float -> larger key; every key > 0
 // for non-NaN input; 0 marks "no value").
 __device__ __forceinline__ unsigned float_key(float f) {

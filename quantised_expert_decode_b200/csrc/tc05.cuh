@@ -1,0 +1,103 @@
+// Fifth-generation tensor core (tcgen05) primitives for sm_100a: tensor
+// memory allocation, shared-memory matrix descriptors, the bf16 MMA with fp32
+// accumulation in tensor memory, completion tracking and accumulator loads.
+#pragma once
+
+#include "common.cuh"
+
+namespace qmoe {
+namespace tc05 {
+
+// ------------------------------------------------------------ tensor memory --
+// Allocation is warp-wide (.sync.aligned): the whole warp calls these. The
+// allocated base address (lane 0, first column) is written to *dst in shared
+// memory. ncols: a power of two in [32, 512].
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Ordering of tcgen05 operations across a thread synchronisation (mbarrier
+// or bar.sync): "before" in the thread that signals, "after" in the one that
+// waits.
+__device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy reads (tensor-core operand fetches) of the same bytes.
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// ------------------------------------------------------------- descriptors --
+// Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzle
+// layout: rows of 64 bf16 (128 bytes) at a 128-byte pitch, groups of 8 rows
+// (1024 bytes, the swizzle atom) at a 1024-byte pitch, and inside each row the
+// 16-byte chunk c stored at chunk position c ^ (row % 8). The operand base must
+// be 1024-byte aligned; the start address of the K-slice kk (16 elements) is
+// base + 32*kk.
+//   bits [0,14) start >> 4 | [16,30) leading offset >> 4 (unused here, 1)
+//   [32,46) stride offset >> 4 (1024 bytes) | [46,48) version 1
+//   [49,52) base offset 0 | [61,64) layout 2 = 128-byte swizzle
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
+// Instruction descriptor of kind::f16 with bf16 A and B (both K-major) and an
+// fp32 accumulator, shape M x N:
+//   [4,6) c format 1 = f32 | [7,10) a format 1 = bf16 | [10,13) b format 1 = bf16
+//   [15] a major 0 = K | [16] b major 0 = K | [17,23) N >> 3 | [24,29) M >> 4
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread. accumulate = 0
+// overwrites D.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  const uint32_t z = 0;
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p; }" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(z)
+      : "memory");
+}
+
+// Makes *bar track completion of every tcgen05 operation this thread issued
+// so far; the barrier receives one arrival when they have completed.
+__device__ __forceinline__ void commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+// Warp-wide load of 16 consecutive 32-bit columns from the warp's 32-lane
+// quadrant: thread i receives lane (taddr.lane + i), columns taddr.col .. +15.
+// The wait for completion is part of the same statement, so the compiler
+// cannot schedule a use of the registers before the data has arrived.
+__device__ __forceinline__ void ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+}  // namespace tc05
+}  // namespace qmoe

@@ -97,6 +97,42 @@ def test_ffn_decode_argument_checks_without_gpu():
     assert call(ex=bad) == 2
 
 
+def test_prefill_argument_checks_without_gpu():
+    lib = q.lib()
+    def ex_(E, H, I, fmt, gu=FAKE, dn=FAKE):
+        return L.qmoe_experts(E, H, I, fmt, gu, dn, q.qmoe_packed_bytes(fmt, 0, E, H, I),
+                              q.qmoe_packed_bytes(fmt, 1, E, H, I))
+    T, k = 4096, 10
+    ex = ex_(512, 2048, 768, L.Q4)
+    wsb = q.qmoe_prefill_workspace_bytes(T, k, 512, 2048, 768)
+    # h rows (T*k + 15*E) x I bf16 dominate the workspace
+    assert wsb >= (T * k + 15 * 512) * 768 * 2
+    assert q.qmoe_prefill_workspace_bytes(0, k, 512, 2048, 768) == 0
+
+    def call(ex=ex, T=T, k=k, wsb=wsb, x=FAKE, idx=FAKE, y=FAKE):
+        return lib.qmoe_ffn_prefill(ctypes.byref(ex), x, T, idx, FAKE, k, y, FAKE, wsb, FAKE, None)
+
+    assert call(x=None) == 1
+    assert call(T=0) == 1
+    assert call(x=FAKE + 8) == 1                            # bf16 rows must be 16-byte aligned
+    assert call(idx=FAKE + 2) == 1
+    assert call(ex=ex_(512, 2048, 768, L.Q2)) == 3          # Q2 prefill is not built
+    assert call(ex=ex_(512, 2048 + 128, 768, L.Q4)) == 3    # H must be a multiple of 256
+    assert call(k=600) == 3
+    assert call(wsb=wsb - 256) == 4
+    bad = ex_(512, 2048, 768, L.Q4)
+    bad.I = 640                                             # sizes no longer match the geometry
+    assert call(ex=bad) == 2
+
+
+def test_bucket_argument_checks_without_gpu():
+    lib = q.lib()
+    assert lib.qmoe_bucket(None, 8, 2, 16, FAKE, FAKE, None, None, FAKE, None) == 1
+    assert lib.qmoe_bucket(FAKE, 0, 2, 16, FAKE, FAKE, None, None, FAKE, None) == 1
+    assert lib.qmoe_bucket(FAKE, 8, 2, 4096, FAKE, FAKE, None, None, FAKE, None) == 3
+    assert lib.qmoe_bucket(FAKE + 2, 8, 2, 16, FAKE, FAKE, None, None, FAKE, None) == 1
+
+
 def test_pack_and_norm_argument_checks_without_gpu():
     lib = q.lib()
     assert lib.qmoe_pack(3, 0, 4, 256, 128, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == 3
