@@ -40,6 +40,8 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="decode48", choices=sorted(WORKLOADS))
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--tokens", type=int, default=None,
+                   help="prefill workload only: tokens per chunk (default: the workload's 4096)")
     return p.parse_args()
 
 
@@ -688,6 +690,8 @@ def main():
     args = parse()
     from synth import configs
     cfg = configs.get(WORKLOADS[args.workload])
+    if args.workload == "prefill" and args.tokens:
+        cfg = cfg.with_(T=args.tokens)
     if args.impl == "reference" and args.workload == "prefill":
         run_prefill_reference(args, cfg)
     elif args.impl == "reference":
