@@ -142,6 +142,30 @@ qmoe_status qmoe_residual_route(const float *x_in, const float *y, float eps, fl
 qmoe_status qmoe_rmsnorm_residual(const float *x_in, const float *y, float eps, float *x_out,
                                   int T, int H, qmoe_stream_t stream);
 
+/* ----------------------------------------------------- router, fixed scratch --
+ * qmoe_route for callers that cannot allocate device memory for a workspace:
+ * a host program that owns only its input and output buffers and has no
+ * allocator, or a serving loop that may not call into one (an allocation can
+ * synchronise the device). This entry point has no counterpart in the
+ * method's sources; it is an interface convenience of this library.
+ * It runs the same single-pass decode router as qmoe_route with fp32 x, with
+ * its scratch (float64 logits and a 256-byte completion ticket) held in one
+ * fixed device array of QMOE_ROUTE_FIXED_SCRATCH_BYTES bytes inside the
+ * library; nothing is allocated.
+ * Limits: 1 <= T <= QMOE_ROUTE_FIXED_MAX_T, E <= QMOE_ROUTE_FIXED_MAX_E,
+ * 1 <= k <= 16, H a multiple of 128; larger requests return UNSUPPORTED.
+ * The first call on each device looks up the array's address and zeroes it
+ * synchronously (cudaGetSymbolAddress, cudaMemset; the ticket must start at
+ * zero and every completed call leaves it at zero). Make that first call
+ * before capturing any stream. Calls that may run at the same time on one
+ * device (other streams, other host threads) share the array and race: keep
+ * them on one stream. */
+#define QMOE_ROUTE_FIXED_MAX_T 8
+#define QMOE_ROUTE_FIXED_MAX_E 1024
+#define QMOE_ROUTE_FIXED_SCRATCH_BYTES (QMOE_ROUTE_FIXED_MAX_T * QMOE_ROUTE_FIXED_MAX_E * 8 + 256)
+qmoe_status qmoe_route_fixed(const float *Wr, const float *bias, const float *x, int T, int H, int E, int k,
+                             int32_t *idx, float *gate, int32_t *dev_status, qmoe_stream_t stream);
+
 /* -------------------------------------------------------------- decode FFN --
  * Routed expert FFN with the gate-weighted combine on the device ([P3]
  * moe_combine, native_moe.cu, "Understanding the Architecture"; [P1] the

@@ -9,7 +9,7 @@ from ._lib import (BF16, DOWN, F32, GATE_UP, Q2, Q4, QmoeError, exported_symbols
                    qmoe_bucket, qmoe_ffn_prefill, qmoe_ffn_prefill_timed, qmoe_prefill_workspace_bytes,
                    qmoe_decode_workspace_bytes, qmoe_experts, qmoe_ffn_decode, qmoe_launch_count, qmoe_pack,
                    qmoe_packed_bytes, qmoe_read_status, qmoe_residual_route, qmoe_rmsnorm_residual, qmoe_route,
-                   qmoe_route_workspace_bytes, qmoe_stack_buffers, qmoe_stack_create, qmoe_stack_decode,
+                   qmoe_route_fixed, qmoe_route_workspace_bytes, qmoe_stack_buffers, qmoe_stack_create, qmoe_stack_decode,
                    qmoe_stack_decode_host, qmoe_stack_desc, qmoe_stack_destroy, qmoe_stack_kernels_per_replay, qmoe_stack_layer_times,
                    qmoe_stack_path,
                    qmoe_stack_workspace_bytes, qmoe_status_string)

@@ -49,6 +49,7 @@ _SIGS = {
     "qmoe_pack": (_I, [_I, _I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "qmoe_route_workspace_bytes": (_SZ, [_I, _I]),
     "qmoe_route": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _SZ, _VP, _VP]),
+    "qmoe_route_fixed": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _VP, _VP, _VP, _VP]),
     "qmoe_residual_route": (_I, [_VP, _VP, _F, _VP, _VP, _VP, _I, _I, _I, _I, _VP, _VP, _VP, _SZ, _VP, _VP]),
     "qmoe_rmsnorm_residual": (_I, [_VP, _VP, _F, _VP, _I, _I, _VP]),
     "qmoe_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
@@ -137,6 +138,12 @@ def qmoe_route(Wr, bias, x, x_dtype, T, H, E, k, idx, gate, workspace, dev_statu
     _check("qmoe_route", lib().qmoe_route(_p(Wr), _p(bias), _p(x), x_dtype, T, H, E, k, _p(idx), _p(gate),
                                           _p(workspace), workspace.numel() * workspace.element_size(),
                                           _p(dev_status), _s(stream)))
+
+
+def qmoe_route_fixed(Wr, bias, x, T, H, E, k, idx, gate, dev_status, stream=None) -> None:
+    """The decode router with its scratch in a fixed device array (no workspace)."""
+    _check("qmoe_route_fixed", lib().qmoe_route_fixed(_p(Wr), _p(bias), _p(x), T, H, E, k, _p(idx), _p(gate),
+                                                      _p(dev_status), _s(stream)))
 
 
 def qmoe_residual_route(x_in, y, eps, x_out, Wr, bias, T, H, E, k, idx, gate, workspace, dev_status,

@@ -1,6 +1,8 @@
 // Router for decode batches (T <= 8): float64 GEMV over fp32 weights, top-k with
 // ties to the lower expert index, renormalised gates; optionally preceded by
 // the residual RMSNorm of the previous layer's output.
+#include <mutex>
+
 #include "common.cuh"
 #include "route_common.cuh"
 
@@ -248,6 +250,69 @@ extern "C" qmoe_status qmoe_residual_route(const float *x_in, const float *y, fl
   a.ticket = reinterpret_cast<unsigned *>(static_cast<char *>(workspace) + decode_ws_bytes(T, E) - 256);
   a.status = dev_status;
   return launch_route_decode(a, true, (cudaStream_t)stream);
+}
+
+// ----------------------------------------------------------- fixed scratch --
+// The decode router for callers that cannot allocate device memory for a
+// workspace: a host program that owns only its input/output buffers and has
+// no allocator, or a serving loop that may not call into one (an allocation
+// can synchronise the device). The scratch lives in one fixed device array
+// per device, so concurrent calls on one device race for it.
+namespace qmoe {
+namespace {
+
+constexpr size_t FIXED_LOGITS_BYTES = (size_t)QMOE_ROUTE_FIXED_MAX_T * QMOE_ROUTE_FIXED_MAX_E * sizeof(double);
+static_assert(QMOE_ROUTE_FIXED_SCRATCH_BYTES == FIXED_LOGITS_BYTES + 256, "fixed scratch layout");
+
+// [0, FIXED_LOGITS_BYTES): float64 logits; then the 256-byte ticket block,
+// which must start at zero (each completed call leaves it at zero).
+__device__ __align__(256) unsigned char g_route_scratch[QMOE_ROUTE_FIXED_SCRATCH_BYTES];
+
+constexpr int FIXED_MAX_DEVICES = 64;
+std::mutex g_fixed_mutex;
+void *g_fixed_ptr[FIXED_MAX_DEVICES];
+
+// First call on a device: look up the array's address and zero it
+// (synchronous; no allocation). Later calls reuse the address.
+qmoe_status fixed_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QMOE_ERR_CUDA;
+  if (dev < 0 || dev >= FIXED_MAX_DEVICES) return QMOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_fixed_mutex);
+  if (!g_fixed_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) return QMOE_ERR_CUDA;
+    if (cudaMemset(p, 0, QMOE_ROUTE_FIXED_SCRATCH_BYTES) != cudaSuccess) return QMOE_ERR_CUDA;
+    g_fixed_ptr[dev] = p;
+  }
+  *out = g_fixed_ptr[dev];
+  return QMOE_OK;
+}
+
+}  // namespace
+}  // namespace qmoe
+
+extern "C" qmoe_status qmoe_route_fixed(const float *Wr, const float *bias, const float *x, int T, int H, int E, int k,
+                                        int32_t *idx, float *gate, int32_t *dev_status, qmoe_stream_t stream) {
+  if (!Wr || !x || !idx || !gate || !dev_status) return QMOE_ERR_INVALID_ARG;
+  if (!aligned16(Wr) || !aligned16(x)) return QMOE_ERR_INVALID_ARG;
+  if (T < 1 || H < 128 || E < 1 || k < 1) return QMOE_ERR_INVALID_ARG;
+  if (H % 128 || k > 16 || k > E) return QMOE_ERR_UNSUPPORTED;
+  if (T > QMOE_ROUTE_FIXED_MAX_T || E > QMOE_ROUTE_FIXED_MAX_E) return QMOE_ERR_UNSUPPORTED;
+  void *scratch = nullptr;
+  const qmoe_status st = fixed_scratch(&scratch);
+  if (st != QMOE_OK) return st;
+  RouteArgs a{};
+  a.Wr = Wr;
+  a.bias = bias;
+  a.x = x;
+  a.T = T; a.H = H; a.E = E; a.k = k;
+  a.idx = idx;
+  a.gate = gate;
+  a.logits = static_cast<double *>(scratch);
+  a.ticket = reinterpret_cast<unsigned *>(static_cast<char *>(scratch) + FIXED_LOGITS_BYTES);
+  a.status = dev_status;
+  return launch_route_decode(a, false, (cudaStream_t)stream);
 }
 
 extern "C" qmoe_status qmoe_rmsnorm_residual(const float *x_in, const float *y, float eps, float *x_out, int T, int H,
