@@ -40,6 +40,8 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="decode48", choices=sorted(WORKLOADS))
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--layers", type=int, default=None,
+                   help="decode workloads only: layers in the stack (default: all 48); for small profiling runs")
     p.add_argument("--tokens", type=int, default=None,
                    help="prefill workload only: tokens per chunk (default: the workload's 4096)")
     return p.parse_args()
@@ -140,17 +142,28 @@ def barrier(world):
 
 
 # ------------------------------------------------------------ traffic file --
-def kernel_source_hash():
+TRAFFIC_PROFILES = {
+    # kernel -> (committed ncu summary, sources that define the kernel)
+    "stack_decode": ("stack_decode_decode48_ncu.md",
+                     ("stack_decode.cu", "decode_tile.cuh", "common.cuh", "layout.cuh", "route_common.cuh")),
+}
+
+
+def kernel_source_hash(names):
     h = hashlib.sha256()
-    for name in ("ffn_decode.cu", "common.cuh", "layout.cuh"):
+    for name in names:
         with open(os.path.join(ROOT, "quantised_expert_decode_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def stored_traffic(workload):
-    """dram bytes per FFN launch from the committed ncu summary, if still current."""
-    path = os.path.join(ROOT, "profiles", f"ffn_decode_{workload}_ncu.md")
+def stored_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's
+    sources have not changed since the counters were taken (else None)."""
+    if kernel not in TRAFFIC_PROFILES:
+        return None
+    fname, sources = TRAFFIC_PROFILES[kernel]
+    path = os.path.join(ROOT, "profiles", fname)
     if not os.path.exists(path):
         return None
     vals = {}
@@ -159,7 +172,7 @@ def stored_traffic(workload):
             if line.startswith("- ") and ":" in line:
                 k, v = line[2:].split(":", 1)
                 vals[k.strip()] = v.strip().strip("`")
-    if vals.get("kernel_source_sha256_16") != kernel_source_hash():
+    if vals.get("kernel_source_sha256_16") != kernel_source_hash(sources):
         return None
     try:
         return float(vals["dram_bytes_per_launch"])
@@ -387,7 +400,7 @@ def run_ours(args, cfg):
         "config": dict(workload_desc(cfg, T), parallelism=f"replicas x{world}"),
         "roofline": {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": hbm,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": stored_traffic(args.workload),
+                     "traffic": stored_traffic("stack_decode") if (fused and cfg.L == 48) else None,
                      "algorithmic_bytes_per_launch": launch_bytes,
                      "avg_launch_us": 1e6 * launch_s,
                      "timing": "CUDA event nodes around the kernel node(s) of a graph replayed over the same "
@@ -482,7 +495,7 @@ def run_layer(args, cfg):
                                    f"{cfg.I}, top-{cfg.k}, {T} token; L2 flushed (256 MB write) between steps"},
             "roofline": {"bound": "hbm", "kernel": "ffn_decode_kernel", "achieved": achieved, "peak": hbm,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
-                         "traffic": stored_traffic(args.workload), "algorithmic_bytes_per_launch": ffn_bytes,
+                         "traffic": None, "algorithmic_bytes_per_launch": ffn_bytes,
                          "avg_launch_us": 1e3 * statistics.mean(ffn_ms),
                          "median_launch_us": 1e3 * statistics.median(ffn_ms)},
             "route_us_mean": 1e3 * statistics.mean(route_ms),
@@ -692,6 +705,8 @@ def main():
     cfg = configs.get(WORKLOADS[args.workload])
     if args.workload == "prefill" and args.tokens:
         cfg = cfg.with_(T=args.tokens)
+    if args.workload in ("decode48", "verify48") and args.layers:
+        cfg = cfg.with_(L=args.layers)
     if args.impl == "reference" and args.workload == "prefill":
         run_prefill_reference(args, cfg)
     elif args.impl == "reference":
