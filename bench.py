@@ -126,13 +126,20 @@ def dist_env():
 
 
 def max_over_ranks(v, world):
+    """Maximum of a per-rank value (a device-timed duration) over all ranks."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(world, steps, units_per_step, ms_max):
+    """Whole-job throughput of N replicas: units all ranks processed / the slowest rank's time."""
+    return world * steps * units_per_step / (ms_max / 1e3)
 
 
 def barrier(world):
@@ -334,7 +341,7 @@ def run_ours(args, cfg):
     ms = e0.elapsed_time(e1)
     clk = clocks.stop()
     ms = max_over_ranks(ms, world)
-    value = world * args.steps * T / (ms / 1e3)
+    value = replica_throughput(world, args.steps, T, ms)
 
     # end to end through the host-buffer entry point (pinned memory)
     xh = torch.from_numpy(xs_host).pin_memory()
@@ -637,7 +644,7 @@ def run_prefill(args, cfg):
         raise RuntimeError("device status set during the timed run")
     g1_ms = [es[0].elapsed_time(es[1]) for es in ev]
     g2_ms = [es[1].elapsed_time(es[2]) for es in ev]
-    value = world * args.steps * T / (ms / 1e3)
+    value = replica_throughput(world, args.steps, T, ms)
 
     # end to end: pinned bf16 x -> device, route + FFN, y -> pinned host
     xh = [torch.from_numpy(a).pin_memory() for a in xs_host]
