@@ -4,28 +4,9 @@
 #include <vector>
 
 #include "common.cuh"
+#include "stack_fused.cuh"
 
 namespace qmoe {
-struct FusedPlan {
-  size_t smem;
-  int nslots, slot_bytes;
-};
-struct FusedBufs {
-  float *wrt;
-  unsigned long long *lacc, *ssacc;
-  float *zbuf, *hbuf;
-  unsigned *bar;
-  const uint8_t **gu, **dn;
-  const float **bias;
-};
-bool fused_stack_plan(int fmt, int E, int H, int I, int k, FusedPlan *p);
-size_t fused_stack_ws_bytes(int L, int E, int H, int I, int k);
-FusedBufs fused_carve(void *ws, int L, int E, int H, int I, int k);
-qmoe_status fused_prepare(const FusedBufs &b, int L, int E, int H, const float *const *Wr,
-                          const qmoe_experts *layers, const float *const *bias, cudaStream_t s);
-qmoe_status fused_launch(const FusedBufs &b, const FusedPlan &p, int fmt, int L, int E, int H, int I, int k, float eps,
-                         const float *x_in, float *x_out, int32_t *idx_rec, float *gate_rec, int32_t *status,
-                         cudaStream_t s, bool cooperative);
 qmoe_status ffn_decode_launch(const qmoe_experts *ex, const float *x, int T, const int32_t *idx, const float *gate,
                               int k, float *y, void *ws, size_t ws_bytes, int32_t *status, cudaStream_t s,
                               bool cooperative);

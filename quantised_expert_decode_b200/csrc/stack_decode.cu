@@ -11,9 +11,12 @@
 //      renormalised gates (one warp, identical in every CTA); then the producer
 //      warp issues this layer's weight copies.
 //   C  gate/up tiles (selected expert j, 16-row tile r, gate or up), one ring
-//      item each: a_g = Wg x or a_u = Wu x for those 16 rows -> global
-//      ---- grid barrier (h complete) ----
-//   D  row owners: h_j = silu(a_g) * a_u, quantise all h_j, down tiles of rows R_c for every selected
+//      item each: a_g = Wg x or a_u = Wu x for those 16 rows -> global; the
+//      warp that completes the last of the four tiles of a 32-row block
+//      forms h = silu(a_g) * a_u for the block, quantises it into limbs and
+//      writes them to global (one block quantised once, by one warp)
+//      ---- grid barrier (h limbs complete) ----
+//   D  row owners: the limbs of every h_j in one bulk copy, down tiles of rows R_c for every selected
 //      expert (prefetched during C), y[R_c] = sum_j g_j * (Wd_j h_j)[R_c] in
 //      slot order, z_{l+1}[R_c] = x_l[R_c] + y[R_c]; then, from the rows
 //      R_c of the next layer's transposed router (prefetched), partial logits
@@ -30,6 +33,7 @@
 #include "decode_tile.cuh"
 #include "layout.cuh"
 #include "route_common.cuh"
+#include "stack_fused.cuh"
 
 namespace qmoe {
 namespace {
@@ -57,6 +61,9 @@ struct StackArgs {
   unsigned long long *lacc;   // [2][E] fixed-point partial-logit sums (two's complement)
   unsigned long long *ssacc;  // [2] fixed-point sum of squares
   float *hbuf;                // [2][k][I]: a_g, a_u
+  uint8_t *lbuf;              // [k][I/32][LIMB_REC]: limbs of h
+  float2 *lscg;               // [k][I/32]: (s, s * sum X) of h's blocks
+  unsigned *qcnt;             // [k][I/32]: tiles of the block completed this layer
   unsigned *bar;
   int32_t *status;
   int nslots, slot_bytes;
@@ -121,6 +128,44 @@ __device__ __forceinline__ bool cons_grid_barrier(const StackArgs &a, SkState *s
 // layer and would otherwise add its registers to the kernel body's).
 __device__ __noinline__ void topk_smem(const double *logits, int E, int k, int32_t *idx, float *gate, TopkScratch *sc) {
   warp_topk_gates_get([&](int e) { return logits[e]; }, E, k, idx, gate, sc);
+}
+
+// One warp: h = silu(a_g) * a_u for the 32 rows of block b of selected
+// expert j (lane i: row 32b + i), quantised exactly as quant_chunk_inl does a
+// 32-element block, limbs and scales written to global; the block's tile
+// counter is reset for the next layer.
+__device__ __noinline__ void quant_h_block(const StackArgs &a, int j, int b, int lane) {
+  __threadfence();   // the other tiles' a_g / a_u (counted before this warp's increment) are visible
+  const int nblkI = a.I / 32;
+  const float gv = __ldcg(a.hbuf + (size_t)j * a.I + b * 32 + lane);
+  const float uv = __ldcg(a.hbuf + ((size_t)a.k + j) * a.I + b * 32 + lane);
+  const float h = silu_f(gv) * uv;
+  float m = fabsf(h);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float sc = 0.0f, inv = 0.0f;
+  if (m > 0.0f) {
+    sc = m * (1.0f / QMAX);
+    inv = __frcp_rn(sc);
+  }
+  const int X = quant_one(h, inv);
+  int l[3];
+  limbs3(X, l[0], l[1], l[2]);
+  uint8_t *rec = a.lbuf + ((size_t)j * nblkI + b) * LIMB_REC;
+#pragma unroll
+  for (int p = 0; p < 3; ++p) {   // lanes 4q..4q+3 -> one little-endian word
+    const uint32_t v = (uint32_t)(l[p] & 0xff);
+    const uint32_t w = v | (__shfl_down_sync(0xffffffffu, v, 1) << 8) | (__shfl_down_sync(0xffffffffu, v, 2) << 16) |
+                       (__shfl_down_sync(0xffffffffu, v, 3) << 24);
+    if ((lane & 3) == 0) *reinterpret_cast<uint32_t *>(rec + p * 32 + lane) = w;
+  }
+  int sx = X;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, o);
+  if (lane == 0) {
+    a.lscg[(size_t)j * nblkI + b] = make_float2(sc, sc * (float)sx);
+    a.qcnt[(size_t)j * nblkI + b] = 0u;
+  }
 }
 
 template <int BITS>
@@ -352,6 +397,15 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
         dst[g] = o.x;
         dst[g + 8] = o.y;
       }
+      // four tiles (gate and up of rows 32b..32b+31) make a block of h; the
+      // warp that completes the fourth quantises the block
+      __syncwarp();
+      unsigned last = 0;
+      if (lane == 0) {
+        __threadfence();
+        last = atomicAdd(a.qcnt + (size_t)j * nblkI + (r >> 1), 1u) == 3u;
+      }
+      if (__shfl_sync(0xffffffffu, last, 0)) quant_h_block(a, j, r >> 1, lane);
     }
     nring += 2 * nunits;
     if (!cons_grid_barrier(a, st, tid)) continue;
@@ -359,45 +413,18 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
     // -------------------------------------------------------------------- D --
     if (rows) {
       {
-        const int nch = I / 128;
-        // a_g and a_u of every selected expert arrive in one bulk copy into
-        // the ring (all of this layer's ring items were consumed before the
-        // barrier), then quantise from shared memory
-        float *hs = reinterpret_cast<float *>(ring);
-        const uint32_t hbytes = (uint32_t)(2 * k * I * 4);
+        // the limbs and block scales of every selected expert's h (quantised
+        // during C) arrive in two bulk copies
+        const uint32_t lbytes = (uint32_t)(k * nblkI * LIMB_REC), sbytes = (uint32_t)(k * nblkI * 8);
         if (tid == 0) {
-          fence_proxy_async();   // h was written by ordinary stores; the ring was read by ordinary loads
-          mbar_arrive_expect_tx(hbar, hbytes);
-          bulk_g2s(hs, a.hbuf, hbytes, hbar);
+          fence_proxy_async();   // global limbs were written by ordinary stores; smem limbs read by ordinary loads
+          mbar_arrive_expect_tx(hbar, lbytes + sbytes);
+          bulk_g2s(limbs, a.lbuf, lbytes, hbar);
+          bulk_g2s(lsc, a.lscg, sbytes, hbar);
         }
-        const bool hok = mbar_wait(hbar, (uint32_t)(l & 1), clock64() + WAIT_BUDGET_CYCLES);
-        if (!hok) {
+        if (!mbar_wait(hbar, (uint32_t)(l & 1), clock64() + WAIT_BUDGET_CYCLES)) {
           set_status(a.status, DEV_TIMEOUT);
           *(volatile int *)&st->abort = 1;
-        }
-        const float *hg = hs, *hu = hs + (size_t)k * I;
-        const int ntask = hok ? k * nch : 0;
-        // three chunks per pass so that their independent chains interleave
-        for (int base = warp; base < ntask; base += 3 * SK_NCW) {
-          float4 h[3];
-#pragma unroll
-          for (int i = 0; i < 3; ++i) {
-            const int task = base + i * SK_NCW;
-            if (task < ntask) {
-              const size_t off = (size_t)(task / nch) * I + (task % nch) * 128;
-              const float4 gv = reinterpret_cast<const float4 *>(hg + off)[lane];
-              const float4 uv = reinterpret_cast<const float4 *>(hu + off)[lane];
-              h[i] = make_float4(silu_f(gv.x) * uv.x, silu_f(gv.y) * uv.y, silu_f(gv.z) * uv.z, silu_f(gv.w) * uv.w);
-            }
-          }
-#pragma unroll
-          for (int i = 0; i < 3; ++i) {
-            const int task = base + i * SK_NCW;
-            if (task < ntask) {
-              const int j = task / nch;
-              quant_chunk_inl(h[i], limbs + (size_t)j * nblkI * LIMB_REC, lsc + (size_t)j * nblkI, task % nch, lane);
-            }
-          }
         }
       }
       named_barrier_sync(CONS_BAR, nth);
@@ -475,11 +502,6 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
 }  // namespace
 
 // ---------------------------------------------------------------- host side --
-struct FusedPlan {
-  size_t smem;
-  int nslots, slot_bytes;
-};
-
 // Can the fused kernel run this stack? Fills the launch plan when it can.
 bool fused_stack_plan(int fmt, int E, int H, int I, int k, FusedPlan *p) {
   if (k > SK_MAXK || E > 1024 || H / 16 > num_sms() || H % 128 || I % 128) return false;
@@ -487,7 +509,7 @@ bool fused_stack_plan(int fmt, int E, int H, int I, int k, FusedPlan *p) {
   const size_t cap = max_smem_optin();
   for (int S = 12; S >= 4; --S) {
     const SkLayout o = sk_layout(fmt, E, H, I, k, S, slot);
-    if (o.total <= cap && (size_t)2 * k * I * 4 <= (size_t)S * slot) {  // D stages a_g, a_u in the ring
+    if (o.total <= cap) {
       p->smem = o.total;
       p->nslots = S;
       p->slot_bytes = slot;
@@ -499,18 +521,11 @@ bool fused_stack_plan(int fmt, int E, int H, int I, int k, FusedPlan *p) {
 
 size_t fused_stack_ws_bytes(int L, int E, int H, int I, int k) {
   auto a = [](size_t v) { return (v + 255) & ~(size_t)255; };
-  return a((size_t)L * H * E * 4) + a(2 * (size_t)E * 8) + 256 + a(2 * (size_t)H * 4) + a(2 * (size_t)k * I * 4) + 256 +
-         3 * a((size_t)L * 8);
+  const size_t nb = (size_t)k * (I / 32);
+  return a((size_t)L * H * E * 4) + a(2 * (size_t)E * 8) + 256 + a(2 * (size_t)H * 4) + a(2 * (size_t)k * I * 4) +
+         a(nb * LIMB_REC) + a(nb * 8) + a(nb * 4) + 256 + 3 * a((size_t)L * 8);
 }
 
-struct FusedBufs {
-  float *wrt;
-  unsigned long long *lacc, *ssacc;
-  float *zbuf, *hbuf;
-  unsigned *bar;
-  const uint8_t **gu, **dn;
-  const float **bias;
-};
 
 FusedBufs fused_carve(void *ws, int L, int E, int H, int I, int k) {
   auto a = [](size_t v) { return (v + 255) & ~(size_t)255; };
@@ -521,6 +536,10 @@ FusedBufs fused_carve(void *ws, int L, int E, int H, int I, int k) {
   b.ssacc = reinterpret_cast<unsigned long long *>(p); p += 256;
   b.zbuf = reinterpret_cast<float *>(p); p += a(2 * (size_t)H * 4);
   b.hbuf = reinterpret_cast<float *>(p); p += a(2 * (size_t)k * I * 4);
+  const size_t nb = (size_t)k * (I / 32);
+  b.lbuf = reinterpret_cast<uint8_t *>(p); p += a(nb * LIMB_REC);
+  b.lscg = reinterpret_cast<float2 *>(p); p += a(nb * 8);
+  b.qcnt = reinterpret_cast<unsigned *>(p); p += a(nb * 4);
   b.bar = reinterpret_cast<unsigned *>(p); p += 256;
   b.gu = reinterpret_cast<const uint8_t **>(p); p += a((size_t)L * 8);
   b.dn = reinterpret_cast<const uint8_t **>(p); p += a((size_t)L * 8);
@@ -570,6 +589,7 @@ qmoe_status fused_launch(const FusedBufs &b, const FusedPlan &p, int fmt, int L,
   a.gu = b.gu; a.dn = b.dn; a.bias = b.bias; a.wrt = b.wrt;
   a.x_in = x_in; a.x_out = x_out; a.idx_rec = idx_rec; a.gate_rec = gate_rec;
   a.zbuf = b.zbuf; a.lacc = b.lacc; a.ssacc = b.ssacc; a.hbuf = b.hbuf; a.bar = b.bar; a.status = status;
+  a.lbuf = b.lbuf; a.lscg = b.lscg; a.qcnt = b.qcnt;
   a.nslots = p.nslots; a.slot_bytes = p.slot_bytes;
   // Gate/up units are split evenly: the h barrier waits for the slowest CTA's
   // gate/up tiles, while the row owners' down tiles and router rows are only

@@ -1,0 +1,40 @@
+// Host-side interface of the fused single-token decode stack, shared by the
+// stack object (stack.cu) and the kernel's translation unit (stack_decode.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "qmoe.h"
+
+namespace qmoe {
+
+struct FusedPlan {
+  size_t smem;
+  int nslots, slot_bytes;
+};
+
+// Device buffers of the fused path, carved from the stack's workspace.
+struct FusedBufs {
+  float *wrt;                      // [L][H][E] transposed routers
+  unsigned long long *lacc, *ssacc;
+  float *zbuf, *hbuf;
+  uint8_t *lbuf;                   // limbs of h, [k][I/32][96]
+  float2 *lscg;                    // block scales of h, [k][I/32]
+  unsigned *qcnt;                  // per-block tile counters, [k][I/32]
+  unsigned *bar;
+  const uint8_t **gu, **dn;
+  const float **bias;
+};
+
+bool fused_stack_plan(int fmt, int E, int H, int I, int k, FusedPlan *p);
+size_t fused_stack_ws_bytes(int L, int E, int H, int I, int k);
+FusedBufs fused_carve(void *ws, int L, int E, int H, int I, int k);
+qmoe_status fused_prepare(const FusedBufs &b, int L, int E, int H, const float *const *Wr,
+                          const qmoe_experts *layers, const float *const *bias, cudaStream_t s);
+qmoe_status fused_launch(const FusedBufs &b, const FusedPlan &p, int fmt, int L, int E, int H, int I, int k, float eps,
+                         const float *x_in, float *x_out, int32_t *idx_rec, float *gate_rec, int32_t *status,
+                         cudaStream_t s, bool cooperative);
+
+}  // namespace qmoe
