@@ -369,15 +369,38 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
         mbar_arrive_expect_tx(&full[s], (uint32_t)tgu);
         bulk_g2s(ring + (size_t)s * a.slot_bytes, src, (uint32_t)tgu, &full[s]);
       }
-      if (lane == 31 && rows) {
-        const uint8_t *dn = a.dn[l];
-        mbar_arrive_expect_tx(dnbar, (uint32_t)(k * tdn));
-        for (int j = 0; j < k; ++j)
-          bulk_g2s(dnbuf + (size_t)j * tdn, dn + ((size_t)st->idx[j] * H16 + c) * (size_t)tdn, (uint32_t)tdn, dnbar);
-      }
-      if (lane == 30 && rows && l + 1 < L) {
-        mbar_arrive_expect_tx(wrtbar, (uint32_t)(16 * E * 4));
-        bulk_g2s(wrtbuf, a.wrt + ((size_t)(l + 1) * H + r0) * E, (uint32_t)(16 * E * 4), wrtbar);
+      if ((lane == 31 || lane == 30) && rows) {
+        // The down tiles and the next layer's router rows are needed only after
+        // the h barrier: issue them once this CTA's gate/up tiles have landed
+        // (every ring item of the layer acquired), so that they do not compete
+        // with the gate/up stream on the critical path.
+        const int want = nring + 2 * nunits;
+        const long long dl = clock64() + WAIT_BUDGET_CYCLES;
+        bool ok = true;
+        while (*(volatile int *)&st->turn < want) {
+          if (*(volatile int *)&st->abort) {
+            ok = false;
+            break;
+          }
+          if (clock64() > dl) {
+            set_status(a.status, DEV_TIMEOUT);
+            *(volatile int *)&st->abort = 1;
+            ok = false;
+            break;
+          }
+          __nanosleep(64);
+        }
+        if (ok && lane == 31) {
+          const uint8_t *dn = a.dn[l];
+          mbar_arrive_expect_tx(dnbar, (uint32_t)(k * tdn));
+          for (int j = 0; j < k; ++j)
+            bulk_g2s(dnbuf + (size_t)j * tdn, dn + ((size_t)st->idx[j] * H16 + c) * (size_t)tdn, (uint32_t)tdn,
+                     dnbar);
+        }
+        if (ok && lane == 30 && l + 1 < L) {
+          mbar_arrive_expect_tx(wrtbar, (uint32_t)(16 * E * 4));
+          bulk_g2s(wrtbuf, a.wrt + ((size_t)(l + 1) * H + r0) * E, (uint32_t)(16 * E * 4), wrtbar);
+        }
       }
       nring += 2 * nunits;
       continue;
