@@ -197,7 +197,9 @@ static qmoe_status check_route_common(const float *Wr, int T, int H, int E, int 
 
 extern "C" size_t qmoe_route_workspace_bytes(int T, int E) {
   if (T <= 0 || E <= 0) return 0;
-  if (T <= RT_MAXT) return decode_ws_bytes(T, E);
+  // T <= 8 with bf16 x runs the prefill router, so cover both
+  if (T <= RT_MAXT) return decode_ws_bytes(T, E) > route_prefill_ws_bytes(T, E) ? decode_ws_bytes(T, E)
+                                                                                : route_prefill_ws_bytes(T, E);
   return route_prefill_ws_bytes(T, E);
 }
 

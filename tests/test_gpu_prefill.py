@@ -93,6 +93,38 @@ def test_prefill_router_fp32_many_tokens_and_ties():
     assert np.max(np.abs(to_np(gate) - og)) < GATE_TOL
 
 
+def test_prefill_router_degenerate_equal_rows_take_the_exact_path():
+    """Every router row equal: all logits tie, more experts are candidates than
+    the candidate list holds, and the router falls back to float64 logits for
+    every expert; ties go to the lower index, gates are uniform."""
+    rs = np.random.default_rng(3)
+    E, H, k, T = 128, 256, 8, 20
+    row = (0.02 * rs.standard_normal(H)).astype(np.float32)
+    Wr_np = np.tile(row, (E, 1))
+    x_np = rs.standard_normal((T, H)).astype(np.float32)
+    idx, gate = route(torch.from_numpy(Wr_np).cuda(), None, torch.from_numpy(x_np).cuda(), k)
+    oi, og, _ = moe.route(x_np.astype(np.float64), Wr_np, None, k)
+    assert np.array_equal(to_np(idx), oi)
+    assert np.array_equal(oi, np.tile(np.arange(k, dtype=np.int32), (T, 1)))
+    assert np.max(np.abs(to_np(gate) - 1.0 / k)) < GATE_TOL
+
+
+def test_prefill_router_bf16_few_tokens_and_ragged_sizes():
+    """bf16 activations with T <= 8 also take the prefill router; T and E not
+    multiples of the GEMM tile."""
+    rs = np.random.default_rng(4)
+    for T, E, k in ((3, 200, 7), (70, 96, 16)):
+        H = 384
+        Wr_np = (0.02 * rs.standard_normal((E, H))).astype(np.float32)
+        b_np = rs.standard_normal(E).astype(np.float32)
+        x_bits = gen.f32_to_bf16_bits(rs.standard_normal((T, H)).astype(np.float32))
+        x = torch.from_numpy(x_bits.view(np.int16)).cuda().view(torch.bfloat16)
+        idx, gate = route(torch.from_numpy(Wr_np).cuda(), torch.from_numpy(b_np).cuda(), x, k, L.BF16)
+        oi, og, _ = moe.route(gen.bf16_bits_to_f32(x_bits).astype(np.float64), Wr_np, b_np, k)
+        assert np.array_equal(to_np(idx), oi), (T, E)
+        assert np.max(np.abs(to_np(gate) - og)) < GATE_TOL
+
+
 # ------------------------------------------------------------- prefill FFN --
 def _prefill(layer, x, idx, gate, k, check=True):
     T = x.shape[0]
