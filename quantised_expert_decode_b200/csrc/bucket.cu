@@ -38,18 +38,27 @@ __global__ void __launch_bounds__(BK_THREADS, 1) bucket_kernel(BucketArgs a) {
   if (tid == 0) bad = 0;
   __syncthreads();
   const int lo = (int)((long long)warp * a.P / BK_WARPS), hi = (int)((long long)(warp + 1) * a.P / BK_WARPS);
-  for (int p = lo + lane; p < hi; p += 32) {
-    const int e = a.idx[p];
-    if (e < 0 || e >= E) {
-      bad = 1;
-      continue;
+  // four pairs per lane per step, loads issued before use
+  for (int p0 = lo + lane; p0 < hi; p0 += 128) {
+    int ev[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) ev[u] = p0 + 32 * u < hi ? a.idx[p0 + 32 * u] : 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int p = p0 + 32 * u;
+      if (p >= hi) continue;
+      const int e = ev[u];
+      if (e < 0 || e >= E) {
+        bad = 1;
+        continue;
+      }
+      if (a.check_dup) {
+        const int j = p % a.k;
+        for (int j2 = 0; j2 < j; ++j2)
+          if (a.idx[p - j + j2] == e) bad = 2;
+      }
+      atomicAdd(&hist[warp * E + e], 1);
     }
-    if (a.check_dup) {
-      const int j = p % a.k;
-      for (int j2 = 0; j2 < j; ++j2)
-        if (a.idx[p - j + j2] == e) bad = 2;
-    }
-    atomicAdd(&hist[warp * E + e], 1);
   }
   __syncthreads();
   if (bad) {
@@ -105,22 +114,37 @@ __global__ void __launch_bounds__(BK_THREADS, 1) bucket_kernel(BucketArgs a) {
     }
   }
   __syncthreads();
-  // pass 2: place this warp's pairs in pair order
-  for (int p0 = lo; p0 < hi; p0 += 32) {
-    const int p = p0 + lane;
-    const bool valid = p < hi;
-    const int e = valid ? a.idx[p] : -1 - lane;     // distinct dummy keys for the tail
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    int pos = 0;
-    if (valid) pos = hist[warp * E + e] + rank;
-    __syncwarp();
-    if (valid && rank == 0) hist[warp * E + e] += __popc(peers);
-    __syncwarp();
-    if (valid) {
-      a.perm[pos] = p;
-      if (a.ptok) a.ptok[pos] = p / a.k;
-      if (a.pgate) a.pgate[pos] = a.gate[p];
+  // pass 2: place this warp's pairs in pair order, 32 at a time; the expert
+  // ids of the next batches are loaded ahead
+  int nxt[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) nxt[u] = lo + lane + 32 * u < hi ? a.idx[lo + lane + 32 * u] : 0;
+  for (int p0 = lo; p0 < hi; p0 += 128) {
+    int cur[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      cur[u] = nxt[u];
+      const int q = p0 + 128 + lane + 32 * u;
+      nxt[u] = q < hi ? a.idx[q] : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int p = p0 + 32 * u + lane;
+      if (p0 + 32 * u >= hi) break;           // warp-uniform
+      const bool valid = p < hi;
+      const int e = valid ? cur[u] : -1 - lane;   // distinct dummy keys for the tail
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      int pos = 0;
+      if (valid) pos = hist[warp * E + e] + rank;
+      __syncwarp();
+      if (valid && rank == 0) hist[warp * E + e] += __popc(peers);
+      __syncwarp();
+      if (valid) {
+        a.perm[pos] = p;
+        if (a.ptok) a.ptok[pos] = p / a.k;
+        if (a.pgate) a.pgate[pos] = a.gate[p];
+      }
     }
   }
 }

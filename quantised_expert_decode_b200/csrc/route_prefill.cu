@@ -48,6 +48,17 @@ __device__ __forceinline__ float load_xf(const void *x, size_t i) {
   return static_cast<const float *>(x)[i];
 }
 
+// Four consecutive activations of token row x_t as floats (bf16 is exact in fp32).
+template <int XDT>
+__device__ __forceinline__ float4 load_x4(const void *x, size_t i) {
+  if (XDT == QMOE_BF16) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(static_cast<const unsigned short *>(x) + i);
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u), __uint_as_float(u.y << 16),
+                       __uint_as_float(u.y & 0xffff0000u));
+  }
+  return *reinterpret_cast<const float4 *>(static_cast<const float *>(x) + i);
+}
+
 // One warp per row: token rows 0..T-1, then router rows T..T+E-1.
 template <int XDT>
 __global__ void __launch_bounds__(256) rq_scale_kernel(const void *__restrict__ x, const float *__restrict__ Wr, int T,
@@ -127,7 +138,13 @@ __global__ void __launch_bounds__(RQ_THREADS, 1) rq_gemm_kernel(const void *__re
   float xv[16], wv[32];
   auto gload = [&](int k0) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) xv[i] = load_xf<XDT>(x, (size_t)xtok * H + k0 + xc + i);
+    for (int q = 0; q < 4; ++q) {
+      const float4 f = load_x4<XDT>(x, (size_t)xtok * H + k0 + xc + 4 * q);
+      xv[4 * q] = f.x;
+      xv[4 * q + 1] = f.y;
+      xv[4 * q + 2] = f.z;
+      xv[4 * q + 3] = f.w;
+    }
     const float4 *wp = reinterpret_cast<const float4 *>(Wr + (size_t)wexp * H + k0 + wc);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -217,15 +234,31 @@ __device__ __forceinline__ double rq_bound(float sx, double n1x, float sw, doubl
   return b * (1.0 + 1e-9) + 1e-12 * (fabs(a) + 1.0);
 }
 
-// Exact-product float64 logit of one (token, expert) pair: one warp.
+// Exact-product float64 logits of token t for experts e0 and e1 (one warp;
+// e1 < 0: only e0). Lane l takes elements 4l..4l+3 of every 128-element chunk.
 template <int XDT>
-__device__ __forceinline__ double exact_logit(const void *x, const float *Wr, const float *bias, int t, int e, int H,
-                                              int lane) {
-  double p = 0.0;
-  const float *w = Wr + (size_t)e * H;
-  for (int h = lane; h < H; h += 32) p = fma((double)load_xf<XDT>(x, (size_t)t * H + h), (double)w[h], p);
-  p = warp_sum_d(p);
-  return bias ? p + (double)bias[e] : p;
+__device__ __forceinline__ void exact_logits2(const void *x, const float *Wr, const float *bias, int t, int e0, int e1,
+                                              int H, int lane, double &out0, double &out1) {
+  double p0 = 0.0, p1 = 0.0;
+  const float *w0 = Wr + (size_t)e0 * H, *w1 = Wr + (size_t)(e1 >= 0 ? e1 : e0) * H;
+#pragma unroll 4
+  for (int h = 4 * lane; h < H; h += 128) {
+    const float4 xv = load_x4<XDT>(x, (size_t)t * H + h);
+    const float4 a = __ldg(reinterpret_cast<const float4 *>(w0 + h));
+    const float4 b = __ldg(reinterpret_cast<const float4 *>(w1 + h));
+    p0 = fma((double)xv.x, (double)a.x, p0);
+    p0 = fma((double)xv.y, (double)a.y, p0);
+    p0 = fma((double)xv.z, (double)a.z, p0);
+    p0 = fma((double)xv.w, (double)a.w, p0);
+    p1 = fma((double)xv.x, (double)b.x, p1);
+    p1 = fma((double)xv.y, (double)b.y, p1);
+    p1 = fma((double)xv.z, (double)b.z, p1);
+    p1 = fma((double)xv.w, (double)b.w, p1);
+  }
+  p0 = warp_sum_d(p0);
+  p1 = warp_sum_d(p1);
+  out0 = bias ? p0 + (double)bias[e0] : p0;
+  out1 = (e1 >= 0 && bias) ? p1 + (double)bias[e1] : p1;
 }
 
 struct SelScratch {
@@ -287,9 +320,13 @@ __device__ void rq_select_token(const void *x, const float *Wr, const float *bia
   const int total = __shfl_sync(0xffffffffu, incl, 31);
   if (total > RQ_CAND) {
     // degenerate: float64 logits of every expert, then the general selection
-    for (int e = 0; e < E; ++e) {
-      const double p = exact_logit<XDT>(x, Wr, bias, t, e, H, lane);
-      if (lane == 0) approx_row[e] = p;
+    for (int e = 0; e < E; e += 2) {
+      double p0, p1;
+      exact_logits2<XDT>(x, Wr, bias, t, e, e + 1 < E ? e + 1 : -1, H, lane, p0, p1);
+      if (lane == 0) {
+        approx_row[e] = p0;
+        if (e + 1 < E) approx_row[e + 1] = p1;
+      }
     }
     __syncwarp();
     __threadfence_block();
@@ -303,9 +340,13 @@ __device__ void rq_select_token(const void *x, const float *Wr, const float *bia
       if (lane + 32 * i < E && v[i] + bnd[i] >= lowk) s->cand[pos++] = lane + 32 * i;
   }
   __syncwarp();
-  for (int c = 0; c < total; ++c) {
-    const double p = exact_logit<XDT>(x, Wr, bias, t, s->cand[c], H, lane);
-    if (lane == 0) s->cand_v[c] = p;
+  for (int c = 0; c < total; c += 2) {
+    double p0, p1;
+    exact_logits2<XDT>(x, Wr, bias, t, s->cand[c], c + 1 < total ? s->cand[c + 1] : -1, H, lane, p0, p1);
+    if (lane == 0) {
+      s->cand_v[c] = p0;
+      if (c + 1 < total) s->cand_v[c + 1] = p1;
+    }
   }
   __syncwarp();
   // rank the candidates exactly (value descending, lower expert first on ties)
