@@ -153,6 +153,7 @@ TRAFFIC_PROFILES = {
     # kernel -> (committed ncu summary, sources that define the kernel)
     "stack_decode": ("stack_decode_decode48_ncu.md",
                      ("stack_decode.cu", "decode_tile.cuh", "common.cuh", "layout.cuh", "route_common.cuh")),
+    "pf_gemm1": ("pf_gemm_prefill4096_ncu.md", ("prefill.cu", "tc05.cuh", "common.cuh", "layout.cuh")),
 }
 
 
@@ -681,7 +682,8 @@ def run_prefill(args, cfg):
         "config": dict(prefill_desc(cfg), parallelism=f"replicas x{world}"),
         "roofline": {"bound": "tensor", "kernel": "pf_gemm_kernel (grouped GEMM 1: gate/up + SiLU*up epilogue)",
                      "achieved": a1, "peak": peak, "peak_kind": peak_kind, "unit": "TFLOP/s", "frac": a1 / peak,
-                     "traffic": None, "algorithmic_flops_per_launch": f_g1, "avg_launch_us": 1e6 * t1,
+                     "traffic": stored_traffic("pf_gemm1") if cfg.T == 4096 else None,
+                     "algorithmic_flops_per_launch": f_g1, "avg_launch_us": 1e6 * t1,
                      "timing": "CUDA events recorded on the launching stream around each GEMM launch"},
         "prefill": {"gemm2_TFLOPs": f_g2 / t2 / 1e12, "gemm2_frac": f_g2 / t2 / 1e12 / peak,
                     "gemm2_us": 1e6 * t2, "ffn_gemms_frac": f_layer / (t1 + t2) / 1e12 / peak,
