@@ -29,7 +29,7 @@ namespace qmoe {
 namespace {
 
 constexpr int RQ_TT = 64;            // tokens per GEMM CTA
-constexpr int RQ_TE = 128;           // experts per GEMM CTA
+constexpr int RQ_TE = 64;            // experts per GEMM CTA
 constexpr int RQ_KC = 64;            // reduction elements per shared-memory chunk
 constexpr int RQ_THREADS = 256;
 constexpr int RQ_ROW = RQ_KC + 16;   // padded int8 row: conflict-free fragment loads
@@ -116,13 +116,13 @@ __device__ __forceinline__ uint32_t pack4b(int a, int b, int c, int d) {
          ((uint32_t)(d & 0xff) << 24);
 }
 
-// Approximate logits of a 64-token x 128-expert tile. Shared memory holds the
+// Approximate logits of a 64-token x 64-expert tile. Shared memory holds the
 // hi and lo limb planes of the current K chunk, [row][RQ_ROW] bytes; global
 // loads of the next chunk are held in registers while the current one is
 // multiplied. Warp (wm, wn) = (w % 4, w / 4) owns tokens 16 wm.. and experts
-// 64 wn.. (8 n-tiles of 8); accumulators: hi*hi, hi*lo + lo*hi, lo*lo.
+// 32 wn.. (4 n-tiles of 8); accumulators: hi*hi, hi*lo + lo*hi, lo*lo.
 template <int XDT>
-__global__ void __launch_bounds__(RQ_THREADS, 1) rq_gemm_kernel(const void *__restrict__ x,
+__global__ void __launch_bounds__(RQ_THREADS, 2) rq_gemm_kernel(const void *__restrict__ x,
                                                                 const float *__restrict__ Wr,
                                                                 const float *__restrict__ bias, int T, int E, int H,
                                                                 Scales sc, double *__restrict__ approx) {
@@ -130,12 +130,12 @@ __global__ void __launch_bounds__(RQ_THREADS, 1) rq_gemm_kernel(const void *__re
   __shared__ __align__(16) uint8_t wsm[2][RQ_TE * RQ_ROW];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
   const int t0 = blockIdx.x * RQ_TT, e0 = blockIdx.y * RQ_TE;
-  // loader roles: x: row tid / 4, 16 values from column (tid % 4) * 16; w: row tid / 2, 32 values
-  const int xr = tid >> 2, xc = (tid & 3) * 16, wr = tid >> 1, wc = (tid & 1) * 32;
+  // loader roles: x and w: row tid / 4, 16 values from column (tid % 4) * 16
+  const int xr = tid >> 2, xc = (tid & 3) * 16, wr = tid >> 2, wc = (tid & 3) * 16;
   const int xtok = min(t0 + xr, T - 1), wexp = min(e0 + wr, E - 1);
   const float xinv = sc.sx[xtok] > 0.0f ? 1.0f / sc.sx[xtok] : 0.0f;
   const float winv = sc.sw[wexp] > 0.0f ? 1.0f / sc.sw[wexp] : 0.0f;
-  float xv[16], wv[32];
+  float xv[16], wv[16];
   auto gload = [&](int k0) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(RQ_THREADS, 1) rq_gemm_kernel(const void *__re
     }
     const float4 *wp = reinterpret_cast<const float4 *>(Wr + (size_t)wexp * H + k0 + wc);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 4; ++i) {
       const float4 f = __ldg(wp + i);
       wv[4 * i] = f.x;
       wv[4 * i + 1] = f.y;
@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(RQ_THREADS, 1) rq_gemm_kernel(const void *__re
       *reinterpret_cast<uint32_t *>(&xs[1][xr * RQ_ROW + xc + 4 * q]) = pack4b(l[0], l[1], l[2], l[3]);
     }
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
+    for (int q = 0; q < 4; ++q) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) quant2(wv[4 * q + i], winv, h[i], l[i]);
       *reinterpret_cast<uint32_t *>(&wsm[0][wr * RQ_ROW + wc + 4 * q]) = pack4b(h[0], h[1], h[2], h[3]);
@@ -173,9 +173,9 @@ __global__ void __launch_bounds__(RQ_THREADS, 1) rq_gemm_kernel(const void *__re
     }
   };
   const int wm = warp & 3, wn = warp >> 2;
-  int hh[8][4], mid[8][4], ll[8][4];
+  int hh[4][4], mid[4][4], ll[4][4];
 #pragma unroll
-  for (int n = 0; n < 8; ++n)
+  for (int n = 0; n < 4; ++n)
 #pragma unroll
     for (int i = 0; i < 4; ++i) hh[n][i] = mid[n][i] = ll[n][i] = 0;
 
@@ -198,8 +198,8 @@ __global__ void __launch_bounds__(RQ_THREADS, 1) rq_gemm_kernel(const void *__re
       al[2] = *reinterpret_cast<const uint32_t *>(&xs[1][ra + 16]);
       al[3] = *reinterpret_cast<const uint32_t *>(&xs[1][rb + 16]);
 #pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        const int rw = (64 * wn + 8 * n + g) * RQ_ROW + ks + 4 * t4;
+      for (int n = 0; n < 4; ++n) {
+        const int rw = (32 * wn + 8 * n + g) * RQ_ROW + ks + 4 * t4;
         const uint32_t bh0 = *reinterpret_cast<const uint32_t *>(&wsm[0][rw]);
         const uint32_t bh1 = *reinterpret_cast<const uint32_t *>(&wsm[0][rw + 16]);
         const uint32_t bl0 = *reinterpret_cast<const uint32_t *>(&wsm[1][rw]);
@@ -213,11 +213,11 @@ __global__ void __launch_bounds__(RQ_THREADS, 1) rq_gemm_kernel(const void *__re
   }
   // accumulator (row, col) of fragment i: rows g / g+8, columns 2 t4 + (i & 1)
 #pragma unroll
-  for (int n = 0; n < 8; ++n) {
+  for (int n = 0; n < 4; ++n) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int tok = t0 + 16 * wm + g + (i >> 1) * 8;
-      const int e = e0 + 64 * wn + 8 * n + 2 * t4 + (i & 1);
+      const int e = e0 + 32 * wn + 8 * n + 2 * t4 + (i & 1);
       if (tok < T && e < E) {
         const long long q = 65536LL * hh[n][i] + 256LL * mid[n][i] + (long long)ll[n][i];
         double v = (double)q * ((double)sc.sx[tok] * (double)sc.sw[e]);
