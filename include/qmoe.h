@@ -198,10 +198,15 @@ qmoe_status qmoe_ffn_decode(const qmoe_experts *experts, const float *x, int T,
  *   perm    int32 [T*k]: perm[offsets[e] + i] = i-th pair (in pair order) of e
  *   active  int32 [E] or NULL: experts with at least one pair, ascending
  *   nactive int32 [1] or NULL: their count
- * Limits: E <= 1024, T*k <= 2^30. One CTA; an index outside [0, E) sets the
- * device status and leaves the outputs unwritten. */
+ * Limits: E <= 1024, T*k <= 2^30. Two launches on `stream` over up to 148
+ * CTAs (a per-CTA expert histogram, then placement); no CTA waits on another.
+ * Workspace: qmoe_bucket_workspace_bytes(T, k, E) bytes, 16-byte aligned, no
+ * initialisation needed. An index outside [0, E) sets the device status and
+ * leaves offsets, perm, active and nactive unwritten. */
+size_t qmoe_bucket_workspace_bytes(int T, int k, int E);
 qmoe_status qmoe_bucket(const int32_t *idx, int T, int k, int E, int32_t *offsets, int32_t *perm,
-                        int32_t *active, int32_t *nactive, int32_t *dev_status, qmoe_stream_t stream);
+                        int32_t *active, int32_t *nactive, void *workspace, size_t workspace_bytes,
+                        int32_t *dev_status, qmoe_stream_t stream);
 
 /* ------------------------------------------------------------- prefill FFN --
  * Routed expert FFN for prefill chunks of many tokens ([P3] batched prefill in

@@ -54,7 +54,8 @@ _SIGS = {
     "qmoe_rmsnorm_residual": (_I, [_VP, _VP, _F, _VP, _I, _I, _VP]),
     "qmoe_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "qmoe_ffn_decode": (_I, [ctypes.POINTER(qmoe_experts), _VP, _I, _VP, _VP, _I, _VP, _VP, _SZ, _VP, _VP]),
-    "qmoe_bucket": (_I, [_VP, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "qmoe_bucket_workspace_bytes": (_SZ, [_I, _I, _I]),
+    "qmoe_bucket": (_I, [_VP, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
     "qmoe_prefill_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "qmoe_ffn_prefill": (_I, [ctypes.POINTER(qmoe_experts), _VP, _I, _VP, _VP, _I, _VP, _VP, _SZ, _VP, _VP]),
     "qmoe_ffn_prefill_timed": (_I, [ctypes.POINTER(qmoe_experts), _VP, _I, _VP, _VP, _I, _VP, _VP, _SZ, _VP, _VP,
@@ -168,8 +169,13 @@ def qmoe_ffn_decode(experts: qmoe_experts, x, T, idx, gate, k, y, workspace, dev
         workspace.numel() * workspace.element_size(), _p(dev_status), _s(stream)))
 
 
-def qmoe_bucket(idx, T, k, E, offsets, perm, active, nactive, dev_status, stream=None) -> None:
+def qmoe_bucket_workspace_bytes(T: int, k: int, E: int) -> int:
+    return lib().qmoe_bucket_workspace_bytes(T, k, E)
+
+
+def qmoe_bucket(idx, T, k, E, offsets, perm, active, nactive, workspace, dev_status, stream=None) -> None:
     _check("qmoe_bucket", lib().qmoe_bucket(_p(idx), T, k, E, _p(offsets), _p(perm), _p(active), _p(nactive),
+                                            _p(workspace), workspace.numel() * workspace.element_size(),
                                             _p(dev_status), _s(stream)))
 
 

@@ -24,11 +24,11 @@
 
 namespace qmoe {
 
-size_t bucket_smem_bytes(int E);
+size_t bucket_ws_bytes(int T, int k, int E);
 bool bucket_supported(int T, int k, int E);
-qmoe_status bucket_launch(const int32_t *idx, const float *gate, int T, int k, int E, int32_t *offsets, int32_t *perm,
-                          int32_t *ptok, float *pgate, int32_t *active, int32_t *nactive, bool check_dup,
-                          int32_t *status, cudaStream_t s);
+qmoe_status bucket_launch(const int32_t *idx, const float *gate, int T, int k, int E, void *ws, int32_t *offsets,
+                          int32_t *perm, int32_t *ptok, float *pgate, int32_t *active, int32_t *nactive,
+                          bool check_dup, int32_t *status, cudaStream_t s);
 
 namespace {
 
@@ -608,7 +608,7 @@ __global__ void __launch_bounds__(1024, 1) pf_plan_kernel(PlanArgs a) {
 
 // ------------------------------------------------------------ workspace --
 struct PfLayout {
-  size_t off, poff, perm, ptok, pgate, ntiles, tiles1, tiles2, h, xp, total;
+  size_t off, poff, perm, ptok, pgate, ntiles, bk, tiles1, tiles2, h, xp, total;
   size_t max_tiles1, max_tiles2, h_rows;
 };
 
@@ -628,6 +628,7 @@ PfLayout pf_layout(int T, int k, int E, int H, int I) {
   L.ptok = o;   o += up256(P * sizeof(int32_t));
   L.pgate = o;  o += up256(P * sizeof(float));
   L.ntiles = o; o += 256;
+  L.bk = o;     o += bucket_ws_bytes(T, k, E);
   L.tiles1 = o; o += up256(L.max_tiles1 * sizeof(int4));
   L.tiles2 = o; o += up256(L.max_tiles2 * sizeof(int4));
   L.h = o;      o += up256(L.h_rows * I * sizeof(__nv_bfloat16));
@@ -741,7 +742,7 @@ static qmoe_status ffn_prefill(const qmoe_experts *ex, const void *x, int T, con
   __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(ws + L.h);
   __nv_bfloat16 *xp = reinterpret_cast<__nv_bfloat16 *>(ws + L.xp);
 
-  qmoe_status st = bucket_launch(idx, gate, T, k, E, off, perm, ptok, pgate, nullptr, nullptr, true, dev_status, s);
+  qmoe_status st = bucket_launch(idx, gate, T, k, E, ws + L.bk, off, perm, ptok, pgate, nullptr, nullptr, true, dev_status, s);
   if (st != QMOE_OK) return st;
   PlanArgs pa{off, E, I / PF_M, H / (2 * PF_M), poff, tiles1, tiles2, ntiles, dev_status};
   pf_plan_kernel<<<1, 1024, 0, s>>>(pa);

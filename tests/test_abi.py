@@ -127,10 +127,18 @@ def test_prefill_argument_checks_without_gpu():
 
 def test_bucket_argument_checks_without_gpu():
     lib = q.lib()
-    assert lib.qmoe_bucket(None, 8, 2, 16, FAKE, FAKE, None, None, FAKE, None) == 1
-    assert lib.qmoe_bucket(FAKE, 0, 2, 16, FAKE, FAKE, None, None, FAKE, None) == 1
-    assert lib.qmoe_bucket(FAKE, 8, 2, 4096, FAKE, FAKE, None, None, FAKE, None) == 3
-    assert lib.qmoe_bucket(FAKE + 2, 8, 2, 16, FAKE, FAKE, None, None, FAKE, None) == 1
+    ws = lib.qmoe_bucket_workspace_bytes(8, 2, 16)
+    assert ws >= 16 * 4 and lib.qmoe_bucket_workspace_bytes(0, 2, 16) == 0
+    # the table holds one row of E counts per CTA; CTAs cover at least 64 tokens each, 148 at most
+    assert lib.qmoe_bucket_workspace_bytes(4096, 10, 512) >= 64 * 512 * 4
+    assert lib.qmoe_bucket_workspace_bytes(1 << 20, 1, 1024) >= 148 * 1024 * 4
+    assert lib.qmoe_bucket(None, 8, 2, 16, FAKE, FAKE, None, None, FAKE, ws, FAKE, None) == 1
+    assert lib.qmoe_bucket(FAKE, 0, 2, 16, FAKE, FAKE, None, None, FAKE, ws, FAKE, None) == 1
+    assert lib.qmoe_bucket(FAKE, 8, 2, 4096, FAKE, FAKE, None, None, FAKE, ws, FAKE, None) == 3
+    assert lib.qmoe_bucket(FAKE + 2, 8, 2, 16, FAKE, FAKE, None, None, FAKE, ws, FAKE, None) == 1
+    assert lib.qmoe_bucket(FAKE, 8, 2, 16, FAKE, FAKE, None, None, None, ws, FAKE, None) == 1
+    assert lib.qmoe_bucket(FAKE, 8, 2, 16, FAKE, FAKE, None, None, FAKE + 4, ws, FAKE, None) == 1
+    assert lib.qmoe_bucket(FAKE, 8, 2, 16, FAKE, FAKE, None, None, FAKE, ws - 4, FAKE, None) == 4
 
 
 def test_pack_and_norm_argument_checks_without_gpu():

@@ -26,8 +26,9 @@ def _bucket(idx_np, E, check=True):
     perm = torch.full((T * k,), -1, dtype=torch.int32, device="cuda")
     act = torch.full((E,), -1, dtype=torch.int32, device="cuda")
     nact = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    ws = torch.full((q.qmoe_bucket_workspace_bytes(T, k, E),), 0x5A, dtype=torch.uint8, device="cuda")
     st = status_word()
-    q.qmoe_bucket(idx, T, k, E, off, perm, act, nact, st)
+    q.qmoe_bucket(idx, T, k, E, off, perm, act, nact, ws, st)
     torch.cuda.synchronize()
     if check:
         assert q.qmoe_read_status(st) == 0
@@ -45,7 +46,7 @@ def _bucket_reference(idx_np, E):
 
 
 @pytest.mark.parametrize("T,k,E", [(1, 1, 1), (1, 10, 512), (37, 4, 64), (4096, 10, 512), (1000, 8, 100),
-                                   (333, 16, 1024)])
+                                   (333, 16, 1024), (9473, 3, 257), (148 * 64 + 1, 2, 33), (30000, 10, 1000)])
 def test_bucket_is_the_stable_sort(T, k, E):
     rs = np.random.default_rng(T * 7 + k)
     # long-tailed loads: a few experts take most pairs (duplicates within a token allowed here)
@@ -66,6 +67,15 @@ def test_bucket_all_pairs_to_one_expert_and_bad_index():
     idx[5, 1] = 16
     *_, st = _bucket(idx, 16, check=False)
     assert q.qmoe_read_status(st) == 7
+
+
+def test_bucket_bad_index_in_a_late_cta_leaves_every_output_unwritten():
+    rs = np.random.default_rng(11)
+    idx = rs.integers(0, 64, size=(20000, 4)).astype(np.int32)
+    idx[19990, 2] = -3
+    off, perm, act, nact, st = _bucket(idx, 64, check=False)
+    assert q.qmoe_read_status(st) == 7
+    assert (off == -1).all() and (perm == -1).all() and (act == -1).all() and nact == -1
 
 
 # ---------------------------------------------------------------- router ----
