@@ -57,7 +57,7 @@ constexpr int PF_MAX_E = 1024;
 
 // warp roles
 constexpr int W_PRODUCER = 0;   // TMA loads of packed weight tiles (+ L2 prefetch)
-constexpr int W_MMA = 1;        // tensor memory owner; lane 0 issues the MMAs
+constexpr int W_MMA = 1;        // tensor memory owner; one elected lane issues the MMAs
 constexpr int W_BLOAD = 2;      // TMA loads of activation rows
 constexpr int W_EPI = 4;        // warps 4-11: accumulator epilogue, two warps per 32-lane quadrant
 constexpr int N_EPI = 8;
@@ -330,6 +330,10 @@ __device__ void pf_dequant(const PfGemm &a, uint8_t *sm, PfBars *b, int nt) {
   }
 }
 
+// The whole warp runs the loop (waits, descriptor arithmetic) so every value
+// stays warp-uniform; one elected lane issues the tensor-core instructions.
+// Issuing from a lone lane in a divergent branch measured about 2.5x slower
+// per MMA, which made the issue loop the limit for small tiles.
 __device__ void pf_mma(const PfGemm &a, uint8_t *sm, PfBars *b, int nt, uint32_t tmem) {
   const uint32_t base = smem_u32(sm);
   // descriptors of stage 0; a stage's start address is added in 16-byte units
@@ -339,34 +343,40 @@ __device__ void pf_mma(const PfGemm &a, uint8_t *sm, PfBars *b, int nt, uint32_t
   for (int ti = blockIdx.x; ti < nt; ti += gridDim.x) {
     const int4 t = a.tiles[ti];
     const uint32_t idesc = tc05::idesc_bf16_f32(PF_M, (t.w + 15) & ~15);
-    if (!pf_wait(&b->acc_empty, (tc & 1) ^ 1, b, a.status)) goto done;
+    if (!pf_wait_warp(&b->acc_empty, (tc & 1) ^ 1, b, a.status)) goto done;
     tc05::fence_after_sync();
     for (int s = 0; s < a.ksteps; ++s, ++g) {
       const int sa = g % PF_SA, sb = g % PF_SB;
-      if (!pf_wait(&b->a_full[sa], (g / PF_SA) & 1, b, a.status)) goto done;
-      if (!pf_wait(&b->b_full[sb], (g / PF_SB) & 1, b, a.status)) goto done;
+      if (!pf_wait_warp(&b->a_full[sa], (g / PF_SA) & 1, b, a.status)) goto done;
+      if (!pf_wait_warp(&b->b_full[sb], (g / PF_SB) & 1, b, a.status)) goto done;
       tc05::fence_after_sync();
       issued = true;
       const uint64_t d0 = da0 + (uint64_t)(sa * (PF_ASTAGE >> 4)), d1 = d0 + (PF_A_BYTES >> 4);
       const uint64_t db = db0 + (uint64_t)(sb * (PF_B_BYTES >> 4));
+      if (tc05::elect_one()) {
 #pragma unroll
-      for (int kk = 0; kk < PF_KS / 16; ++kk) {
-        const uint32_t acc = (s | kk) != 0;
-        tc05::mma_bf16(tmem, d0 + 2 * kk, db + 2 * kk, idesc, acc);
-        tc05::mma_bf16(tmem + 256, d1 + 2 * kk, db + 2 * kk, idesc, acc);
+        for (int kk = 0; kk < PF_KS / 16; ++kk) {
+          const uint32_t acc = (s | kk) != 0;
+          tc05::mma_bf16(tmem, d0 + 2 * kk, db + 2 * kk, idesc, acc);
+          tc05::mma_bf16(tmem + 256, d1 + 2 * kk, db + 2 * kk, idesc, acc);
+        }
+        tc05::commit(&b->a_empty[sa]);
+        tc05::commit(&b->b_empty[sb]);
       }
-      tc05::commit(&b->a_empty[sa]);
-      tc05::commit(&b->b_empty[sb]);
+      __syncwarp();
     }
-    tc05::commit(&b->acc_full);
+    if (tc05::elect_one()) tc05::commit(&b->acc_full);
+    __syncwarp();
     ++tc;
   }
 done:
-  // every MMA this thread issued has completed before tensor memory is freed
-  if (issued) {
+  // every MMA the issuing lane (lane 0: the lowest lane of the converged
+  // warp) issued has completed before tensor memory is freed
+  if (issued && (threadIdx.x & 31) == 0) {
     tc05::commit(&b->fin);
     if (!mbar_wait(&b->fin, 0, clock64() + WAIT_BUDGET_CYCLES)) set_status(a.status, DEV_TIMEOUT);
   }
+  __syncwarp();
 }
 
 __device__ __forceinline__ float silu(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
@@ -474,8 +484,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const __grid_con
     if (lane == 0) pf_producer(a, sm, b, nt);
     __syncwarp();
   } else if (warp == W_MMA) {
-    if (lane == 0) pf_mma(a, sm, b, nt, tmem);
-    __syncwarp();
+    pf_mma(a, sm, b, nt, tmem);
   } else if (warp == W_BLOAD) {
     if (lane == 0) pf_bloader(a, sm, b, nt);
     __syncwarp();

@@ -34,6 +34,13 @@ __device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence
 // async-proxy reads (tensor-core operand fetches) of the same bytes.
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// One lane of the (converged) warp returns true: the lowest active lane.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile("{ .reg .pred P; elect.sync _|P, 0xffffffff; selp.b32 %0, 1, 0, P; }" : "=r"(pred));
+  return pred != 0;
+}
+
 // ------------------------------------------------------------- descriptors --
 // Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzle
 // layout: rows of 64 bf16 (128 bytes) at a 128-byte pitch, groups of 8 rows
