@@ -11,8 +11,11 @@
 // X_e is the bf16 activation rows of the tokens routed to e, gathered by
 // token id; h is kept in bucket order with every expert's rows padded to a
 // multiple of 16. The weights form the 128-row MMA operand and the tokens the
-// N operand (16..256, a multiple of 16), so an expert with n tokens costs
-// ceil(n/16)*16 columns, not a 128-row tile.
+// N operand (16..PF_N, a multiple of 16), so an expert with n tokens costs
+// ceil(n/16)*16 columns, not a 128-row tile. Tensor memory holds two
+// accumulator slots of 256 columns: a tile of at most 128 tokens takes one
+// (its two accumulators side by side), so the epilogue of one such tile
+// overlaps the main loop of the next; a wider tile takes both.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -52,7 +55,9 @@ constexpr int PF_OFF_BAR = PF_OFF_PK + PF_PS * PF_PK;
 constexpr int PF_SMEM = PF_OFF_BAR + 256 + 1024;        // barriers + alignment slack
 constexpr int PF_PREFETCH = 16;                         // k-steps of packed weights prefetched into L2 ahead
 constexpr int PF_PF_BOX = 8;                            // k-steps per L2 prefetch
-constexpr int PF_TMEM_COLS = 512;                       // two fp32 accumulators of up to 256 columns
+constexpr int PF_TMEM_COLS = 512;
+constexpr int PF_SLOT = PF_TMEM_COLS / 2;               // columns of one accumulator slot
+constexpr int PF_NARROW = PF_SLOT / 2;                  // widest tile that fits one slot
 constexpr int PF_MAX_E = 1024;
 
 // warp roles
@@ -69,7 +74,7 @@ struct PfBars {
   uint64_t pk_full[PF_PS], pk_empty[PF_PS];
   uint64_t a_full[PF_SA], a_empty[PF_SA];
   uint64_t b_full[PF_SB], b_empty[PF_SB];
-  uint64_t acc_full, acc_empty, fin;
+  uint64_t acc_full[2], acc_empty[2], fin;
   uint32_t tmem_base;
   int abort;
 };
@@ -330,6 +335,28 @@ __device__ void pf_dequant(const PfGemm &a, uint8_t *sm, PfBars *b, int nt) {
   }
 }
 
+// Accumulator slots, walked the same way by the MMA warp and the epilogue
+// warps: a narrow tile (at most PF_NARROW tokens) takes the next slot, its
+// second accumulator PF_NARROW columns after the first; a wide tile takes both
+// slots, its second accumulator in slot 1. use[s] counts the tiles that took
+// slot s, which gives the phase of that slot's barriers.
+struct AccSlots {
+  uint32_t use[2] = {0, 0};
+  int next = 0;
+  int first, second_off;   // of the current tile
+  bool wide;
+  __device__ void take(int tokens) {
+    wide = tokens > PF_NARROW;
+    first = wide ? 0 : next;
+    second_off = wide ? PF_SLOT : PF_NARROW;
+  }
+  __device__ void done() {
+    ++use[first];
+    if (wide) ++use[1];
+    next = wide ? 0 : first ^ 1;
+  }
+};
+
 // The whole warp runs the loop (waits, descriptor arithmetic) so every value
 // stays warp-uniform; one elected lane issues the tensor-core instructions.
 // Issuing from a lone lane in a divergent branch measured about 2.5x slower
@@ -338,12 +365,16 @@ __device__ void pf_mma(const PfGemm &a, uint8_t *sm, PfBars *b, int nt, uint32_t
   const uint32_t base = smem_u32(sm);
   // descriptors of stage 0; a stage's start address is added in 16-byte units
   const uint64_t da0 = tc05::sw128_desc(base), db0 = tc05::sw128_desc(base + PF_OFF_B);
-  uint32_t g = 0, tc = 0;
+  uint32_t g = 0;
+  AccSlots sl;
   bool issued = false;
   for (int ti = blockIdx.x; ti < nt; ti += gridDim.x) {
     const int4 t = a.tiles[ti];
     const uint32_t idesc = tc05::idesc_bf16_f32(PF_M, (t.w + 15) & ~15);
-    if (!pf_wait_warp(&b->acc_empty, (tc & 1) ^ 1, b, a.status)) goto done;
+    sl.take(t.w);
+    const uint32_t acc0 = tmem + sl.first * PF_SLOT, acc1 = acc0 + sl.second_off;
+    if (!pf_wait_warp(&b->acc_empty[sl.first], (sl.use[sl.first] & 1) ^ 1, b, a.status)) goto done;
+    if (sl.wide && !pf_wait_warp(&b->acc_empty[1], (sl.use[1] & 1) ^ 1, b, a.status)) goto done;
     tc05::fence_after_sync();
     for (int s = 0; s < a.ksteps; ++s, ++g) {
       const int sa = g % PF_SA, sb = g % PF_SB;
@@ -357,17 +388,20 @@ __device__ void pf_mma(const PfGemm &a, uint8_t *sm, PfBars *b, int nt, uint32_t
 #pragma unroll
         for (int kk = 0; kk < PF_KS / 16; ++kk) {
           const uint32_t acc = (s | kk) != 0;
-          tc05::mma_bf16(tmem, d0 + 2 * kk, db + 2 * kk, idesc, acc);
-          tc05::mma_bf16(tmem + 256, d1 + 2 * kk, db + 2 * kk, idesc, acc);
+          tc05::mma_bf16(acc0, d0 + 2 * kk, db + 2 * kk, idesc, acc);
+          tc05::mma_bf16(acc1, d1 + 2 * kk, db + 2 * kk, idesc, acc);
         }
         tc05::commit(&b->a_empty[sa]);
         tc05::commit(&b->b_empty[sb]);
       }
       __syncwarp();
     }
-    if (tc05::elect_one()) tc05::commit(&b->acc_full);
+    if (tc05::elect_one()) {
+      tc05::commit(&b->acc_full[sl.first]);
+      if (sl.wide) tc05::commit(&b->acc_full[1]);
+    }
     __syncwarp();
-    ++tc;
+    sl.done();
   }
 done:
   // every MMA the issuing lane (lane 0: the lowest lane of the converged
@@ -388,17 +422,20 @@ __device__ void pf_epilogue(const PfGemm &a, PfBars *b, int nt, uint32_t tmem) {
   const int q = (threadIdx.x >> 5) & 3, lane = threadIdx.x & 31, par = ew >> 2;
   const int r = 32 * q + lane;
   const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
-  uint32_t tc = 0;
+  AccSlots sl;
   for (int ti = blockIdx.x; ti < nt; ti += gridDim.x) {
     const int4 t = a.tiles[ti];
     const int N = (t.w + 15) & ~15;
-    if (!pf_wait_warp(&b->acc_full, tc & 1, b, a.status, true)) return;
+    sl.take(t.w);
+    const uint32_t ts = tq + sl.first * PF_SLOT, tu = ts + sl.second_off;
+    if (!pf_wait_warp(&b->acc_full[sl.first], sl.use[sl.first] & 1, b, a.status, true)) return;
+    if (sl.wide && !pf_wait_warp(&b->acc_full[1], sl.use[1] & 1, b, a.status, true)) return;
     tc05::fence_after_sync();
     if (a.mode == 0) {
       __nv_bfloat16 *h = a.hout + (size_t)(a.poff[t.x] + t.z) * a.ldh + t.y * PF_M + r;
       for (int c0 = 16 * par; c0 < N; c0 += 32) {
         float gv[16], uv[16];
-        tc05::ld16x2(tq + c0, tq + 256 + c0, gv, uv);
+        tc05::ld16x2(ts + c0, tu + c0, gv, uv);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           // lanes 2m and 2m+1 hold adjacent features: even lanes store the pair
@@ -414,7 +451,7 @@ __device__ void pf_epilogue(const PfGemm &a, PfBars *b, int nt, uint32_t tmem) {
       float *yb = a.y + t.y * (2 * PF_M) + r;
       for (int c0 = 16 * par; c0 < N; c0 += 32) {
         float v0[16], v1[16];
-        tc05::ld16x2(tq + c0, tq + 256 + c0, v0, v1);
+        tc05::ld16x2(ts + c0, tu + c0, v0, v1);
         // lane i < 16 fetches column c0 + i's token and gate; shuffles broadcast them
         int tk = 0;
         float gt = 0.0f;
@@ -436,8 +473,11 @@ __device__ void pf_epilogue(const PfGemm &a, PfBars *b, int nt, uint32_t tmem) {
     }
     tc05::fence_before_sync();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&b->acc_empty);
-    ++tc;
+    if (lane == 0) {
+      mbar_arrive(&b->acc_empty[sl.first]);
+      if (sl.wide) mbar_arrive(&b->acc_empty[1]);
+    }
+    sl.done();
   }
 }
 
@@ -459,8 +499,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) pf_gemm_kernel(const __grid_con
       mbar_init(&b->b_full[i], 1);
       mbar_init(&b->b_empty[i], 1);
     }
-    mbar_init(&b->acc_full, 1);
-    mbar_init(&b->acc_empty, N_EPI);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&b->acc_full[i], 1);
+      mbar_init(&b->acc_empty[i], N_EPI);
+    }
     mbar_init(&b->fin, 1);
     b->abort = 0;
     fence_mbar_init();
@@ -537,7 +579,7 @@ struct PlanArgs {
   const int32_t *status;
 };
 
-// Tiles of at most 256 pairs per expert: the full 256-pair chunks first, in
+// Tiles of at most PF_N pairs per expert: the full PF_N-pair chunks first, in
 // (expert, chunk, feature block) order, then each expert's remainder chunk,
 // largest remainder first (ties by expert index), all feature blocks of one
 // remainder adjacent. CTAs take tiles round-robin.
