@@ -192,6 +192,9 @@ def qmoe_ffn_prefill(experts: qmoe_experts, x, T, idx, gate, k, y, workspace, de
 def qmoe_ffn_prefill_timed(experts: qmoe_experts, x, T, idx, gate, k, y, workspace, dev_status, events,
                            stream=None) -> None:
     """``events``: three torch.cuda.Event(enable_timing=True) objects."""
+    for e in events:
+        if not e.cuda_event:   # torch creates the CUDA event at its first record
+            e.record()
     arr = (_VP * 3)(*[e.cuda_event for e in events])
     _check("qmoe_ffn_prefill_timed", lib().qmoe_ffn_prefill_timed(
         ctypes.byref(experts), _p(x), T, _p(idx), _p(gate), k, _p(y), _p(workspace),
