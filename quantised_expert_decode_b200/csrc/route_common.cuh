@@ -2,13 +2,15 @@
 // logits (used by the decode and prefill routers).
 //
 // Selection order: logit descending, expert index ascending on equal logits.
-// 1. Every logit gets an fp32 key (round-to-nearest of the float64 value, made
-//    order-preserving as an unsigned integer). Rounding is monotone, so the
-//    k largest float64 logits are among the k largest keys, counted with
-//    multiplicity.
-// 2. Rounds of warp max-reductions remove the largest remaining key (all its
-//    copies) until at least k keys are removed; the last removed key is the
-//    threshold and every key >= threshold is a candidate.
+// 1. Every logit gets an fp32 key (round-to-nearest of the float64 value, -0
+//    taken as +0, made order-preserving as an unsigned integer). Rounding is
+//    monotone and equal logits get equal keys, so the k largest float64
+//    logits are among the k largest keys, counted with multiplicity.
+// 2. Threshold: the k-th largest of the 32 per-lane maximum keys (ties by
+//    lane). At least k keys (those lane maxima) are >= it, so it is at most
+//    the k-th largest key and every key >= threshold is a candidate: a
+//    superset of the k largest. One pass of 32 independent shuffles ranks the
+//    lane maxima, instead of k dependent rounds of warp reductions.
 // 3. Candidates are ranked exactly on their float64 logits (index breaks
 //    ties). Ranks below k give the slots.
 // 4. gate_j = exp(l_j - l_0) / sum_j' exp(l_j' - l_0) over the selected slots.
@@ -40,7 +42,7 @@ __device__ inline void warp_topk_gates_m(Get get, int E, int k, int32_t *idx_out
                                          TopkScratch *sc) {
   const int lane = threadIdx.x & 31;
   double val[M];
-  unsigned key[M], rem[M];
+  unsigned key[M];
 #pragma unroll
   for (int j = 0; j < M; ++j) {
     const int e = lane + 32 * j;
@@ -49,28 +51,24 @@ __device__ inline void warp_topk_gates_m(Get get, int E, int k, int32_t *idx_out
 #pragma unroll
   for (int j = 0; j < M; ++j) {
     const int e = lane + 32 * j;
-    key[j] = e < E ? float_key(__double2float_rn(val[j])) : 0u;
-    rem[j] = key[j];
+    // -0 and +0 are equal logits (ranked by index), so they share one key
+    const float f = __double2float_rn(val[j]);
+    key[j] = e < E ? float_key(f == 0.0f ? 0.0f : f) : 0u;
   }
-  unsigned thr = 0;
-  int removed = 0;
-  while (removed < k) {
-    unsigned local = 0;
+  unsigned lmax = 0;
 #pragma unroll
-    for (int j = 0; j < M; ++j) local = max(local, rem[j]);
-    const unsigned mx = __reduce_max_sync(0xffffffffu, local);
-    if (mx == 0u) break;
-    int c = 0;
+  for (int j = 0; j < M; ++j) lmax = max(lmax, key[j]);
+  int rank = 0;   // lanes whose maximum ranks above this lane's
 #pragma unroll
-    for (int j = 0; j < M; ++j) {
-      if (rem[j] == mx) {
-        rem[j] = 0u;
-        ++c;
-      }
-    }
-    removed += (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
-    thr = mx;
+  for (int s2 = 0; s2 < 32; ++s2) {
+    const unsigned o = __shfl_sync(0xffffffffu, lmax, s2);
+    rank += (o > lmax || (o == lmax && s2 < lane)) ? 1 : 0;
   }
+  // ranks are a permutation of 0..31; k <= TOPK_MAX_K <= 32. Lanes without a
+  // valid key have maximum 0, so with fewer than k such lanes thr is 0 and
+  // every valid key is a candidate.
+  const unsigned at = __ballot_sync(0xffffffffu, rank == k - 1);
+  const unsigned thr = __shfl_sync(0xffffffffu, lmax, __ffs(at) - 1);
   // candidates: keys >= thr
   int mine = 0;
 #pragma unroll
