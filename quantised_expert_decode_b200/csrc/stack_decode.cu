@@ -195,15 +195,20 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
   const int G = (int)gridDim.x, c = blockIdx.x;
   const bool rows = c < H16;
   const int r0 = 16 * c;
-  // gate/up units (selected expert j, 16-row tile r) of this CTA, balanced by bytes
+  // gate/up items (selected expert j, matrix gate or up, 16-row tile r) of this
+  // CTA, balanced by bytes. Items, not (gate, up) pairs, are the unit of
+  // assignment: the two halves of a pair meet through the per-block counters
+  // in global memory, and a CTA then holds at most ceil(2 k I16 / G) items (7
+  // for 960 items on 148 CTAs), one per consumer warp, where pairs gave some
+  // CTAs 8 items and one warp two tiles in a row.
   auto wcum = [&](int cc) -> long long {
     const int nr = cc < H16 ? cc : H16;
     return (long long)nr * a.w_rows + (long long)(cc - nr) * a.w_free;
   };
-  const int NU = k * I16;
+  const int NI = 2 * k * I16;   // item i: unit i >> 1 = (j, r), matrix i & 1
   const long long WT = wcum(G);
-  const int ulo = (int)(wcum(c) * NU / WT), uhi = (int)(wcum(c + 1) * NU / WT);
-  const int nunits = uhi - ulo;
+  const int ilo = (int)(wcum(c) * NI / WT), ihi = (int)(wcum(c + 1) * NI / WT);
+  const int nitems = ihi - ilo;
   const int nth = SK_NCW * 32;
   const bool producer = warp == SK_NCW;
 
@@ -350,7 +355,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
       fence_proxy_async();   // ring memory was last read with ordinary loads
       const uint8_t *gu = a.gu[l];
       const int first = nring + ((lane - nring % S) % S + S) % S;  // first item of slot `lane`
-      for (int n = first; lane < S && n < nring + 2 * nunits; n += S) {
+      for (int n = first; lane < S && n < nring + nitems; n += S) {
         const int s = n % S;
         if (n >= S) {
           const long long dl = clock64() + WAIT_BUDGET_CYCLES;
@@ -363,8 +368,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
           }
           if (!ok) break;
         }
-        const int m = (n - nring) >> 1, mat = (n - nring) & 1;
-        const int u = ulo + m, j = u / I16, r = u % I16;
+        const int i = ilo + (n - nring), u = i >> 1, mat = i & 1;
+        const int j = u / I16, r = u % I16;
         const uint8_t *src = gu + (((size_t)st->idx[j] * 2 + mat) * I16 + r) * (size_t)tgu;
         mbar_arrive_expect_tx(&full[s], (uint32_t)tgu);
         bulk_g2s(ring + (size_t)s * a.slot_bytes, src, (uint32_t)tgu, &full[s]);
@@ -374,7 +379,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
         // the h barrier: issue them once this CTA's gate/up tiles have landed
         // (every ring item of the layer acquired), so that they do not compete
         // with the gate/up stream on the critical path.
-        const int want = nring + 2 * nunits;
+        const int want = nring + nitems;
         const long long dl = clock64() + WAIT_BUDGET_CYCLES;
         bool ok = true;
         while (*(volatile int *)&st->turn < want) {
@@ -402,15 +407,15 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
           bulk_g2s(wrtbuf, a.wrt + ((size_t)(l + 1) * H + r0) * E, (uint32_t)(16 * E * 4), wrtbar);
         }
       }
-      nring += 2 * nunits;
+      nring += nitems;
       continue;
     }
 
     // -------------------------------------------------------------------- C --
-    for (int m = warp; m < 2 * nunits; m += SK_NCW) {
+    for (int m = warp; m < nitems; m += SK_NCW) {
       const int n = nring + m;
       if (!wait_full(n)) break;
-      const int u = ulo + (m >> 1), mat = m & 1, j = u / I16, r = u % I16;
+      const int i = ilo + m, u = i >> 1, mat = i & 1, j = u / I16, r = u % I16;
       const float2 o = tile_dot1<BITS, 4>(ring + (size_t)(n % S) * a.slot_bytes, nblkH, limbs, lsc);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[n % S]);
@@ -430,7 +435,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
       }
       if (__shfl_sync(0xffffffffu, last, 0)) quant_h_block(a, j, r >> 1, lane);
     }
-    nring += 2 * nunits;
+    nring += nitems;
     if (!cons_grid_barrier(a, st, tid)) continue;
 
     // -------------------------------------------------------------------- D --
