@@ -135,7 +135,8 @@ __device__ __noinline__ void topk_smem(const double *logits, int E, int k, int32
 // 32-element block, limbs and scales written to global; the block's tile
 // counter is reset for the next layer.
 __device__ __noinline__ void quant_h_block(const StackArgs &a, int j, int b, int lane) {
-  __threadfence();   // the other tiles' a_g / a_u (counted before this warp's increment) are visible
+  // the other tiles' a_g / a_u are visible: their warps released them with
+  // the block counter's increments, which lane 0 acquired with its own
   const int nblkI = a.I / 32;
   const float gv = __ldcg(a.hbuf + (size_t)j * a.I + b * 32 + lane);
   const float uv = __ldcg(a.hbuf + ((size_t)a.k + j) * a.I + b * 32 + lane);
@@ -429,10 +430,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
       // warp that completes the fourth quantises the block
       __syncwarp();
       unsigned last = 0;
-      if (lane == 0) {
-        __threadfence();
-        last = atomicAdd(a.qcnt + (size_t)j * nblkI + (r >> 1), 1u) == 3u;
-      }
+      if (lane == 0)   // release this tile's values; the fourth arriver acquires all four
+        last = atom_add_acq_rel_gpu(a.qcnt + (size_t)j * nblkI + (r >> 1), 1u) == 3u;
       if (__shfl_sync(0xffffffffu, last, 0)) quant_h_block(a, j, r >> 1, lane);
     }
     nring += nitems;
