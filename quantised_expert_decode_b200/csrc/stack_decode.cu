@@ -413,6 +413,15 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
     }
 
     // -------------------------------------------------------------------- C --
+    // Each consumer warp first asks L2 for its own items with ordinary
+    // prefetches. They travel the load path beside the producer's bulk copies
+    // of the same bytes, so more of the layer's weights are in flight per SM.
+    for (int m = warp; m < nitems; m += SK_NCW) {
+      const int i = ilo + m, u = i >> 1, mat = i & 1, j = u / I16, r = u % I16;
+      const uint8_t *src = a.gu[l] + (((size_t)st->idx[j] * 2 + mat) * I16 + r) * (size_t)tgu;
+      for (int off = lane * 128; off < tgu; off += 32 * 128)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(src + off));
+    }
     for (int m = warp; m < nitems; m += SK_NCW) {
       const int n = nring + m;
       if (!wait_full(n)) break;
