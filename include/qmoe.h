@@ -49,7 +49,7 @@ typedef enum {
   QMOE_OK = 0,
   QMOE_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, size out of range */
   QMOE_ERR_GEOMETRY = 2,      /* tensor shapes disagree with the expert handle */
-  QMOE_ERR_UNSUPPORTED = 3,   /* valid request outside what this build supports */
+  QMOE_ERR_UNSUPPORTED = 3,   /* valid request outside what the library supports */
   QMOE_ERR_WORKSPACE = 4,     /* workspace smaller than *_workspace_bytes() */
   QMOE_ERR_CUDA = 5,          /* a CUDA runtime call failed */
   QMOE_ERR_TIMEOUT = 6,       /* a device-side wait exceeded its budget */
