@@ -94,6 +94,12 @@ struct Acc {
 // copy of the code, which keeps the instruction footprint small.
 //   NP = 1: one accumulator tile holds 2 blocks of the token (2 tiles per chunk)
 //   NP >= 2: one tile holds 2 tokens of one block; NQ = NP/2 tiles per block
+// Every variant forms a token's result in the same floating-point order: the
+// blocks of even and of odd index accumulate separately (in increasing block
+// order, each half of a limb pair on its own lane), the two halves are added,
+// then even + odd. So a token's output does not depend on how many tokens of
+// the batch share the expert (NP), and a verify batch reproduces single-token
+// decoding bit for bit.
 template <int BITS, int NP>
 __device__ __noinline__ Acc tile_dot(const uint8_t *tile, int nblk, const uint8_t *limbs, const float2 *lsc,
                                      const int *vid, int n) {
@@ -110,10 +116,12 @@ __device__ __noinline__ Acc tile_dot(const uint8_t *tile, int nblk, const uint8_
   const float wgt = ohalf ? 1.0f : 256.0f;
   const uint8_t *sbase = tile + 64 * nblk * BITS;   // scales follow the codes
   float acc[2][NQ];
+  float acc_odd[2][NQ];   // NP >= 2: odd blocks (for NP == 1 the lanes of pair 1 hold them)
   int pv[NQ], ov[NQ];
 #pragma unroll
   for (int q = 0; q < NQ; ++q) {
     acc[0][q] = acc[1][q] = 0.0f;
+    acc_odd[0][q] = acc_odd[1][q] = 0.0f;
     const int ptq = (NP == 1) ? 0 : 2 * q + pP;
     const int otq = (NP == 1) ? 0 : 2 * q + oP;
     pv[q] = (ptq < n && pslot != 2) ? vid[ptq] : -1;
@@ -174,20 +182,30 @@ __device__ __noinline__ Acc tile_dot(const uint8_t *tile, int nblk, const uint8_
           const uint2 dm = *reinterpret_cast<const uint2 *>(sbase + (bo * 8 + g) * 8);
           const float sw = ss.x * wgt;
           const float mt = ohalf ? 0.0f : ss.y;    // the min term once per pair
-          acc[0][q] = fmaf(h2f(dm.x & 0xffffu), sw * v0, fmaf(h2f(dm.x >> 16), mt, acc[0][q]));
-          acc[1][q] = fmaf(h2f(dm.y & 0xffffu), sw * v1, fmaf(h2f(dm.y >> 16), mt, acc[1][q]));
+          if (NP == 1 || (bo & 1) == 0) {
+            acc[0][q] = fmaf(h2f(dm.x & 0xffffu), sw * v0, fmaf(h2f(dm.x >> 16), mt, acc[0][q]));
+            acc[1][q] = fmaf(h2f(dm.y & 0xffffu), sw * v1, fmaf(h2f(dm.y >> 16), mt, acc[1][q]));
+          } else {
+            acc_odd[0][q] = fmaf(h2f(dm.x & 0xffffu), sw * v0, fmaf(h2f(dm.x >> 16), mt, acc_odd[0][q]));
+            acc_odd[1][q] = fmaf(h2f(dm.y & 0xffffu), sw * v1, fmaf(h2f(dm.y >> 16), mt, acc_odd[1][q]));
+          }
         }
       }
     }
   }
-  // combine the lanes that share a token: the two halves of a pair, and for
-  // NP == 1 also the two pairs (two blocks of the same token)
+  // combine the lanes that share a token: the two halves of a pair, then even
+  // + odd blocks (for NP == 1 the other pair of lanes, else acc_odd)
 #pragma unroll
   for (int q = 0; q < NQ; ++q) {
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       acc[r][q] += __shfl_xor_sync(0xffffffffu, acc[r][q], 1);
-      if (NP == 1) acc[r][q] += __shfl_xor_sync(0xffffffffu, acc[r][q], 2);
+      if (NP == 1) {
+        acc[r][q] += __shfl_xor_sync(0xffffffffu, acc[r][q], 2);
+      } else {
+        acc_odd[r][q] += __shfl_xor_sync(0xffffffffu, acc_odd[r][q], 1);
+        acc[r][q] += acc_odd[r][q];
+      }
     }
   }
   Acc out;

@@ -110,3 +110,35 @@ def test_stack_48_layers_q4_verify_batch():
     stack, x0, _ = _run(cfg, cfg.L)
     _compare(cfg, stack, x0, cfg.L)
     stack.close()
+
+
+def test_verify_batch_equals_single_token_decoding_bit_for_bit():
+    """A verify batch (8 correlated tokens, Q4 experts, per-layer path) reproduces
+    every token decoded alone through the same per-layer path bit for bit:
+    routes, gates and the final activations. A token's arithmetic (exact
+    integer block sums, then one fixed floating-point order) does not depend on
+    which other tokens of the batch share its experts."""
+    cfg = configs.get(3)
+    n_layers = 8
+    layers, routers, biases = device_layers(SEED, cfg, n_layers)
+    batch = DecodeStack(layers, routers, biases, cfg.T, cfg.k, cfg.eps, layerwise=True)
+    one = DecodeStack(layers, routers, biases, 1, cfg.k, cfg.eps, layerwise=True)
+    assert batch.path == 0 and one.path == 0
+    x0 = torch.from_numpy(gen.tokens(SEED, cfg, 0)).cuda()
+    batch.x_in.copy_(x0)
+    batch.decode()
+    torch.cuda.synchronize()
+    assert batch.status() == 0
+    # the batch does share experts, so the multi-token tile variants run
+    idx = to_np(batch.idx)
+    assert min(len(np.unique(idx[l])) for l in range(n_layers)) < cfg.T * cfg.k
+    for t in range(cfg.T):
+        one.x_in.copy_(x0[t:t + 1])
+        one.decode()
+        torch.cuda.synchronize()
+        assert one.status() == 0
+        assert torch.equal(one.idx[:, 0], batch.idx[:, t]), t
+        assert torch.equal(one.gate[:, 0], batch.gate[:, t]), t
+        assert torch.equal(one.x_out[0], batch.x_out[t]), t
+    one.close()
+    batch.close()
