@@ -1,0 +1,65 @@
+"""Host-side logic of bench.py, on the CPU: the ncu-summary traffic lookup, the
+clock-sample summary and the replica throughput arithmetic."""
+import os
+
+import pytest
+
+import bench
+
+
+def test_stored_traffic_parses_the_committed_summaries():
+    for kernel, (fname, _) in bench.TRAFFIC_PROFILES.items():
+        assert os.path.exists(os.path.join(bench.ROOT, "profiles", fname)), fname
+        v = bench.stored_traffic(kernel)
+        # null is allowed (sources changed since the capture); a value must be a byte count
+        assert v is None or v > 1e6, (kernel, v)
+
+
+def test_stored_traffic_is_null_once_the_sources_change(monkeypatch):
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda names: "0" * 16)
+    for kernel in bench.TRAFFIC_PROFILES:
+        assert bench.stored_traffic(kernel) is None
+    assert bench.stored_traffic("no_such_kernel") is None
+
+
+def test_decode_traffic_matches_its_algorithmic_bytes():
+    """The fused decode stack reads each selected expert and each router once:
+    48 x (10 x 1,769,472 + 4,194,304) bytes per token."""
+    v = bench.stored_traffic("stack_decode")
+    if v is None:
+        pytest.skip("decode kernel sources changed since the committed capture")
+    algorithmic = 48 * (10 * 1_769_472 + 4_194_304)
+    assert 1.0 <= v / algorithmic < 1.05
+
+
+def _clock_summary(tmp_path, lines):
+    c = object.__new__(bench.Clocks)
+    c.path = str(tmp_path / "clocks.csv")
+    with open(c.path, "w") as f:
+        f.write("\n".join(lines) + "\n")
+    c.f = open(os.devnull, "w")
+    c.p = None
+    return c.stop()
+
+
+def test_clock_summary_median_max_and_reasons(tmp_path):
+    row = "2026/01/01 00:00:00.000, {sm}, 1965, 700.0, 0x0, {hw}, Not Active, Not Active, {cap}"
+    lines = [row.format(sm=s, hw="Not Active", cap=c) for s, c in
+             ((1965, "Not Active"), (1950, "Active"), (1965, "Not Active"))]
+    s = _clock_summary(tmp_path, lines)
+    assert s["sm_mhz"] == 1965 and s["sm_max_mhz"] == 1965 and s["samples"] == 3
+    assert s["reasons"] == ["sw_power_cap"]
+    lines.append(row.format(sm=1200, hw="Active", cap="Not Active"))
+    s = _clock_summary(tmp_path, lines)
+    assert s["reasons"] == ["hw_slowdown", "sw_power_cap"]
+
+
+def test_clock_summary_without_samples(tmp_path):
+    s = _clock_summary(tmp_path, [])
+    assert s["sm_mhz"] is None and s["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_replica_throughput_sums_work_over_the_slowest_rank():
+    # 4 replicas, 10 steps of 1 token each, slowest rank 20 ms: 40 tokens / 0.02 s
+    assert bench.replica_throughput(4, 10, 1, 20.0) == pytest.approx(2000.0)
+    assert bench.max_over_ranks(3.5, 1) == 3.5
