@@ -1,0 +1,63 @@
+"""The integer arithmetic of the decode contraction, checked on the CPU with its
+rules restated: activations quantised to X with |X| <= 8,355,711 (24-bit fixed
+point per 32-element block), split into three balanced signed 8-bit limbs,
+multiplied by the codes on the integer tensor cores and recombined. Every step
+must be exact for the block sums to be exact integers."""
+import numpy as np
+
+QMAX = 8_355_711   # 127 * 65536 + 127 * 256 + 127
+
+
+def limbs3(X):
+    """Balanced base-256 digits of X, as the decode kernels form them."""
+    X = np.asarray(X, dtype=np.int64)
+    l0 = ((X + 128) & 255) - 128
+    X1 = (X - l0) >> 8
+    l1 = ((X1 + 128) & 255) - 128
+    l2 = (X1 - l1) >> 8
+    return l2, l1, l0
+
+
+def i2f_small(v):
+    """int -> float through the 1.5 * 2^23 magic number (valid for |v| < 2^22)."""
+    bits = (np.int64(0x4B400000) + np.asarray(v, dtype=np.int64)).astype(np.uint32)
+    return bits.view(np.float32) - np.float32(12582912.0)
+
+
+def test_limbs_reconstruct_exactly_and_fit_signed_bytes():
+    rs = np.random.default_rng(1)
+    X = np.concatenate([np.arange(-QMAX, -QMAX + 70000), np.arange(-70000, 70000), np.arange(QMAX - 70000, QMAX + 1),
+                        rs.integers(-QMAX, QMAX + 1, 200000)])
+    l2, l1, l0 = limbs3(X)
+    for l in (l2, l1, l0):
+        assert l.min() >= -128 and l.max() <= 127
+    assert np.array_equal(65536 * l2 + 256 * l1 + l0, X)
+
+
+def test_magic_conversion_is_exact_over_its_range():
+    v = np.arange(-(1 << 22), 1 << 22, dtype=np.int64)
+    assert np.array_equal(i2f_small(v).astype(np.int64), v)
+
+
+def test_block_sums_stay_in_the_exact_ranges():
+    # Q2 codes 0..3, Q4 codes 0..15; |limb| <= 128; 32 products per block
+    hi_q2 = 32 * 3 * (128 * 256 + 128)      # |256 * sum q l2 + sum q l1|
+    hi_q4 = 32 * 15 * (128 * 256 + 128)
+    assert hi_q2 < (1 << 22)                # the magic conversion is exact (Q2)
+    assert hi_q4 < (1 << 24)                # an ordinary int -> fp32 conversion is exact (Q4)
+    assert 32 * QMAX < (1 << 31)            # the block sum of X fits int32
+
+
+def test_recombined_columns_equal_the_code_activation_product():
+    """The hi lanes form (256 * sum q l2 + sum q l1) * 256 and the lo lanes
+    sum q l0; their sum is sum q X for every block, exactly."""
+    rs = np.random.default_rng(2)
+    for bits in (2, 4):
+        q = rs.integers(0, 1 << bits, (1000, 32))
+        X = rs.integers(-QMAX, QMAX + 1, (1000, 32))
+        X[:10] = QMAX
+        X[10:20] = -QMAX
+        l2, l1, l0 = limbs3(X)
+        d2, d1, d0 = (q * l2).sum(1), (q * l1).sum(1), (q * l0).sum(1)
+        hi = (256 * d2 + d1) * 256
+        assert np.array_equal(hi + d0, (q * X).sum(1)), bits
