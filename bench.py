@@ -82,8 +82,8 @@ class Clocks:
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, dev_uuid):
-        self.path = tempfile.mktemp(suffix=".csv")
-        self.f = open(self.path, "w")
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        self.f = os.fdopen(fd, "w")
         args = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "100"]
         if dev_uuid:
             args[1:1] = ["-i", dev_uuid]
