@@ -59,17 +59,15 @@ def run_layer(seed: int, cfg: Config, x: np.ndarray, layer: int = 0):
 def run_stack(seed: int, cfg: Config, x0: np.ndarray, n_layers: int | None = None):
     """Residual stack over the first ``n_layers`` layers (all by default).
 
-    Returns the final activations and per-layer (x_in, idx, gate, y).
-    Experts of a finished layer are dropped to bound host memory.
+    Returns the final activations and per-layer (x_in, idx, gate, y), as
+    ``moe.stack`` computes them on the generated layers. Experts of a finished
+    layer are dropped to bound host memory.
     """
     n = cfg.L if n_layers is None else n_layers
-    x = np.asarray(x0, dtype=np.float64)
-    recs = []
-    for l in range(n):
-        L = Layer(seed, cfg, l)
-        idx, g, _ = moe.route(x, L.Wr, L.bias, cfg.k)
-        y = moe.moe_layer(x, idx, g, L.expert)
-        recs.append((x, idx, g, y))
-        x = moe.rmsnorm_residual(x, y, cfg.eps) if cfg.residual else y
-        L.drop()
-    return x, recs
+
+    def layers():
+        for l in range(n):
+            L = Layer(seed, cfg, l)
+            yield L.Wr, L.bias, L.expert
+            L.drop()
+    return moe.stack(x0, layers(), cfg.k, cfg.eps, residual=cfg.residual)

@@ -299,3 +299,86 @@ def test_stack_keeps_unit_rms():
     x, recs = moe.stack(x0, layers, k, 1e-6)
     assert len(recs) == 3
     assert np.allclose(np.sqrt(np.mean(x * x, axis=1)), 1.0, atol=1e-6)
+
+
+# ----------------------------------------------------- stack composition --
+# Two layers of four constant experts (every weight of a matrix equal) and
+# constant router rows. With constant matrices the expert FFN collapses to a
+# scalar of S = sum_h x_h: a_g = w_g S and a_u = w_u S on every row, so
+# y_e = I w_d w_u S silu(w_g S) on every output element, and a constant router
+# row alpha_e gives the logit alpha_e S. The residual stack is then a chain of
+# plain scalar formulas, worked below in Python floats independently of the
+# oracle's matrix code.
+_SP_H, _SP_I = 64, 32
+_SP_CODES = {0: (3, 2, 1), 1: (2, 3, 0), 2: (1, 3, 3), 3: (0, 0, 2)}   # expert -> (gate, up, down) Q2 code
+_SP_ALPHA = ([2.0 ** -8, 2.0 ** -6, 2.0 ** -7, -2.0 ** -7], [-2.0 ** -6, 2.0 ** -8, 2.0 ** -7, 2.0 ** -6])
+_SP_D, _SP_M = 2.0 ** -6, -1.5 * 2.0 ** -6     # w = d c + m = (c - 1.5) / 64
+
+
+def _sp_layers():
+    H, I = _SP_H, _SP_I
+
+    def const(c, rows, K):
+        return moe.dequantize(np.tile(_const_bytes(2, c, K), (rows, 1)),
+                              np.tile(_scale_bits(_SP_D, _SP_M, K // 32), (rows, 1, 1)), 2)
+    experts = {e: (const(g, I, H), const(u, I, H), const(d, H, I)) for e, (g, u, d) in _SP_CODES.items()}
+    return [(np.tile(np.array(a, dtype=np.float32)[:, None], (1, H)), None, experts.__getitem__)
+            for a in _SP_ALPHA]
+
+
+def _sp_closed_form(x0, mistake=None):
+    """Scalar walk of the stack; ``mistake`` switches in a plausible composition
+    error: "norm_y" normalises y alone (residual dropped), "no_norm" passes
+    x + y on without the norm."""
+    w = lambda c: _SP_D * c + _SP_M
+    silu = lambda a: a / (1.0 + math.exp(-a))
+    x = [float(v) for v in x0]
+    recs = []
+    for alpha in _SP_ALPHA:
+        S = sum(x)
+        logit = [a * S for a in alpha]
+        sel = sorted(range(4), key=lambda e: (-logit[e], e))[:2]      # 4 experts, by hand: value desc, index asc
+        ex = [math.exp(logit[e] - logit[sel[0]]) for e in sel]
+        g = [v / sum(ex) for v in ex]
+        y = 0.0
+        for gj, e in zip(g, sel):
+            cg, cu, cd = _SP_CODES[e]
+            y += gj * _SP_I * w(cd) * w(cu) * S * silu(w(cg) * S)
+        recs.append((sel, g, y))
+        z = [y] * len(x) if mistake == "norm_y" else [xi + y for xi in x]
+        ms = sum(v * v for v in z) / len(z)
+        x = z if mistake == "no_norm" else [v / math.sqrt(ms + 1e-6) for v in z]
+    return np.array(x), recs
+
+
+def test_stack_composition_closed_form():
+    x0 = np.array([[0.5 + h / 64.0 for h in range(_SP_H)]], dtype=np.float32)
+    x, recs = moe.stack(x0, _sp_layers(), 2, 1e-6)
+    ref, ref_recs = _sp_closed_form(x0[0])
+    for (x_in, idx, g, y), (sel, gs, ys) in zip(recs, ref_recs):
+        assert idx[0].tolist() == sel
+        assert np.allclose(g[0], gs, rtol=1e-13, atol=0)
+        assert np.allclose(y[0], ys, rtol=1e-12, atol=1e-15)
+    assert np.allclose(x[0], ref, rtol=1e-12, atol=0)
+    # the pin discriminates: each plausible mistake moves the result far beyond the bound
+    for bad in (_sp_closed_form(x0[0], "norm_y")[0], _sp_closed_form(x0[0], "no_norm")[0]):
+        assert np.max(np.abs(bad - ref)) > 1e-2
+    # routing layer 1 on the un-normalised residual sum changes its gates
+    S_z = float(np.sum(x0[0] + ref_recs[0][2]))
+    assert abs(S_z - float(np.sum(recs[1][0]))) > 1.0
+
+
+def test_workload_stack_is_the_oracle_stack():
+    """``oracle.workload.run_stack`` feeds generated layers to ``moe.stack``
+    (one loop); the per-layer records agree with explicit single-layer calls."""
+    from oracle import workload as W
+    from synth import configs, gen
+    cfg = configs.get(0).with_(L=2, residual=True)
+    x0 = gen.tokens(0, cfg, 0).astype(np.float64)
+    x, recs = W.run_stack(0, cfg, x0, 2)
+    y0, i0, g0, _ = W.run_layer(0, cfg, x0, 0)
+    assert np.array_equal(recs[0][1], i0) and np.array_equal(recs[0][3], y0)
+    x1 = moe.rmsnorm_residual(x0, y0, cfg.eps)
+    y1, i1, _, _ = W.run_layer(0, cfg, x1, 1)
+    assert np.array_equal(recs[1][1], i1)
+    assert np.array_equal(x, moe.rmsnorm_residual(x1, y1, cfg.eps))
