@@ -1,12 +1,19 @@
 #!/usr/bin/env python
-"""Benchmark of the routed-MoE FFN decode path on B200.
+"""Benchmark of the routed-MoE FFN path on B200.
 
-Default workload: the 48-layer decode stack (512 Q2 experts per layer, hidden
-2048, intermediate 768, top-10, one token per step, residual RMSNorm), one CUDA
-graph replay per token. Prints one JSON line on rank 0.
+Default workload (the headline): the 48-layer decode stack (512 Q2 experts
+per layer, hidden 2048, intermediate 768, top-10, one token per step, residual
+RMSNorm), one CUDA graph replay per token, timed with CUDA events over K
+steps after W warm-up steps. The same JSON line then carries two more seeds of
+that workload and the other workloads, each measured on freshly generated
+weights with its own roofline, clocks and CPU-oracle baseline:
+
+  config1_layer    one Q2 decode layer, one token, L2 flushed between steps
+  config3_verify   8 correlated tokens through 48 Q4 layers (verify batch)
+  config4_prefill  a 4096-token bf16 chunk through one Q4 layer
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode48|verify48]
+                    [--workload decode48|verify48|layer|prefill] [--headline-only]
 
 N > 1 runs N independent replicas (one process per GPU under torchrun; the
 path has no exchange step), timed on the device, max over ranks.
@@ -40,6 +47,8 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="decode48", choices=sorted(WORKLOADS))
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--headline-only", action="store_true",
+                   help="decode48: only the 48-layer single-token stack (no extra seeds, no other workloads)")
     p.add_argument("--layers", type=int, default=None,
                    help="decode workloads only: layers in the stack (default: all 48); for small profiling runs")
     p.add_argument("--tokens", type=int, default=None,
@@ -57,13 +66,14 @@ def peaks():
 
 
 def tensor_peak():
-    """Dense bf16 TFLOP/s: the sustained figure (kernels timed inside a long loop)."""
+    """Dense bf16 TFLOP/s for a kernel timed per launch (about half a
+    millisecond, not inside a seconds-long loop): the burst figure."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
             d = json.load(f)
-        return float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured (sustained)"
-    return 1400.0, "fallback (sustained)"
+        return float(d["bf16_tflops"]), "measured (burst)"
+    return 1590.0, "fallback (burst)"
 
 
 def workload_desc(cfg, T):
@@ -76,7 +86,56 @@ def workload_desc(cfg, T):
 
 
 # ------------------------------------------------------------------ clocks --
+REASON_BITS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
+
+
+def summarize_clock_samples(samples, max_mhz):
+    """samples: (sm_mhz, reason_bitmask) pairs taken during a timed region."""
+    if not samples:
+        return {"sm_mhz": None, "sm_max_mhz": max_mhz, "reasons": ["no samples"], "samples": 0}
+    reasons = sorted({n for _, r in samples for n, bit in REASON_BITS if r & bit})
+    return {"sm_mhz": statistics.median(m for m, _ in samples), "sm_max_mhz": max_mhz, "reasons": reasons,
+            "samples": len(samples), "sm_mhz_min": min(m for m, _ in samples)}
+
+
+class NvmlClocks:
+    """SM clock and throttle reasons sampled through NVML every ~2 ms on a
+    host thread while the timed region runs (several samples even for a
+    region of a few tens of milliseconds)."""
+
+    def __init__(self, dev_uuid, period_s=0.002):
+        import threading
+
+        import pynvml
+        pynvml.nvmlInit()
+        self.nv = pynvml
+        self.h = pynvml.nvmlDeviceGetHandleByUUID(dev_uuid)
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.samples = []
+        self.period = period_s
+        self.stop_ev = threading.Event()
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append((float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)),
+                                     int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def stop(self):
+        self.stop_ev.set()
+        self.t.join(timeout=5)
+        return summarize_clock_samples(self.samples, self.max_mhz)
+
+
 class Clocks:
+    """Fallback sampler: nvidia-smi at 100 ms."""
     Q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -115,6 +174,16 @@ class Clocks:
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": reasons, "samples": len(rows)}
+
+
+def clock_sampler(local):
+    import torch
+    props = torch.cuda.get_device_properties(local)
+    uuid = getattr(props, "uuid", None) and f"GPU-{props.uuid}"
+    try:
+        return NvmlClocks(uuid)
+    except Exception:
+        return Clocks(uuid)
 
 
 # ---------------------------------------------------------- dist helpers --
@@ -227,15 +296,17 @@ def oracle_token_time(cfg, x0, n_layers):
     return spent
 
 
-def cpu_baseline(cfg, T):
+def cpu_baseline(cfg, T, n_layers=None, repeats=1):
+    """The oracle on the host cores over ``n_layers`` layers of one step
+    (default: all layers for one token, 2 layers for a batch), ``repeats``
+    times, scaled to the workload's layer count."""
     from synth import gen
-    n = cfg.L if T == 1 else 4
-    x0 = gen.tokens(SEED, cfg, 0)
-    s = oracle_token_time(cfg, x0, n)
-    tok_s = T / (s * cfg.L / n)
+    n = n_layers if n_layers else (cfg.L if T == 1 else 2)
+    s = sum(oracle_token_time(cfg, gen.tokens(SEED, cfg, r), n) for r in range(repeats))
+    tok_s = repeats * T / (s * cfg.L / n)
     return {"value": tok_s, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{T} token(s) through {n} of {cfg.L} layers (float64 NumPy, weight generation "
-                      f"excluded), scaled to {cfg.L} layers; {s:.1f} s of CPU work"}
+            "sample": f"{repeats} step(s) of {T} token(s) through {n} of {cfg.L} layer(s) (float64 NumPy, weight "
+                      f"generation excluded), scaled to {cfg.L} layer(s); {s:.1f} s of CPU work"}
 
 
 # -------------------------------------------------------------- reference --
@@ -296,7 +367,29 @@ def run_reference(args, cfg, T):
 
 
 # ------------------------------------------------------------------- ours --
-def run_ours(args, cfg):
+def init_dist(local, world):
+    import torch
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        if not dist.is_initialized():
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+
+
+def free_device():
+    import gc
+    import torch
+    gc.collect()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def measure_stack(args, cfg, seed=SEED, full=True):
+    """One graph replay per step of the decode stack: device-resident inputs
+    (value), the host-buffer entry point (e2e) and, with ``full``, per-kernel
+    event timing for the roofline. Returns the line's fields."""
     import numpy as np
     import torch
 
@@ -305,139 +398,159 @@ def run_ours(args, cfg):
     from synth.workload import device_layers
 
     rank, world, local = dist_env()
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
     T = cfg.T
-    layers, routers, biases = device_layers(SEED, cfg)
+    layers, routers, biases = device_layers(seed, cfg)
     stack = DecodeStack(layers, routers, biases, T, cfg.k, cfg.eps)
-    tstack = DecodeStack(layers, routers, biases, T, cfg.k, cfg.eps, timing=True)
     n_in = min(args.steps + args.warmup, 4096)
-    xs_host = np.stack([gen.tokens(SEED + 1000 * rank, cfg, s) for s in range(n_in)])   # [n, T, H]
+    xs_host = np.stack([gen.tokens(seed + 1000 * rank, cfg, st) for st in range(n_in)])   # [n, T, H]
     xs = torch.from_numpy(xs_host).cuda()
     stream = torch.cuda.current_stream()
 
-    def step(s):
-        stack.x_in.copy_(xs[s % n_in], non_blocking=True)
+    def step(i):
+        stack.x_in.copy_(xs[i % n_in], non_blocking=True)
         stack.decode(stream)
 
-    for s in range(args.warmup):
-        step(s)
+    for i in range(args.warmup):
+        step(i)
     torch.cuda.synchronize()
     if stack.status() != 0:
         raise RuntimeError("device status set during warm-up")
-    props = torch.cuda.get_device_properties(local)
-    clocks = Clocks(getattr(props, "uuid", None) and f"GPU-{props.uuid}")
+    clocks = clock_sampler(local)
     barrier(world)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for s in range(args.steps):
-        step(args.warmup + s)
+    for i in range(args.steps):
+        step(args.warmup + i)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
-    ms = e0.elapsed_time(e1)
     clk = clocks.stop()
-    ms = max_over_ranks(ms, world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
     value = replica_throughput(world, args.steps, T, ms)
+    if stack.status() != 0:
+        raise RuntimeError("device status set during the timed run")
+    idx = stack.idx.cpu().numpy()
+    uniq = [len(set(idx[l].ravel().tolist())) for l in range(cfg.L)]
+    out = {"value": value, "ms_per_step": ms / args.steps, "clocks": clk,
+           "gpu_launches": args.steps * stack.kernels_per_replay, "seed": seed}
+    if not full:
+        stack.close()
+        del stack, layers, routers, biases, xs
+        free_device()
+        return out
 
     # end to end through the host-buffer entry point (pinned memory)
     xh = torch.from_numpy(xs_host).pin_memory()
     outh = torch.empty((T, cfg.H), dtype=torch.float32).pin_memory()
-    n_e2e = args.steps
     torch.cuda.synchronize()
     barrier(world)
     e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2.record(stream)
-    for s in range(n_e2e):
-        stack.decode_host(xh[s % n_in], outh, stream)
+    for i in range(args.steps):
+        stack.decode_host(xh[i % n_in], outh, stream)
     e3.record(stream)
     torch.cuda.synchronize()
     ms_e2e = max_over_ranks(e2.elapsed_time(e3), world)
     if stack.status() != 0:
-        raise RuntimeError("device status set during the timed run")
+        raise RuntimeError("device status set during the e2e run")
+    stack.close()
 
-    # kernel durations: the same steps through the graph with event nodes around
+    # kernel durations: the same steps through a graph with event nodes around
     # every route and FFN node (event nodes split the programmatic edges, so
-    # this graph is timed separately from the headline)
-    n_t = min(args.steps, 500)
-    for s in range(args.warmup):
-        tstack.x_in.copy_(xs[s % n_in], non_blocking=True)
+    # this graph is timed apart from the headline); the mean over the replays
+    tstack = DecodeStack(layers, routers, biases, T, cfg.k, cfg.eps, timing=True)
+    for i in range(args.warmup):
+        tstack.x_in.copy_(xs[i % n_in], non_blocking=True)
         tstack.decode(stream)
     torch.cuda.synchronize()
-    e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    per_layer = []
-    e4.record(stream)
-    for s in range(n_t):
-        tstack.x_in.copy_(xs[(args.warmup + s) % n_in], non_blocking=True)
+    route_ms = np.zeros(cfg.L)
+    ffn_ms = np.zeros(cfg.L)
+    n_t = args.steps
+    for i in range(n_t):
+        tstack.x_in.copy_(xs[(args.warmup + i) % n_in], non_blocking=True)
         tstack.decode(stream)
-    e5.record(stream)
-    torch.cuda.synchronize()
-    route_ms, ffn_ms = tstack.layer_times()
-    ms_timing_graph = e4.elapsed_time(e5) / n_t
+        r, f = tstack.layer_times()
+        route_ms += np.asarray(r)
+        ffn_ms += np.asarray(f)
+    route_ms /= n_t
+    ffn_ms /= n_t
     if tstack.status() != 0:
         raise RuntimeError("device status set during the timing-graph run")
+    fused = tstack.path == 1
+    phases = None
+    if fused:
+        # median CTA's clock at each phase point of a layer, from the layer's
+        # start, averaged over the layers of the last replay (in microseconds
+        # at the sampled SM clock)
+        tr = tstack.phase_trace().astype(np.float64)                     # [L, CTAs, points]
+        rel = np.median(tr[:, :, 1:7] - tr[:, :, :1], axis=1).mean(axis=0)
+        mhz = clk.get("sm_mhz") or clk.get("sm_max_mhz") or 1965.0
+        names = ["topk_done", "tiles_start", "tiles_done", "barrier1_passed", "down_done", "barrier2_passed"]
+        phases = {n: float(v) / mhz for n, v in zip(names, rel)}
+    tstack.close()
+    del layers, routers, biases, xs
+    free_device()
 
     hbm, peak_kind = peaks()
-    idx = stack.idx.cpu().numpy()
-    uniq = [len(set(idx[l].ravel().tolist())) for l in range(cfg.L)]
     ffn_bytes = [u * cfg.expert_bytes() for u in uniq]
     expert_bytes_step = sum(ffn_bytes)
     router_bytes_step = cfg.L * cfg.router_bytes()
     step_s = ms / 1e3 / args.steps
-    fused = stack.path == 1
     if fused:
         # one persistent kernel per token: it streams every expert and router byte
-        kernel = "stack_decode_kernel (fused 48-layer decode)"
+        kernel = "stack_decode_kernel (fused decode stack, one launch per token)"
         launch_bytes = float(expert_bytes_step + router_bytes_step)
-        launch_s = sum(ffn_ms) / 1e3
+        launch_s = float(ffn_ms.sum()) / 1e3
         achieved = launch_bytes / launch_s / 1e9
     else:
-        kernel = "ffn_decode_kernel"
-        launch_bytes = statistics.mean(ffn_bytes)
-        launch_s = statistics.mean(ffn_ms) / 1e3
+        kernel = "ffn_decode_kernel (one launch per layer)"
+        launch_bytes = float(statistics.mean(ffn_bytes))
+        launch_s = float(ffn_ms.mean()) / 1e3
         achieved = statistics.mean(b / (t / 1e3) for b, t in zip(ffn_bytes, ffn_ms)) / 1e9
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "u8 codes x s8 activation limbs -> s32 (tensor core), f32 epilogue, f64 router",
-        "data": "synthetic (seeded SplitMix64 weights, Box-Muller activations)",
-        "config": dict(workload_desc(cfg, T), parallelism=f"replicas x{world}"),
+    out.update({
         "roofline": {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": hbm,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
                      "traffic": stored_traffic("stack_decode") if (fused and cfg.L == 48) else None,
-                     "algorithmic_bytes_per_launch": launch_bytes,
-                     "avg_launch_us": 1e6 * launch_s,
-                     "timing": "CUDA event nodes around the kernel node(s) of a graph replayed over the same "
-                               "steps (last replay)"},
+                     "algorithmic_bytes_per_launch": launch_bytes, "avg_launch_us": 1e6 * launch_s,
+                     "timing": f"CUDA event nodes around the kernel node(s) of a graph, mean of {n_t} replays"},
         "stack": {"path": "fused persistent kernel" if fused else "per-layer kernels (route + FFN) with PDL",
                   "expert_bytes_per_step": expert_bytes_step, "router_bytes_per_step": router_bytes_step,
                   "expert_GBps": expert_bytes_step / step_s / 1e9,
                   "all_weight_GBps": (expert_bytes_step + router_bytes_step) / step_s / 1e9,
                   "frac_all_weight_of_measured_hbm": (expert_bytes_step + router_bytes_step) / step_s / 1e9 / hbm,
                   "frac_expert_of_8TBps": expert_bytes_step / step_s / 8e12,
-                  "route_us_mean": 1e3 * statistics.mean(route_ms), "ffn_us_mean": 1e3 * statistics.mean(ffn_ms),
-                  "ms_per_step_event_graph": ms_timing_graph,
+                  "route_us_mean": 1e3 * float(route_ms.mean()), "ffn_us_mean": 1e3 * float(ffn_ms.mean()),
+                  "fused_phase_us_from_layer_start": phases,
                   "unique_experts_per_layer_mean": statistics.mean(uniq),
                   "reuse_pairs_per_unique_expert": T * cfg.k / statistics.mean(uniq)},
-        "e2e": {"value": world * n_e2e * T / (ms_e2e / 1e3), "unit": "tokens/s",
+        "e2e": {"value": world * args.steps * T / (ms_e2e / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * cfg.H * 4, "d2h_bytes_per_step": T * cfg.H * 4,
                 "path": "qmoe_stack_decode_host: pinned host x -> graph replay -> pinned host output"},
-        "clocks": clk,
-        "gpu_launches": args.steps * stack.kernels_per_replay,
+    })
+    return out
+
+
+def stack_line(args, cfg, m):
+    rank, world, _ = dist_env()
+    T = cfg.T
+    line = {
+        "metric": METRIC, "value": m["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u8 codes x s8 activation limbs -> s32 (tensor core), f32 epilogue, f64 router",
+        "data": "synthetic (seeded SplitMix64 weights, Box-Muller activations)",
+        "config": dict(workload_desc(cfg, T), parallelism=f"replicas x{world}"),
+        "roofline": m["roofline"], "stack": m["stack"], "e2e": m["e2e"], "clocks": m["clocks"],
+        "gpu_launches": m["gpu_launches"],
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, T)
-    stack.close()
-    tstack.close()
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    return line
+
+
+def sub_line(line, keep=("value", "unit", "ms_per_step", "config", "roofline", "cpu_baseline", "e2e", "clocks",
+                         "gpu_launches", "stack", "prefill", "metric", "route_us_mean")):
+    return {k: v for k, v in line.items() if k in keep}
 
 
 def run_layer(args, cfg):
@@ -451,12 +564,11 @@ def run_layer(args, cfg):
     from synth.workload import device_layers
 
     rank, world, local = dist_env()
-    torch.cuda.set_device(local)
     layers, routers, _ = device_layers(SEED, cfg, 1)
     layer, Wr = layers[0], routers[0]
     T = cfg.T
     n_in = args.steps + args.warmup
-    xs = torch.from_numpy(np.stack([gen.tokens(SEED, cfg, s) for s in range(n_in)])).cuda()
+    xs = torch.from_numpy(np.stack([gen.tokens(SEED + 1000 * rank, cfg, i) for i in range(n_in)])).cuda()
     idx = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
     gate = torch.empty((T, cfg.k), dtype=torch.float32, device="cuda")
     y = torch.empty((T, cfg.H), dtype=torch.float32, device="cuda")
@@ -464,51 +576,68 @@ def run_layer(args, cfg):
     rws = torch.zeros(q.qmoe_route_workspace_bytes(T, cfg.E), dtype=torch.uint8, device="cuda")
     fws = torch.zeros(q.qmoe_decode_workspace_bytes(T, cfg.k, cfg.H, cfg.I), dtype=torch.uint8, device="cuda")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device="cuda")     # 256 MB
+    flush_sink = torch.empty(1, dtype=torch.float32, device="cuda")
     h = layer.handle()
     stream = torch.cuda.current_stream()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
 
-    def step(s, e=None):
-        flush.fill_(s & 255)
+    def step(i, e=None):
+        # flush: a 256 MB write evicts the layer's weights from L2; a 256 MB
+        # read then evicts the dirty lines the write left, so their write-back
+        # to HBM happens here and not inside the timed kernels
+        flush.fill_(i & 255)
+        torch.sum(flush_rd, out=flush_sink)
         if e:
             e[0].record(stream)
-        q.qmoe_route(Wr, None, xs[s], q.F32, T, cfg.H, cfg.E, cfg.k, idx, gate, rws, st, stream)
+        q.qmoe_route(Wr, None, xs[i], q.F32, T, cfg.H, cfg.E, cfg.k, idx, gate, rws, st, stream)
         if e:
             e[1].record(stream)
-        q.qmoe_ffn_decode(h, xs[s], T, idx, gate, cfg.k, y, fws, st, stream)
+        q.qmoe_ffn_decode(h, xs[i], T, idx, gate, cfg.k, y, fws, st, stream)
         if e:
             e[2].record(stream)
 
-    for s in range(args.warmup):
-        step(s)
+    for i in range(args.warmup):
+        step(i)
     torch.cuda.synchronize()
-    for s in range(args.steps):
-        step(args.warmup + s, ev[s])
+    clocks = clock_sampler(local)
+    barrier(world)
+    for i in range(args.steps):
+        step(args.warmup + i, ev[i])
     torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
     if q.qmoe_read_status(st) != 0:
         raise RuntimeError("device status set")
     route_ms = [e[0].elapsed_time(e[1]) for e in ev]
     ffn_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    layer_s = (sum(route_ms) + sum(ffn_ms)) / 1e3
+    layer_ms = max_over_ranks(sum(route_ms) + sum(ffn_ms), world)
     hbm, peak_kind = peaks()
     ffn_bytes = cfg.k * cfg.expert_bytes()
     achieved = ffn_bytes / (statistics.mean(ffn_ms) / 1e3) / 1e9
     line = {"metric": "routed-MoE decode layer tokens/s (one layer); HBM GB/s on expert bytes vs peak",
-            "value": args.steps * T / layer_s, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": 1e3 * layer_s / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None,
+            "value": replica_throughput(world, args.steps, T, layer_ms), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": layer_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "u8 codes x s8 activation limbs -> s32 (tensor core), f32 epilogue, f64 router",
             "data": "synthetic",
             "config": {"workload": f"one decode layer: {cfg.E} Q{cfg.fmt} experts, hidden {cfg.H}, intermediate "
-                                   f"{cfg.I}, top-{cfg.k}, {T} token; L2 flushed (256 MB write) between steps"},
+                                   f"{cfg.I}, top-{cfg.k}, {T} token; L2 flushed between steps (256 MB write, "
+                                   f"then 256 MB read); "
+                                   f"step time = route + FFN kernel time (the flush excluded)"},
             "roofline": {"bound": "hbm", "kernel": "ffn_decode_kernel", "achieved": achieved, "peak": hbm,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
                          "traffic": None, "algorithmic_bytes_per_launch": ffn_bytes,
                          "avg_launch_us": 1e3 * statistics.mean(ffn_ms),
-                         "median_launch_us": 1e3 * statistics.median(ffn_ms)},
-            "route_us_mean": 1e3 * statistics.mean(route_ms),
+                         "median_launch_us": 1e3 * statistics.median(ffn_ms),
+                         "timing": "CUDA events on the launching stream around each launch"},
+            "route_us_mean": 1e3 * statistics.mean(route_ms), "clocks": clk,
             "gpu_launches": 2 * args.steps}
-    print(json.dumps(line), flush=True)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, T, n_layers=1, repeats=3)
+    del layers, routers, xs, flush, flush_rd
+    free_device()
+    return line
 
 
 # ---------------------------------------------------------------- prefill --
@@ -589,11 +718,6 @@ def run_prefill(args, cfg):
     from synth.workload import device_layers
 
     rank, world, local = dist_env()
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
     T, k, E, H, I = cfg.T, cfg.k, cfg.E, cfg.H, cfg.I
     layers, routers, biases = device_layers(SEED, cfg, 1)
     layer, Wr, bias = layers[0], routers[0], biases[0]
@@ -626,8 +750,7 @@ def run_prefill(args, cfg):
     torch.cuda.synchronize()
     if int(st.item()) != 0:
         raise RuntimeError("device status set during warm-up")
-    props = torch.cuda.get_device_properties(local)
-    clocks = Clocks(getattr(props, "uuid", None) and f"GPU-{props.uuid}")
+    clocks = clock_sampler(local)
     barrier(world)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -646,6 +769,25 @@ def run_prefill(args, cfg):
     g1_ms = [es[0].elapsed_time(es[1]) for es in ev]
     g2_ms = [es[1].elapsed_time(es[2]) for es in ev]
     value = replica_throughput(world, args.steps, T, ms)
+
+    # the same steps with the earlier combine (fp32 atomic additions into y,
+    # not reproducible bit for bit), to record what the slot-ordered combine costs
+    ev_a = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for es in ev_a:
+        for e in es:
+            e.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e4.record(stream)
+    for i in range(args.steps):
+        x = xs[(args.warmup + i) % n_in]
+        q.qmoe_route(Wr, bias, x, L.BF16, T, H, E, k, idx, gate, rws, st, stream)
+        q.qmoe_ffn_prefill_timed(h, x, T, idx, gate, k, y, pws, st, ev_a[i], stream, flags=L.PREFILL_ATOMIC_COMBINE)
+    e5.record(stream)
+    torch.cuda.synchronize()
+    ms_atomic = max_over_ranks(e4.elapsed_time(e5), world)
+    g2a_ms = [es[1].elapsed_time(es[2]) for es in ev_a]
 
     # end to end: pinned bf16 x -> device, route + FFN, y -> pinned host
     xh = [torch.from_numpy(a).pin_memory() for a in xs_host]
@@ -689,7 +831,13 @@ def run_prefill(args, cfg):
                     "gemm2_us": 1e6 * t2, "ffn_gemms_frac": f_layer / (t1 + t2) / 1e12 / peak,
                     "layer_TFLOPs_per_step": f_layer / (ms / 1e3 / args.steps) / 1e12,
                     "pairs": pairs, "active_experts": int((counts > 0).sum()), "max_expert_load": int(counts.max()),
-                    "mma_columns_padded_over_pairs": padded / pairs},
+                    "mma_columns_padded_over_pairs": padded / pairs,
+                    "combine": {"kind": "slot-ordered (GEMM 2 writes gate-scaled pair rows, a combine kernel adds "
+                                        "each token's rows in slot order): reproducible bit for bit",
+                                "ms_per_step": ms / args.steps,
+                                "atomic_ms_per_step": ms_atomic / args.steps,
+                                "gemm2_us_atomic": 1e3 * statistics.mean(g2a_ms),
+                                "cost_vs_atomic": ms / ms_atomic - 1.0}},
         "e2e": {"value": world * args.steps * T / (ms_e2e / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 4,
                 "path": "pinned bf16 x -> device, qmoe_route + qmoe_ffn_prefill, y -> pinned host"},
@@ -697,15 +845,13 @@ def run_prefill(args, cfg):
         "gpu_launches": launches,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        per_tok, tr, tf = oracle_prefill_time(cfg, 16)
+        per_tok, tr, tf = oracle_prefill_time(cfg, 8)
         line["cpu_baseline"] = {"value": 1.0 / per_tok, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"routing of all {T} tokens ({tr:.1f} s, charged per token) + expert FFNs "
-                                          f"and combine of 16 tokens ({tf:.1f} s); weight generation excluded"}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+                                          f"and combine of 8 tokens ({tf:.1f} s); weight generation excluded"}
+    del layers, routers, biases, xs, pws
+    free_device()
+    return line
 
 
 def main():
@@ -718,14 +864,37 @@ def main():
         cfg = cfg.with_(L=args.layers)
     if args.impl == "reference" and args.workload == "prefill":
         run_prefill_reference(args, cfg)
-    elif args.impl == "reference":
+        return
+    if args.impl == "reference":
         run_reference(args, cfg, cfg.T)
-    elif args.workload == "prefill":
-        run_prefill(args, cfg)
+        return
+    rank, world, local = dist_env()
+    init_dist(local, world)
+    if args.workload == "prefill":
+        line = run_prefill(args, cfg)
     elif args.workload == "layer":
-        run_layer(args, cfg)
+        line = run_layer(args, cfg)
     else:
-        run_ours(args, cfg)
+        line = stack_line(args, cfg, measure_stack(args, cfg))
+        if args.workload == "decode48" and not args.headline_only:
+            # the headline workload with two more seeds (weights and tokens),
+            # then the other workloads, each on freshly generated weights
+            line["seeds"] = [{"seed": SEED, "value": line["value"], "ms_per_step": line["ms_per_step"]}]
+            for sd in (SEED + 1, SEED + 2):
+                m = measure_stack(args, cfg, seed=sd, full=False)
+                line["seeds"].append({"seed": sd, "value": m["value"], "ms_per_step": m["ms_per_step"],
+                                      "clocks": m["clocks"]})
+            line["config1_layer"] = sub_line(run_layer(args, configs.get(1)))
+            c3 = configs.get(3)
+            line["config3_verify"] = sub_line(stack_line(args, c3, measure_stack(args, c3)))
+            line["config4_prefill"] = sub_line(run_prefill(args, configs.get(4)))
+            line["gpu_launches_all_workloads"] = (line["gpu_launches"] + sum(
+                line[k_]["gpu_launches"] for k_ in ("config1_layer", "config3_verify", "config4_prefill")))
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
 
 
 if __name__ == "__main__":

@@ -53,7 +53,9 @@ typedef enum {
   QMOE_ERR_WORKSPACE = 4,     /* workspace smaller than *_workspace_bytes() */
   QMOE_ERR_CUDA = 5,          /* a CUDA runtime call failed */
   QMOE_ERR_TIMEOUT = 6,       /* a device-side wait exceeded its budget */
-  QMOE_ERR_DEVICE_STATUS = 7  /* invalid routed index seen on the device */
+  QMOE_ERR_DEVICE_STATUS = 7, /* invalid routed index seen on the device */
+  QMOE_ERR_RANGE = 8          /* decode activations too large for the exact router sums:
+                                 a 16-element slice's partial logit reached 2^33 */
 } qmoe_status;
 
 enum { QMOE_Q2 = 2, QMOE_Q4 = 4 };        /* block formats (bits per code) */
@@ -65,8 +67,9 @@ enum { QMOE_GATE_UP = 0, QMOE_DOWN = 1 }; /* packed matrix kinds */
  *   down   : E experts x down [H,I]               (reduction axis I)
  * gate_up_bytes / down_bytes are the sizes of the two buffers; a handle whose
  * sizes differ from qmoe_packed_bytes() of its E/H/I/fmt is refused with
- * QMOE_ERR_GEOMETRY ("a wrong expert geometry must be refused rather than
- * mis-indexed", [P3] "Understanding the Architecture").
+ * QMOE_ERR_GEOMETRY: the expert-source contract of [P3] "Understanding the
+ * Architecture" turns a geometry mismatch into an error instead of reading
+ * the wrong rows.
  * Geometry limits: H and I multiples of 128; E <= 1024. */
 typedef struct {
   int E, H, I, fmt;
@@ -106,8 +109,8 @@ qmoe_status qmoe_pack(int fmt, int kind, int E, int H, int I,
 
 /* ---------------------------------------------------------------- router --
  * Router GEMV, softmax, top-k with renormalised gates ([P3] router_top10.cu,
- * "Understanding the Architecture"; "the router names ten experts per token",
- * [P3] end-to-end paragraph). For each token t:
+ * "Understanding the Architecture"; ten experts per token in [P3]'s end-to-end
+ * walk-through). For each token t:
  *   l[t,e] = sum_h x[t,h] * Wr[e,h] (+ bias[e])     accumulated in float64
  *   idx[t,:] = the k largest l[t,:], by value descending, ties to lower e
  *   gate[t,j] = exp(l[t,idx[t,j]] - l[t,idx[t,0]]) / sum_j' exp(...)
@@ -126,8 +129,8 @@ qmoe_status qmoe_route(const float *Wr, const float *bias, const void *x, int x_
                        void *workspace, size_t workspace_bytes, int32_t *dev_status,
                        qmoe_stream_t stream);
 
-/* Residual RMSNorm fused in front of the router (the residual stack every
- * block reads and writes, [P3] "Understanding the Architecture"):
+/* Residual RMSNorm fused in front of the router (the gated residual stream
+ * shared by all blocks, [P3] "Understanding the Architecture"):
  *   x_out[t,:] = z / sqrt(mean(z^2) + eps),  z = x_in[t,:] + y[t,:]
  * then routes x_out exactly like qmoe_route (fp32 activations, T <= 8).
  * x_out must not alias x_in or y. */
@@ -137,8 +140,9 @@ qmoe_status qmoe_residual_route(const float *x_in, const float *y, float eps, fl
                                 size_t workspace_bytes, int32_t *dev_status,
                                 qmoe_stream_t stream);
 
-/* Standalone residual RMSNorm: x_out = RMSNorm(x_in + y), fp32 [T,H]. x_out
- * may alias x_in. */
+/* Standalone residual RMSNorm: x_out = RMSNorm(x_in + y), fp32 [T,H], with the
+ * same arithmetic as the norm inside qmoe_residual_route (and the fused stack).
+ * x_out may alias x_in. H a multiple of 16. */
 qmoe_status qmoe_rmsnorm_residual(const float *x_in, const float *y, float eps, float *x_out,
                                   int T, int H, qmoe_stream_t stream);
 
@@ -176,8 +180,9 @@ qmoe_status qmoe_route_fixed(const float *Wr, const float *bias, const float *x,
  * x fp32 [T,H]; idx int32 [T,k]; gate fp32 [T,k]; y fp32 [T,H] (overwritten).
  * Limits: 1 <= T <= 8, 1 <= k <= 16. One cooperative grid of one CTA per SM:
  * weights stream through shared memory with bulk asynchronous copies and are
- * contracted on tensor cores (codes x 16-bit fixed-point activations, exact
- * integer products, fp32 scaling per block).
+ * contracted on tensor cores (codes x activations in 24-bit fixed point per
+ * 32-element block, held as three signed 8-bit limbs; exact integer block
+ * sums, fp32 scaling per block).
  * Workspace: qmoe_decode_workspace_bytes(T, k, H, I), zeroed once before first
  * use (every completed call leaves its barrier words as it found them).
  * Errors: GEOMETRY if the handle's H/I/E do not match; device status for an
@@ -218,30 +223,39 @@ qmoe_status qmoe_bucket(const int32_t *idx, int T, int k, int E, int32_t *offset
  * GEMMs on the tcgen05 tensor cores - bf16 operands (Q4 weights dequantised
  * to bf16 in shared memory, w = bf16(d)*q + bf16(m) rounded once), fp32
  * accumulation in tensor memory; the intermediate silu(g)*u is rounded to
- * bf16 between the two GEMMs; the gate-weighted combine is a sum of fp32
- * atomic additions, so its order (and the last bits of y) may vary between
- * runs. Expected relative error against exact arithmetic: about 1e-3.
+ * bf16 between the two GEMMs. The second GEMM writes every routed pair's
+ * gate-scaled output row (fp32, in bucket order) to the workspace, and a
+ * combine kernel adds each token's k rows in slot order, so y is the same bit
+ * for bit on every run. Measured relative error against the float64 oracle
+ * at the 4096-token workload: about 8e-3 rel-RMS (bf16 operands), every token
+ * row below 2e-2.
  * Limits: fmt Q4, H a multiple of 256, I a multiple of 128, k <= E <= 1024,
- * T*k <= 2^28. Workspace: qmoe_prefill_workspace_bytes(T, k, E, H, I) bytes,
- * no initialisation needed. *dev_status must be 0 on entry (a nonzero value
- * skips the GEMMs); an index outside [0, E) or an expert repeated within one
- * token's route sets it. */
+ * T*k <= 2^28. Workspace: qmoe_prefill_workspace_bytes(T, k, E, H, I) bytes
+ * (T*k*H*4 of it for the pair rows), no initialisation needed. *dev_status
+ * must be 0 on entry (a nonzero value skips the GEMMs); an index outside
+ * [0, E) or an expert repeated within one token's route sets it. */
 size_t qmoe_prefill_workspace_bytes(int T, int k, int E, int H, int I);
 qmoe_status qmoe_ffn_prefill(const qmoe_experts *experts, const void *x, int T, const int32_t *idx,
                              const float *gate, int k, float *y, void *workspace, size_t workspace_bytes,
                              int32_t *dev_status, qmoe_stream_t stream);
 /* qmoe_ffn_prefill with kernel timing: events is a host array of three
  * cudaEvent_t (created by the caller, timing enabled) recorded on `stream`
- * right before the first grouped GEMM, between the two, and after the second;
- * cudaEventElapsedTime of consecutive pairs gives the two GEMM durations. */
+ * right before the first grouped GEMM, between the two, and after the second
+ * (before the combine); cudaEventElapsedTime of consecutive pairs gives the
+ * two GEMM durations. flags: 0, or QMOE_PREFILL_ATOMIC_COMBINE for the
+ * earlier combine (fp32 atomic additions straight into y from the second
+ * GEMM; no combine kernel, run-to-run variation in y's last bits), kept to
+ * measure one against the other. */
+enum { QMOE_PREFILL_ATOMIC_COMBINE = 1 };
 qmoe_status qmoe_ffn_prefill_timed(const qmoe_experts *experts, const void *x, int T, const int32_t *idx,
                                    const float *gate, int k, float *y, void *workspace, size_t workspace_bytes,
-                                   int32_t *dev_status, qmoe_stream_t stream, void *const *events);
+                                   int32_t *dev_status, qmoe_stream_t stream, void *const *events, int flags);
 
 /* ------------------------------------------------------------ layer stack --
  * L layers of route -> FFN -> residual RMSNorm captured once into one CUDA
- * graph ([P3]: 48 captured layer graphs; "a graph bakes in its arguments, so
- * per-token values arrive through fixed-address device buffers").
+ * graph ([P3] "Understanding the Architecture": 48 captured layer graphs; a
+ * captured graph keeps the pointers it was recorded with, so each token's
+ * values are written into buffers whose addresses never change).
  *   x_0 = input;  for l: (idx_l, gate_l) = route_l(x_l);  y_l = FFN_l(x_l);
  *                       x_{l+1} = RMSNorm(x_l + y_l)
  *   output = x_L
@@ -260,7 +274,7 @@ typedef struct {
   const float *const *Wr;      /* L device pointers, fp32 [E,H] */
   const float *const *bias;    /* NULL or L device pointers (entries may be NULL) */
   const qmoe_experts *layers;  /* L handles with identical E/H/I/fmt */
-  int flags;                   /* 0 or QMOE_STACK_TIMING */
+  int flags;                   /* 0 or a combination of QMOE_STACK_TIMING, QMOE_STACK_LAYERWISE */
 } qmoe_stack_desc;
 
 typedef struct qmoe_stack qmoe_stack;
@@ -278,6 +292,13 @@ qmoe_status qmoe_stack_buffers(const qmoe_stack *stack, float **x_in, float **x_
 /* Kernel launches in one replay of the stack's graph: 2L + 1 on the per-layer
  * path, 1 on the fused path. */
 int qmoe_stack_kernels_per_replay(const qmoe_stack *stack);
+/* Device address of the fused path's 32-bit grid-barrier counter inside the
+ * stack's workspace (bit 31 flips once per grid barrier; it must read zero
+ * between replays), or NULL on the per-layer path. For diagnostics and for
+ * tests that make a barrier run out of its time budget: a counter preset to
+ * 0x7FFFFFFF can never complete for some CTAs, so the replay ends with
+ * QMOE_ERR_TIMEOUT after about one second instead of hanging. */
+uint32_t *qmoe_stack_barrier_word(const qmoe_stack *stack);
 /* Which path the stack runs. QMOE_PATH_FUSED (single-token stacks whose
  * geometry fits one SM's shared memory): one persistent kernel runs all L
  * layers with two grid barriers per layer; router logits there are formed from
@@ -285,13 +306,23 @@ int qmoe_stack_kernels_per_replay(const qmoe_stack *stack);
  * float64 dot product per expert. QMOE_PATH_LAYERWISE: qmoe_residual_route and
  * qmoe_ffn_decode per layer, chained with programmatic dependent launch. */
 int qmoe_stack_path(const qmoe_stack *stack);
-/* Per-layer durations (ms) of the most recent completed replay, measured by
- * the event nodes of a QMOE_STACK_TIMING stack: route_ms[l] spans layer l's
- * router (with its fused residual RMSNorm), ffn_ms[l] its FFN kernel. Host
- * arrays of L floats (either may be NULL). Synchronous; UNSUPPORTED without
- * the flag. On the fused path the single kernel's duration is split evenly:
- * route_ms[l] = 0 and ffn_ms[l] = kernel / L. */
+/* Per-layer durations (ms) of the most recent completed replay of a
+ * QMOE_STACK_TIMING stack: route_ms[l] spans layer l's router (with its fused
+ * residual RMSNorm), ffn_ms[l] its FFN. Host arrays of L floats (either may be
+ * NULL). Synchronous; UNSUPPORTED without the flag. Per-layer path: event
+ * nodes around every kernel node. Fused path: the kernel's event-timed
+ * duration split over the layers in proportion to each layer's median CTA
+ * clock span; route_ms[l] is the part from the layer's start to its top-k. */
 qmoe_status qmoe_stack_layer_times(const qmoe_stack *stack, float *route_ms, float *ffn_ms);
+/* Raw phase stamps of the most recent replay of a QMOE_STACK_TIMING fused
+ * stack: SM clock cycles (clock64 of each CTA's first consumer thread, so
+ * compare only stamps of one CTA), int64 [L][*ctas][*points]: layer start,
+ * top-k done, gate/up tiles start, gate/up tiles done, first grid barrier
+ * passed, down tiles and router partials done, second grid barrier passed
+ * (slot 7 unused). count is the capacity of cycles_host in entries (WORKSPACE
+ * if too small). UNSUPPORTED on the per-layer path or without the flag.
+ * Synchronises the device. */
+qmoe_status qmoe_stack_trace(const qmoe_stack *stack, int64_t *cycles_host, size_t count, int *ctas, int *points);
 /* One graph replay on `stream`: reads the stack's input buffer, writes its
  * output buffer. */
 qmoe_status qmoe_stack_decode(qmoe_stack *stack, qmoe_stream_t stream);

@@ -12,20 +12,20 @@ What is computed, and where it comes from:
   with 2-bit (Q2) or 4-bit (Q4) codes ``q``.  The pages name only third-party
   GGUF quant types (pyshine Strata tour, "How It Works"); the format here is
   the one the workload definitions fix.
-* Router: logits ``l = Wr x (+ b)``; the ``k`` largest are selected ("the
-  router names ten experts per token", pyshine Strata tour, end-to-end
-  paragraph; router kernel ``router_top10.cu``, same page, "Understanding the
+* Router: logits ``l = Wr x (+ b)``; the ``k`` largest are selected (ten
+  experts per token in the pyshine Strata tour's end-to-end walk-through;
+  router kernel ``router_top10.cu``, same page, "Understanding the
   Architecture"), ties to the lower expert index; gates are the softmax over
   the selected logits, which equals softmax over all experts followed by
   renormalisation over the selection.
 * Expert FFN: ``h = silu(Wg x) * (Wu x)``, ``y_e = Wd h`` with
   ``silu(a) = a / (1 + exp(-a))``.
 * Combine: ``y = sum_j g_j y_{e_j}`` in slot order, applied once on the device
-  side of the engine ("moe_combine ... does that summation", pyshine Strata
+  side of the engine (the device-side ``moe_combine`` of the pyshine Strata
   tour, "Understanding the Architecture").
 * Residual stack: ``x <- RMSNorm(x + y)`` with ``eps = 1e-6`` and no learned
-  gain ("gated residual stack that every block reads and writes", same
-  section; the reduced form is the plainest reading).
+  gain (the gated residual stream shared by all blocks, same section; the
+  reduced form is the plainest reading).
 
 Logits are certified: they are computed with a float64 matrix product, and
 every token whose top-(k+1) ordering could be changed by that product's

@@ -22,7 +22,7 @@ STACK_LAYERWISE = 2
 PATH_LAYERWISE, PATH_FUSED = 0, 1
 
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "GEOMETRY", 3: "UNSUPPORTED", 4: "WORKSPACE",
-                5: "CUDA", 6: "TIMEOUT", 7: "DEVICE_STATUS"}
+                5: "CUDA", 6: "TIMEOUT", 7: "DEVICE_STATUS", 8: "RANGE"}
 
 
 class QmoeError(RuntimeError):
@@ -59,12 +59,14 @@ _SIGS = {
     "qmoe_prefill_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "qmoe_ffn_prefill": (_I, [ctypes.POINTER(qmoe_experts), _VP, _I, _VP, _VP, _I, _VP, _VP, _SZ, _VP, _VP]),
     "qmoe_ffn_prefill_timed": (_I, [ctypes.POINTER(qmoe_experts), _VP, _I, _VP, _VP, _I, _VP, _VP, _SZ, _VP, _VP,
-                                    ctypes.POINTER(_VP)]),
+                                    ctypes.POINTER(_VP), _I]),
     "qmoe_stack_workspace_bytes": (_SZ, [ctypes.POINTER(qmoe_stack_desc)]),
     "qmoe_stack_create": (_I, [ctypes.POINTER(qmoe_stack_desc), _VP, _SZ, _VP, ctypes.POINTER(_VP)]),
     "qmoe_stack_destroy": (_I, [_VP]),
     "qmoe_stack_buffers": (_I, [_VP, ctypes.POINTER(_VP), ctypes.POINTER(_VP), ctypes.POINTER(_VP),
                                 ctypes.POINTER(_VP), ctypes.POINTER(_VP)]),
+    "qmoe_stack_barrier_word": (_VP, [_VP]),
+    "qmoe_stack_trace": (_I, [_VP, _VP, _SZ, _VP, _VP]),
     "qmoe_stack_kernels_per_replay": (_I, [_VP]),
     "qmoe_stack_path": (_I, [_VP]),
     "qmoe_stack_decode": (_I, [_VP, _VP]),
@@ -189,8 +191,11 @@ def qmoe_ffn_prefill(experts: qmoe_experts, x, T, idx, gate, k, y, workspace, de
         workspace.numel() * workspace.element_size(), _p(dev_status), _s(stream)))
 
 
+PREFILL_ATOMIC_COMBINE = 1
+
+
 def qmoe_ffn_prefill_timed(experts: qmoe_experts, x, T, idx, gate, k, y, workspace, dev_status, events,
-                           stream=None) -> None:
+                           stream=None, flags=0) -> None:
     """``events``: three torch.cuda.Event(enable_timing=True) objects."""
     for e in events:
         if not e.cuda_event:   # torch creates the CUDA event at its first record
@@ -198,7 +203,7 @@ def qmoe_ffn_prefill_timed(experts: qmoe_experts, x, T, idx, gate, k, y, workspa
     arr = (_VP * 3)(*[e.cuda_event for e in events])
     _check("qmoe_ffn_prefill_timed", lib().qmoe_ffn_prefill_timed(
         ctypes.byref(experts), _p(x), T, _p(idx), _p(gate), k, _p(y), _p(workspace),
-        workspace.numel() * workspace.element_size(), _p(dev_status), _s(stream), arr))
+        workspace.numel() * workspace.element_size(), _p(dev_status), _s(stream), arr, flags))
 
 
 def qmoe_stack_workspace_bytes(desc: qmoe_stack_desc) -> int:
@@ -225,6 +230,20 @@ def qmoe_stack_buffers(stack: int) -> dict:
 
 def qmoe_stack_kernels_per_replay(stack: int) -> int:
     return lib().qmoe_stack_kernels_per_replay(stack)
+
+
+def qmoe_stack_trace(stack: int, L: int, max_ctas: int = 1024, points: int = 8):
+    """Phase stamps (SM cycles) of the last replay: numpy int64 [L, ctas, points]."""
+    import numpy as np
+    buf = np.zeros(L * max_ctas * points, dtype=np.int64)
+    g, p = ctypes.c_int(0), ctypes.c_int(0)
+    _check("qmoe_stack_trace", lib().qmoe_stack_trace(stack, buf.ctypes.data, buf.size, ctypes.byref(g),
+                                                      ctypes.byref(p)))
+    return buf[:L * g.value * p.value].reshape(L, g.value, p.value)
+
+
+def qmoe_stack_barrier_word(stack: int) -> int | None:
+    return lib().qmoe_stack_barrier_word(stack)
 
 
 def qmoe_stack_path(stack: int) -> int:

@@ -39,6 +39,7 @@ extern "C" const char *qmoe_status_string(qmoe_status s) {
     case QMOE_ERR_CUDA: return "CUDA runtime error";
     case QMOE_ERR_TIMEOUT: return "device wait exceeded its budget";
     case QMOE_ERR_DEVICE_STATUS: return "invalid routed expert index seen on the device";
+    case QMOE_ERR_RANGE: return "activation too large for the exact decode sums";
   }
   return "unknown status";
 }
@@ -50,6 +51,7 @@ extern "C" qmoe_status qmoe_read_status(const int32_t *dev_status) {
   switch (v) {
     case qmoe::DEV_OK: return QMOE_OK;
     case qmoe::DEV_TIMEOUT: return QMOE_ERR_TIMEOUT;
+    case qmoe::DEV_RANGE: return QMOE_ERR_RANGE;
     default: return QMOE_ERR_DEVICE_STATUS;
   }
 }

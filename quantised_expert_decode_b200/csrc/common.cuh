@@ -21,6 +21,7 @@ constexpr int32_t DEV_OK = 0;
 constexpr int32_t DEV_BAD_INDEX = 1;
 constexpr int32_t DEV_DUP_INDEX = 2;
 constexpr int32_t DEV_TIMEOUT = 3;
+constexpr int32_t DEV_RANGE = 4;   // a decode partial sum too large for the exact fixed-point sums
 
 // Time budget of every device-side wait, in SM clock cycles (~1 s at 2 GHz).
 constexpr long long WAIT_BUDGET_CYCLES = 2000000000LL;
@@ -126,13 +127,18 @@ __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
 // Grid-wide barrier for a co-resident grid (cooperative launch). Called by one
 // thread per CTA after its CTA-local barrier. The counter's top bit flips once
 // per barrier: CTA 0 adds 0x80000000 - (G-1), every other CTA adds 1, so the
-// total added per barrier is exactly 0x80000000 and the low bits return to 0.
-// Returns false when the wait ran out of its budget.
+// total added per barrier is exactly 0x80000000, the low bits return to 0 and
+// the flip comes with the last arrival, whatever the order. A fence publishes
+// this CTA's writes (ordered before it by the CTA barrier); the arrival is an
+// acquire-release add, so the last arrival, whose own add flips the bit,
+// acquires everyone else's writes without another round trip to L2; the
+// others poll with acquire loads. Returns false when the wait ran out of its budget.
 __device__ __forceinline__ bool grid_barrier_one_thread(unsigned *bar, unsigned nblocks) {
-  unsigned inc = (blockIdx.x == 0) ? (0x80000000u - (nblocks - 1u)) : 1u;
-  __threadfence();
-  unsigned old = atomicAdd(bar, inc);
-  long long deadline = clock64() + WAIT_BUDGET_CYCLES;
+  const unsigned inc = (blockIdx.x == 0) ? (0x80000000u - (nblocks - 1u)) : 1u;
+  __threadfence();   // cumulative: covers the writes of the CTA ordered before by its barrier
+  const unsigned old = atom_add_acq_rel_gpu(bar, inc);
+  if (((old + inc) ^ old) & 0x80000000u) return true;
+  const long long deadline = clock64() + WAIT_BUDGET_CYCLES;
   while (((ld_acquire_gpu(bar) ^ old) & 0x80000000u) == 0u) {
     if (clock64() > deadline) return false;
   }

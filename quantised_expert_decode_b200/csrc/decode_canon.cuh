@@ -1,0 +1,137 @@
+// Floating-point steps of decoding, written once for every decode path.
+//
+// The per-layer kernels (router with its residual RMSNorm, expert FFN, final
+// norm) and the fused layer-stack kernel split the same work differently
+// across threads and CTAs. A token's routes, gates and activations still come
+// out bit for bit the same on both paths, and whatever verify batch the token
+// sits in, because every rounding step below is fixed here and every sum whose
+// parts are formed in different places is an exact integer sum:
+//
+//   slices     the hidden axis is cut into 16-element slices c (h = 16c + i);
+//   partials   a slice's router partial sum_i Wr[e][16c+i] z[16c+i] and its
+//              sum of squares sum_i z[16c+i]^2 are float64 fma chains in
+//              element order i = 0..15;
+//   logits     each router partial is split into two integers (hi at 2^-20,
+//              lo at 2^-60); integers add exactly in any order, so a row summed
+//              by one warp and a row summed over 128 CTAs with atomics agree;
+//   squares    the slice sums of squares are added in one fixed order: lane l
+//              of a warp adds slices l, l + 32, l + 64, ... in turn, then the
+//              32 lane sums meet in a butterfly (xor 16, 8, 4, 2, 1); the fused
+//              kernel stores the slice sums and every CTA adds them this way;
+//   norm       rinv = 1 / sqrt(SS / H + eps) in float64; the activations the
+//              experts see are x = z * (float)rinv; router logits are
+//              (sum of partials of z) * rinv + bias, using Wr (z / rms) =
+//              (Wr z) / rms, so the logits need no second pass after the norm;
+//   combine    y = sum_j gate_j * r_j in slot order, one rounding per multiply
+//              and per add; z_next = x + y.
+//
+// A router partial of magnitude 2^33 or more (or NaN) cannot be split exactly;
+// it is reported through the device status (DEV_RANGE) instead.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace qmoe {
+namespace canon {
+namespace {
+
+constexpr int SLICE = 16;
+constexpr double FIX_HI = 1048576.0;                        // 2^20
+constexpr double FIX_HI_INV = 1.0 / 1048576.0;              // 2^-20
+constexpr double FIX_LO = 1152921504606846976.0;            // 2^60
+constexpr double FIX_LO_INV = 1.0 / 1152921504606846976.0;  // 2^-60
+constexpr double FIX_RANGE = 8589934592.0;                  // 2^33
+
+// p -> (hi, lo) with p = hi 2^-20 + lo 2^-60 up to the rounding of lo.
+// hi 2^-20 is the multiple of 2^-20 nearest p; the remainder r is a multiple
+// of min(ulp(p), 2^-20) below 2^-21 in magnitude, so p - hi 2^-20 is exact.
+// Returns false (and zeros) when |p| >= 2^33 or p is NaN.
+__device__ __forceinline__ bool split(double p, long long &hi, long long &lo) {
+  if (!(fabs(p) < FIX_RANGE)) {
+    hi = 0;
+    lo = 0;
+    return false;
+  }
+  hi = __double2ll_rn(__dmul_rn(p, FIX_HI));
+  const double r = __dsub_rn(p, __dmul_rn((double)hi, FIX_HI_INV));
+  lo = __double2ll_rn(__dmul_rn(r, FIX_LO));
+  return true;
+}
+
+// Exact integer totals -> float64 (two exact scalings, one rounding in the add;
+// (double)HI is exact below 2^53).
+__device__ __forceinline__ double join(long long hi, long long lo) {
+  return __dadd_rn(__dmul_rn((double)hi, FIX_HI_INV), __dmul_rn((double)lo, FIX_LO_INV));
+}
+
+// Router partial of one slice: w(i), z(i) for i = 0..15.
+template <class W, class Z>
+__device__ __forceinline__ double slice_dot(W w, Z z) {
+  double p = 0.0;
+#pragma unroll
+  for (int i = 0; i < SLICE; ++i) p = fma((double)w(i), (double)z(i), p);
+  return p;
+}
+
+// Sum of squares of one slice.
+template <class Z>
+__device__ __forceinline__ double slice_sumsq(Z z) {
+  double p = 0.0;
+#pragma unroll
+  for (int i = 0; i < SLICE; ++i) {
+    const double v = (double)z(i);
+    p = fma(v, v, p);
+  }
+  return p;
+}
+
+// Sum of squares of a token from its slice sums q(c), c < nsl, in the fixed
+// order above; every lane of the calling warp returns the same value.
+// Up to PRE slice sums per lane are fetched before any is added, so slice sums
+// read from global memory cost one round trip, not one per slice.
+template <int PRE = 4, class Q>
+__device__ __forceinline__ double warp_sumsq(Q q, int nsl) {
+  const int lane = threadIdx.x & 31;
+  double v[PRE];
+#pragma unroll
+  for (int m = 0; m < PRE; ++m) v[m] = lane + 32 * m < nsl ? q(lane + 32 * m) : 0.0;
+  double s = 0.0;
+#pragma unroll
+  for (int m = 0; m < PRE; ++m)
+    if (lane + 32 * m < nsl) s = __dadd_rn(s, v[m]);
+  for (int c = lane + 32 * PRE; c < nsl; c += 32) s = __dadd_rn(s, q(c));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, o));
+  return s;
+}
+
+// 1 / rms from the sum of squares of H elements.
+__device__ __forceinline__ double norm_rinv(double ss, int H, float eps) {
+  return __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)H), (double)eps)));
+}
+
+__device__ __forceinline__ double logit(double partial_sum, double rinv, double bias) {
+  return __dadd_rn(__dmul_rn(partial_sum, rinv), bias);
+}
+
+// One slot of the combine: y + g * r.
+__device__ __forceinline__ float combine_step(float y, float g, float r) { return __fadd_rn(y, __fmul_rn(g, r)); }
+
+__device__ __forceinline__ float silu(float a) { return __fdiv_rn(a, __fadd_rn(1.0f, expf(-a))); }
+
+__device__ __forceinline__ float hval(float a_g, float a_u) { return __fmul_rn(silu(a_g), a_u); }
+
+// Warp-wide exact sum of (hi, lo) pairs.
+__device__ __forceinline__ void warp_sum_fix(long long &hi, long long &lo) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    hi += __shfl_xor_sync(0xffffffffu, hi, o);
+    lo += __shfl_xor_sync(0xffffffffu, lo, o);
+  }
+}
+
+}  // namespace
+}  // namespace canon
+}  // namespace qmoe

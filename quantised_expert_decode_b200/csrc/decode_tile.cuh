@@ -31,6 +31,13 @@ __device__ __forceinline__ float i2f_small(int v) {
   return __int_as_float(0x4B400000 + v) - 12582912.0f;
 }
 
+// hi * 256 + lo as a float, exactly, for |hi|, |lo| < 2^16 (the block sums of
+// one limb pair: at most 32 * 15 * 128 in magnitude): both convert exactly,
+// hi * 256 is exact and the sum stays below 2^24. Four full-rate operations
+// and one fused multiply-add, no conversion-unit instruction (those issue at a
+// fraction of the rate and were the busiest pipe of the tile loop).
+__device__ __forceinline__ float limb_pair(int hi, int lo) { return fmaf(i2f_small(hi), 256.0f, i2f_small(lo)); }
+
 __device__ __forceinline__ float h2f(uint32_t bits16) { return __half2float(__ushort_as_half((unsigned short)bits16)); }
 
 // Quantise a 128-element chunk (4 blocks of 32) held one float4 per lane: lane
@@ -39,8 +46,21 @@ __device__ __forceinline__ float h2f(uint32_t bits16) { return __half2float(__us
 // same quantised values as its code term, so the whole block sees one
 // consistent activation s*X and the only error is that of quantising v.
 __device__ __forceinline__ int quant_one(float v, float inv) {
-  const int X = __float2int_rn(v * inv);
+  const int X = __float2int_rn(__fmul_rn(v, inv));
   return max(-8355711, min(8355711, X));
+}
+
+// Scale of a 32-element block from its largest magnitude a: s = a / QMAX taken
+// as a * (1 / QMAX), and the reciprocal used to quantise. Every decode path
+// quantises with these two values, so a block's limbs and (s, s * sum X) are
+// the same bits wherever it is quantised.
+__device__ __forceinline__ void block_scale(float a, float &s, float &inv) {
+  s = 0.0f;
+  inv = 0.0f;
+  if (a > 0.0f) {
+    s = __fmul_rn(a, 1.0f / QMAX);
+    inv = __frcp_rn(s);
+  }
 }
 
 // balanced base-256 digits of |X| <= 8355711, each in [-128, 127]
@@ -61,11 +81,8 @@ __device__ __noinline__ void quant_chunk(float4 v, uint8_t *limbs_vec, float2 *l
   a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
   a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
   a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
-  float s = 0.0f, inv = 0.0f;
-  if (a > 0.0f) {
-    s = a / QMAX;
-    inv = QMAX / a;
-  }
+  float s, inv;
+  block_scale(a, s, inv);
   const int X0 = quant_one(v.x, inv), X1 = quant_one(v.y, inv), X2 = quant_one(v.z, inv), X3 = quant_one(v.w, inv);
   int a2, a1, a0, b2, b1, b0, c2, c1, c0, d2, d1, d0;
   limbs3(X0, a2, a1, a0);
@@ -81,7 +98,7 @@ __device__ __noinline__ void quant_chunk(float4 v, uint8_t *limbs_vec, float2 *l
   sx += __shfl_xor_sync(0xffffffffu, sx, 1);
   sx += __shfl_xor_sync(0xffffffffu, sx, 2);
   sx += __shfl_xor_sync(0xffffffffu, sx, 4);
-  if ((lane & 7) == 0) lsc_vec[blk] = make_float2(s, s * (float)sx);
+  if ((lane & 7) == 0) lsc_vec[blk] = make_float2(s, __fmul_rn(s, (float)sx));
 }
 
 struct Acc {
@@ -176,8 +193,8 @@ __device__ __noinline__ Acc tile_dot(const uint8_t *tile, int nblk, const uint8_
         }
         if (ov[q] >= 0) {
           const int bo = c * 4 + sb * BS + obeta;
-          const float v0 = (float)(d0 * 256 + d1);
-          const float v1 = (float)(d2 * 256 + d3);
+          const float v0 = limb_pair(d0, d1);
+          const float v1 = limb_pair(d2, d3);
           const float2 ss = lsc[(size_t)ov[q] * nblk + bo];
           const uint2 dm = *reinterpret_cast<const uint2 *>(sbase + (bo * 8 + g) * 8);
           const float sw = ss.x * wgt;
@@ -317,10 +334,8 @@ __device__ __noinline__ float2 tile_dot1(const uint8_t *tile, int nblk, const ui
 #pragma unroll
         for (int sb = 0; sb < 2; ++sb) {
           const int bo = (c0 + ch) * 4 + sb * 2 + oP;
-          // |v| <= 32*3*128*257 < 2^22 for 2-bit codes; 4-bit codes need the conversion
-          const int i0 = D[ch][sb][0] * 256 + D[ch][sb][1], i1 = D[ch][sb][2] * 256 + D[ch][sb][3];
-          const float v0 = BITS == 2 ? i2f_small(i0) : (float)i0;
-          const float v1 = BITS == 2 ? i2f_small(i1) : (float)i1;
+          const float v0 = limb_pair(D[ch][sb][0], D[ch][sb][1]);
+          const float v1 = limb_pair(D[ch][sb][2], D[ch][sb][3]);
           const float2 ss = lsc[bo];
           const uint2 dm = *reinterpret_cast<const uint2 *>(sbase + (bo * 8 + g) * 8);
           const float sw = ss.x * wgt;
@@ -338,20 +353,16 @@ __device__ __noinline__ float2 tile_dot1(const uint8_t *tile, int nblk, const ui
   return make_float2(acc0, acc1);
 }
 
-// Inline form of quant_chunk with a reciprocal in place of the divisions, for
-// loops whose iterations the compiler may interleave. s and inv need not be
-// exact inverses: the contraction uses s itself, so s * X still tracks v to
-// within rounding of the quantisation.
+// Inline form of quant_chunk, for loops whose iterations the compiler may
+// interleave. s and inv need not be exact inverses: the contraction uses s
+// itself, so s * X still tracks v to within rounding of the quantisation.
 __device__ __forceinline__ void quant_chunk_inl(float4 v, uint8_t *limbs_vec, float2 *lsc_vec, int chunk, int lane) {
   float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
   a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
   a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
   a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
-  float s = 0.0f, inv = 0.0f;
-  if (a > 0.0f) {
-    s = a * (1.0f / QMAX);
-    inv = __frcp_rn(s);
-  }
+  float s, inv;
+  block_scale(a, s, inv);
   const int X0 = quant_one(v.x, inv), X1 = quant_one(v.y, inv), X2 = quant_one(v.z, inv), X3 = quant_one(v.w, inv);
   int a2, a1, a0, b2, b1, b0, c2, c1, c0, d2, d1, d0;
   limbs3(X0, a2, a1, a0);
@@ -367,7 +378,7 @@ __device__ __forceinline__ void quant_chunk_inl(float4 v, uint8_t *limbs_vec, fl
   sx += __shfl_xor_sync(0xffffffffu, sx, 1);
   sx += __shfl_xor_sync(0xffffffffu, sx, 2);
   sx += __shfl_xor_sync(0xffffffffu, sx, 4);
-  if ((lane & 7) == 0) lsc_vec[blk] = make_float2(s, s * (float)sx);
+  if ((lane & 7) == 0) lsc_vec[blk] = make_float2(s, __fmul_rn(s, (float)sx));
 }
 
 // Quantise activation vectors of 128-element chunks; task = vec * nch + chunk.
@@ -394,7 +405,6 @@ __device__ __forceinline__ void quant_tasks(int ntask, int nch, int nblk, uint8_
   }
 }
 
-__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + expf(-a)); }
 
 
 }  // namespace

@@ -17,6 +17,7 @@
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "decode_canon.cuh"
 #include "decode_tile.cuh"
 #include "layout.cuh"
 
@@ -33,7 +34,6 @@ constexpr int CONSUMER_BAR = 1;            // named barrier id for the consumer 
 struct Plan {
   int err;
   int abort;
-  int turn;  // next ring item whose arrival a consumer warp may wait for
   int U;
   int ue[FD_MAXP];
   int nt[FD_MAXP];
@@ -45,7 +45,27 @@ struct Plan {
   float sgate[FD_MAXP];
   unsigned bm[32];
   int vids[NCW][FD_MAXT];  // per consumer warp: limb-region vectors of the current item
+  int lo1, hi1, lo2, hi2;  // this CTA's gate/up and down item ranges
 };
+
+// Relative cost of a tile whose expert serves n tokens: the bytes (the same
+// for every tile) plus the tensor-core and epilogue work of the tile-dot
+// variant for n vectors (1, 2, 4 or 8), which grows about linearly above two.
+__device__ __forceinline__ int tile_cost(int n) { return n <= 1 ? 4 : n <= 2 ? 5 : n <= 4 ? 8 : 14; }
+
+// First item whose starting cost is at least `target`, items numbered expert
+// by expert (per_expert items each, all at the expert's tile cost).
+__device__ int item_at_cost(const Plan *pl, int U, int per_expert, long long target) {
+  long long acc = 0;
+  for (int u = 0; u < U; ++u) {
+    const int w = tile_cost(pl->nt[u]);
+    if (target <= acc) return u * per_expert;
+    const long long i = (target - acc + w - 1) / w;
+    if (i < per_expert) return u * per_expert + (int)i;
+    acc += (long long)per_expert * w;
+  }
+  return U * per_expert;
+}
 
 struct FfnArgs {
   const uint8_t *gu;
@@ -60,6 +80,7 @@ struct FfnArgs {
   int32_t *status;
   int T, k, E, H, I;
   int slot_bytes, nslots;
+  int ncons;       // consumer warps that take ring items; nslots is a multiple of it
   int limb_bytes;  // activation-limb region
   int lsc_count;   // float2 entries of the limb-scale table
 };
@@ -165,7 +186,6 @@ __device__ void build_plan(const FfnArgs &a, Plan *pl) {
     pl->U = U;
     pl->err = 0;
     pl->abort = 0;
-    pl->turn = 0;
   }
   __syncwarp();
 #pragma unroll
@@ -209,14 +229,24 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
   }
   // Everything above overlaps the previous kernel; idx, gate and x are its outputs.
   pdl_wait();
-  if (warp == 0) build_plan(a, pl);
+  if (warp == 0) {
+    build_plan(a, pl);
+    // split both phases' items over the CTAs by cost, not by count: a tile
+    // shared by 8 tokens costs several times a single-token tile
+    if (lane == 0 && !pl->err) {
+      long long W = 0;
+      for (int u = 0; u < pl->U; ++u) W += tile_cost(pl->nt[u]);
+      const long long W1 = W * 2 * I16, W2 = W * H16;
+      pl->lo1 = item_at_cost(pl, pl->U, 2 * I16, W1 * blockIdx.x / G);
+      pl->hi1 = item_at_cost(pl, pl->U, 2 * I16, W1 * (blockIdx.x + 1) / G);
+      pl->lo2 = item_at_cost(pl, pl->U, H16, W2 * blockIdx.x / G);
+      pl->hi2 = item_at_cost(pl, pl->U, H16, W2 * (blockIdx.x + 1) / G);
+    }
+  }
   __syncthreads();
   if (pl->err) return;
 
-  const int U = pl->U;
-  const int N1 = 2 * U * I16, N2 = U * H16;
-  const int lo1 = (int)((long long)blockIdx.x * N1 / G), hi1 = (int)((long long)(blockIdx.x + 1) * N1 / G);
-  const int lo2 = (int)((long long)blockIdx.x * N2 / G), hi2 = (int)((long long)(blockIdx.x + 1) * N2 / G);
+  const int lo1 = pl->lo1, hi1 = pl->hi1, lo2 = pl->lo2, hi2 = pl->hi2;
   const int n1 = hi1 - lo1, ntot = n1 + (hi2 - lo2);
 
   if (warp == NCW) {
@@ -281,29 +311,22 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
   }
   named_barrier_sync(CONSUMER_BAR, nth);
 
-  // Waits for ring item n. Consumer warps take these waits in item order (the
-  // turn counter): when item n is awaited every earlier item has arrived, so
-  // its slot's barrier is at most one phase behind and the parity is exact.
+  // Waits for ring item n. Item n goes to slot n % S and to consumer warp
+  // n % NA, and S is a multiple of NA, so every slot has one consumer warp,
+  // which takes the slot's phases in order: when it waits for item n it has
+  // already consumed item n - S of the same slot, so the slot's barrier is in
+  // the phase of item n and the parity wait is exact.
+  const int NA = a.ncons;
   auto wait_full = [&](int n) -> bool {
     const long long dl = clock64() + WAIT_BUDGET_CYCLES;
-    bool ok = true;
-    while (*(volatile int *)&pl->turn != n) {
+    const uint32_t par = (uint32_t)((n / S) & 1);
+    while (!mbar_try_wait(&full[n % S], par)) {
       if (*(volatile int *)&pl->abort) return false;
       if (clock64() > dl) {
-        ok = false;
-        break;
+        set_status(a.status, DEV_TIMEOUT);
+        *(volatile int *)&pl->abort = 1;
+        return false;
       }
-    }
-    if (ok) ok = mbar_wait(&full[n % S], (uint32_t)((n / S) & 1), dl);
-    if (!ok) {
-      set_status(a.status, DEV_TIMEOUT);
-      *(volatile int *)&pl->abort = 1;
-      return false;
-    }
-    __syncwarp();
-    if (lane == 0) {
-      __threadfence_block();
-      *(volatile int *)&pl->turn = n + 1;
     }
     return true;
   };
@@ -314,7 +337,7 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
   const int g = lane >> 2, t = lane & 3;
 
   // phase 1: gate / up
-  for (int n = warp; n < n1; n += NCW) {
+  for (int n = warp; warp < NA && n < n1; n += NA) {
     if (!wait_full(n)) break;
     const int i = lo1 + n;
     const int u = i / (2 * I16), m = (i / I16) & 1, r = i % I16;
@@ -372,14 +395,15 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
         const float *ab = abuf + (size_t)(pb0 + lv) * 2 * I + c * 128;
         float4 gv = __ldcg(reinterpret_cast<const float4 *>(ab) + lane);
         float4 uv = __ldcg(reinterpret_cast<const float4 *>(ab + I) + lane);
-        return make_float4(silu_f(gv.x) * uv.x, silu_f(gv.y) * uv.y, silu_f(gv.z) * uv.z, silu_f(gv.w) * uv.w);
+        return make_float4(canon::hval(gv.x, uv.x), canon::hval(gv.y, uv.y), canon::hval(gv.z, uv.z),
+                           canon::hval(gv.w, uv.w));
       });
     }
     named_barrier_sync(CONSUMER_BAR, nth);
     const int item_end = min(hi2, u1 * H16);
     for (int it2 = item; it2 < item_end; ++it2) {
       const int n = n1 + (it2 - lo2);
-      if (n % NCW != warp) continue;
+      if (n % NA != warp) continue;
       if (!wait_full(n)) break;
       const int u = it2 / H16, r = it2 % H16;
       const int nu = pl->nt[u], pb = pl->pbase[u];
@@ -396,8 +420,8 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
           const int p = pb + tau;
           const float gw = pl->pgate[p];
           float *dst = a.part + ((size_t)pl->ptok[p] * k + pl->pslot[p]) * H + r * 16;
-          dst[g] = gw * acc.r0[q];
-          dst[g + 8] = gw * acc.r1[q];
+          dst[g] = __fmul_rn(gw, acc.r0[q]);
+          dst[g + 8] = __fmul_rn(gw, acc.r1[q]);
         }
       }
       release(n);
@@ -429,11 +453,14 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
 #pragma unroll
     for (int j = 0; j < FD_MAXK; ++j)
       if (j < k) v[j] = __ldcg(p4 + ((size_t)tt * k + j) * H4 + h);
+    // slot order, one rounding per add: the combine of decode_canon.cuh
+    // (gate * result was rounded once in phase 2)
     float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int j = 0; j < FD_MAXK; ++j)
       if (j < k) {
-        sum.x += v[j].x; sum.y += v[j].y; sum.z += v[j].z; sum.w += v[j].w;
+        sum.x = __fadd_rn(sum.x, v[j].x); sum.y = __fadd_rn(sum.y, v[j].y);
+        sum.z = __fadd_rn(sum.z, v[j].z); sum.w = __fadd_rn(sum.w, v[j].w);
       }
     y4[o] = sum;
   }
@@ -496,11 +523,22 @@ qmoe_status qmoe::ffn_decode_launch(const qmoe_experts *ex, const float *x, int 
   a.limb_bytes = ((limb_x > limb_h ? limb_x : limb_h) + 127) & ~127;
   int lsc_x = T * (H / 32), lsc_h = (a.limb_bytes / (I * 3)) * (I / 32);
   a.lsc_count = lsc_x > lsc_h ? lsc_x : lsc_h;
-  size_t cap = max_smem_optin();
-  int S = 16;
-  while (S >= 2 && smem_layout(S, a.slot_bytes, a.limb_bytes, a.lsc_count).total > cap) --S;
+  // Ring depth S and consumer warps NA (S a multiple of NA): as many consumer
+  // warps as possible, then the deepest ring that fits.
+  const size_t cap = max_smem_optin();
+  int S = 0, NA = 0;
+  for (int s2 = 16; s2 >= 2; --s2) {
+    if (smem_layout(s2, a.slot_bytes, a.limb_bytes, a.lsc_count).total > cap) continue;
+    int na = NCW;
+    while (s2 % na) --na;
+    if (na > NA) {
+      NA = na;
+      S = s2;
+    }
+  }
   if (S < 2) return QMOE_ERR_UNSUPPORTED;
   a.nslots = S;
+  a.ncons = NA;
   size_t smem = smem_layout(S, a.slot_bytes, a.limb_bytes, a.lsc_count).total;
 
   const void *fn = (bits == 2) ? (const void *)ffn_decode_kernel<2> : (const void *)ffn_decode_kernel<4>;

@@ -7,7 +7,12 @@
 //       G = Wg[f,:] X_e^T,  U = Wu[f,:] X_e^T      (fp32 in tensor memory)
 //       h[pair, f] = bf16(silu(G) * U)
 //   GEMM 2, per expert e and 256 hidden features o:
-//       Y = Wd[o,:] h_e^T;  y[token, o] += gate[pair] * Y   (fp32 reductions)
+//       Y = Wd[o,:] h_e^T;  part[pair, o] = gate[pair] * Y  (fp32, bucket order)
+//   combine, per token t: y[t, :] = sum over slots j (in slot order) of
+//       part[pair (t, j), :]     - every run adds the same terms in the same
+//       order, so y is reproducible bit for bit. (The earlier form, fp32
+//       atomic additions straight into y, is kept behind a flag of the timed
+//       entry point for comparison; its order, and y's last bits, vary.)
 // X_e is the bf16 activation rows of the tokens routed to e, gathered by
 // token id; h is kept in bucket order with every expert's rows padded to a
 // multiple of 16. The weights form the 128-row MMA operand and the tokens the
@@ -100,9 +105,9 @@ struct PfGemm {
   const float *pgate;
   __nv_bfloat16 *hout;       // GEMM 1 output, [rows, I]
   int ldh;
-  float *y;                  // GEMM 2 output, [T, H]
+  float *y;                  // GEMM 2 output, [T, H] (mode 1) or [pairs, H] in bucket order (mode 2)
   int ldy;
-  int mode;                  // 0: silu(G) * U -> h; 1: gate-scaled reduction into y
+  int mode;                  // 0: silu(G) * U -> h; 1: gate-scaled reduction into y; 2: gate-scaled pair rows
   int32_t *status;
 };
 
@@ -446,6 +451,24 @@ __device__ void pf_epilogue(const PfGemm &a, PfBars *b, int nt, uint32_t tmem) {
             *reinterpret_cast<__nv_bfloat162 *>(h + (size_t)n * a.ldh) = __floats2bfloat162_rn(hv, hn);
         }
       }
+    } else if (a.mode == 2) {
+      const int pos0 = a.off[t.x] + t.z;
+      float *pb = a.y + (size_t)pos0 * a.ldy + t.y * (2 * PF_M) + r;
+      for (int c0 = 16 * par; c0 < N; c0 += 32) {
+        float v0[16], v1[16];
+        tc05::ld16x2(ts + c0, tu + c0, v0, v1);
+        float gt = 0.0f;
+        if (lane < 16 && c0 + lane < t.w) gt = a.pgate[pos0 + c0 + lane];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float gi = __shfl_sync(0xffffffffu, gt, i);
+          if (c0 + i < t.w) {
+            float *pr = pb + (size_t)(c0 + i) * a.ldy;
+            pr[0] = __fmul_rn(gi, v0[i]);
+            pr[PF_M] = __fmul_rn(gi, v1[i]);
+          }
+        }
+      }
     } else {
       const int pos0 = a.off[t.x] + t.z;
       float *yb = a.y + t.y * (2 * PF_M) + r;
@@ -583,6 +606,30 @@ struct PlanArgs {
 // (expert, chunk, feature block) order, then each expert's remainder chunk,
 // largest remainder first (ties by expert index), all feature blocks of one
 // remainder adjacent. CTAs take tiles round-robin.
+// Position of every pair (t, j) in bucket order: inv[perm[i]] = i.
+__global__ void pf_inverse_kernel(const int32_t *perm, int P, int32_t *inv, const int32_t *status) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < P && *reinterpret_cast<volatile const int32_t *>(status) == 0) inv[perm[i]] = i;
+}
+
+// y[t, :] = sum_j part[inv[t k + j], :] in slot order, one rounding per add.
+// One thread per 4 features of a token; H4 = H / 4.
+__global__ void __launch_bounds__(256) pf_combine_kernel(const float4 *part, const int32_t *inv, int T, int k, int H4,
+                                                         float4 *y, const int32_t *status) {
+  const long long o = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (o >= (long long)T * H4 || *reinterpret_cast<volatile const int32_t *>(status) != 0) return;
+  const int t = (int)(o / H4), c = (int)(o % H4);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < k; ++j) {
+    const float4 v = __ldg(part + (size_t)inv[t * k + j] * H4 + c);
+    acc.x = __fadd_rn(acc.x, v.x);
+    acc.y = __fadd_rn(acc.y, v.y);
+    acc.z = __fadd_rn(acc.z, v.z);
+    acc.w = __fadd_rn(acc.w, v.w);
+  }
+  y[o] = acc;
+}
+
 __global__ void __launch_bounds__(1024, 1) pf_plan_kernel(PlanArgs a) {
   __shared__ int s_rem[PF_MAX_E];
   __shared__ int wt[3][32];
@@ -659,7 +706,7 @@ __global__ void __launch_bounds__(1024, 1) pf_plan_kernel(PlanArgs a) {
 
 // ------------------------------------------------------------ workspace --
 struct PfLayout {
-  size_t off, poff, perm, ptok, pgate, ntiles, bk, tiles1, tiles2, h, xp, total;
+  size_t off, poff, perm, ptok, pgate, ntiles, bk, tiles1, tiles2, h, xp, inv, part, total;
   size_t max_tiles1, max_tiles2, h_rows;
 };
 
@@ -684,6 +731,8 @@ PfLayout pf_layout(int T, int k, int E, int H, int I) {
   L.tiles2 = o; o += up256(L.max_tiles2 * sizeof(int4));
   L.h = o;      o += up256(L.h_rows * I * sizeof(__nv_bfloat16));
   L.xp = o;     o += up256(L.h_rows * H * sizeof(__nv_bfloat16));
+  L.inv = o;    o += up256(P * sizeof(int32_t));
+  L.part = o;   o += up256(P * H * sizeof(float));
   L.total = o;
   return L;
 }
@@ -761,7 +810,8 @@ extern "C" size_t qmoe_prefill_workspace_bytes(int T, int k, int E, int H, int I
 
 static qmoe_status ffn_prefill(const qmoe_experts *ex, const void *x, int T, const int32_t *idx, const float *gate,
                                int k, float *y, void *workspace, size_t workspace_bytes, int32_t *dev_status,
-                               qmoe_stream_t stream, void *const *events) {
+                               qmoe_stream_t stream, void *const *events, int flags) {
+  const bool atomic_combine = (flags & QMOE_PREFILL_ATOMIC_COMBINE) != 0;
   if (!ex || !x || !idx || !gate || !y || !workspace || !dev_status) return QMOE_ERR_INVALID_ARG;
   if (T < 1 || k < 1) return QMOE_ERR_INVALID_ARG;
   const int E = ex->E, H = ex->H, I = ex->I;
@@ -799,7 +849,16 @@ static qmoe_status ffn_prefill(const qmoe_experts *ex, const void *x, int T, con
   pf_plan_kernel<<<1, 1024, 0, s>>>(pa);
   note_launch();
   if (cudaGetLastError() != cudaSuccess) return QMOE_ERR_CUDA;
-  if (cudaMemsetAsync(y, 0, (size_t)T * H * sizeof(float), s) != cudaSuccess) return QMOE_ERR_CUDA;
+  int32_t *inv = reinterpret_cast<int32_t *>(ws + L.inv);
+  float *part = reinterpret_cast<float *>(ws + L.part);
+  const int P = T * k;
+  if (atomic_combine) {
+    if (cudaMemsetAsync(y, 0, (size_t)T * H * sizeof(float), s) != cudaSuccess) return QMOE_ERR_CUDA;
+  } else {
+    pf_inverse_kernel<<<(P + 255) / 256, 256, 0, s>>>(perm, P, inv, dev_status);
+    note_launch();
+    if (cudaGetLastError() != cudaSuccess) return QMOE_ERR_CUDA;
+  }
   pf_gather_kernel<<<(unsigned)((L.h_rows + 7) / 8), 256, 0, s>>>(static_cast<const uint4 *>(x), H / 8, off, poff, ptok,
                                                                    E, (int)L.h_rows, reinterpret_cast<uint4 *>(xp),
                                                                    dev_status);
@@ -838,25 +897,33 @@ static qmoe_status ffn_prefill(const qmoe_experts *ex, const void *x, int T, con
   g2.tiles = tiles2;
   g2.ntiles = ntiles + 1;
   g2.hout = nullptr;
-  g2.y = y;
+  g2.y = atomic_combine ? y : part;
   g2.ldy = H;
-  g2.mode = 1;
+  g2.mode = atomic_combine ? 1 : 2;
   st = pf_gemm_launch(g2, s);
   if (st != QMOE_OK) return st;
   if (events && cudaEventRecord(static_cast<cudaEvent_t>(events[2]), s) != cudaSuccess) return QMOE_ERR_CUDA;
+  if (!atomic_combine) {
+    const long long n = (long long)T * (H / 4);
+    pf_combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(reinterpret_cast<const float4 *>(part), inv, T, k,
+                                                                 H / 4, reinterpret_cast<float4 *>(y), dev_status);
+    note_launch();
+    if (cudaGetLastError() != cudaSuccess) return QMOE_ERR_CUDA;
+  }
   return QMOE_OK;
 }
 
 extern "C" qmoe_status qmoe_ffn_prefill(const qmoe_experts *ex, const void *x, int T, const int32_t *idx,
                                         const float *gate, int k, float *y, void *workspace, size_t workspace_bytes,
                                         int32_t *dev_status, qmoe_stream_t stream) {
-  return ffn_prefill(ex, x, T, idx, gate, k, y, workspace, workspace_bytes, dev_status, stream, nullptr);
+  return ffn_prefill(ex, x, T, idx, gate, k, y, workspace, workspace_bytes, dev_status, stream, nullptr, 0);
 }
 
 extern "C" qmoe_status qmoe_ffn_prefill_timed(const qmoe_experts *ex, const void *x, int T, const int32_t *idx,
                                               const float *gate, int k, float *y, void *workspace,
                                               size_t workspace_bytes, int32_t *dev_status, qmoe_stream_t stream,
-                                              void *const *events) {
+                                              void *const *events, int flags) {
   if (!events || !events[0] || !events[1] || !events[2]) return QMOE_ERR_INVALID_ARG;
-  return ffn_prefill(ex, x, T, idx, gate, k, y, workspace, workspace_bytes, dev_status, stream, events);
+  if (flags & ~QMOE_PREFILL_ATOMIC_COMBINE) return QMOE_ERR_INVALID_ARG;
+  return ffn_prefill(ex, x, T, idx, gate, k, y, workspace, workspace_bytes, dev_status, stream, events, flags);
 }

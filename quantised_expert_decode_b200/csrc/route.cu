@@ -1,17 +1,21 @@
-// Router for decode batches (T <= 8): float64 GEMV over fp32 weights, top-k with
-// ties to the lower expert index, renormalised gates; optionally preceded by
-// the residual RMSNorm of the previous layer's output.
+// Router for decode batches (T <= 8): float64 router logits from exact
+// fixed-point sums of 16-element slice partials, top-k with ties to the lower
+// expert index, renormalised gates; optionally preceded by the residual
+// RMSNorm of the previous layer's output. The arithmetic is the one of
+// decode_canon.cuh, shared with the fused layer-stack kernel.
 #include <mutex>
 
 #include "common.cuh"
+#include "decode_canon.cuh"
 #include "route_common.cuh"
 
 namespace qmoe {
 namespace {
 
-constexpr int RT_THREADS = 128;  // 4 warps, one router row per warp at a time
+constexpr int RT_WARPS = 8;                // one router row per warp; one token per warp for the top-k
+constexpr int RT_THREADS = 32 * RT_WARPS;
 constexpr int RT_MAXT = 8;
-constexpr int RT_PREFETCH = 16;  // float4 per lane held across the dependency wait
+constexpr int RT_PRE = 4;                  // slices per lane held in registers (all of H <= 2048)
 
 struct RouteArgs {
   const float *Wr;
@@ -28,136 +32,198 @@ struct RouteArgs {
   int32_t *status;
 };
 
-template <bool RESID>
-__global__ void __launch_bounds__(RT_THREADS) route_decode_kernel(RouteArgs a) {
-  extern __shared__ float4 xs4[];  // [T][H/4]
-  __shared__ float inv_rms[RT_MAXT];
-  __shared__ unsigned is_last;
-  __shared__ TopkScratch topk_sc[RT_THREADS / 32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int T = a.T, H = a.H, E = a.E, H4 = H / 4;
+// z = x (+ y) of every token sits in shared memory with one pad float after
+// every 32: element h of token t at t * HP + h + h / 32 (HP = H + H / 32). A
+// lane reads the 16 elements of one slice, lanes 16 elements apart; the pad
+// spreads the 32 lanes of a warp over the 32 banks.
+__host__ __device__ inline int route_hp(int H) { return H + H / 32; }
+__device__ __forceinline__ int zpos(int h) { return h + (h >> 5); }
+inline size_t route_smem_bytes(int T, int H) { return (size_t)T * route_hp(H) * 4; }
 
-  // This warp's router row does not depend on the previous kernel: fetch it
-  // into registers (H <= 2048 entirely) before waiting for that kernel.
-  const int e_row = blockIdx.x * (RT_THREADS / 32) + warp;
-  float4 wpre[RT_PREFETCH];
+template <bool RESID>
+__global__ void __launch_bounds__(RT_THREADS, 1) route_decode_kernel(RouteArgs a) {
+  extern __shared__ __align__(16) float zs[];  // [T][HP], padded
+  __shared__ double rinv_s[RT_MAXT];
+  __shared__ float inv_s[RT_MAXT];
+  __shared__ unsigned is_last;
+  __shared__ int range_bad;
+  __shared__ TopkScratch topk_sc[RT_WARPS];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int T = a.T, H = a.H, E = a.E, nsl = H / canon::SLICE, HP = route_hp(H);
+  const int e_row = blockIdx.x * RT_WARPS + warp;
+
+  // This warp's router row does not depend on the previous kernel: fetch the
+  // lane's slices (c = lane + 32 j) into registers before waiting for it.
+  float4 wpre[RT_PRE][4];
   if (e_row < E) {
     const float4 *w4 = reinterpret_cast<const float4 *>(a.Wr + (size_t)e_row * H);
 #pragma unroll
-    for (int j = 0; j < RT_PREFETCH; ++j)
-      if (lane + 32 * j < H4) wpre[j] = __ldg(w4 + lane + 32 * j);
+    for (int j = 0; j < RT_PRE; ++j) {
+      const int c = lane + 32 * j;
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        if (c < nsl) wpre[j][m] = __ldg(w4 + c * 4 + m);
+    }
   }
+  if (tid == 0) range_bad = 0;
   pdl_wait();
   pdl_launch_dependents();
 
-  const float4 *x4 = reinterpret_cast<const float4 *>(a.x);
-  const float4 *y4 = reinterpret_cast<const float4 *>(a.y);
-  for (int i = tid; i < T * H4; i += RT_THREADS) {
-    float4 v = x4[i];
-    if (RESID) {
-      float4 w = y4[i];
-      v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+  // z = x (+ y) into the padded layout; eight float4 of each input in flight
+  // per thread
+  {
+    const float4 *x4 = reinterpret_cast<const float4 *>(a.x);
+    const float4 *y4 = reinterpret_cast<const float4 *>(a.y);
+    const int n4 = T * H / 4, H4 = H / 4;
+    constexpr int B = 8;
+    for (int i0 = tid; i0 < n4; i0 += B * RT_THREADS) {
+      float4 xv[B], yv[B];
+#pragma unroll
+      for (int u = 0; u < B; ++u) {
+        const int i = i0 + u * RT_THREADS;
+        if (i < n4) {
+          xv[u] = __ldcg(x4 + i);
+          if (RESID) yv[u] = __ldcg(y4 + i);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < B; ++u) {
+        const int i = i0 + u * RT_THREADS;
+        if (i < n4) {
+          float4 v = xv[u];
+          if (RESID) {
+            v.x = __fadd_rn(v.x, yv[u].x); v.y = __fadd_rn(v.y, yv[u].y);
+            v.z = __fadd_rn(v.z, yv[u].z); v.w = __fadd_rn(v.w, yv[u].w);
+          }
+          const int t = i / H4, h = 4 * (i % H4);
+          float *zt = zs + (size_t)t * HP;
+          zt[zpos(h)] = v.x; zt[zpos(h + 1)] = v.y; zt[zpos(h + 2)] = v.z; zt[zpos(h + 3)] = v.w;
+        }
+      }
     }
-    xs4[i] = v;
   }
   __syncthreads();
   if (RESID) {
-    for (int t = warp; t < T; t += RT_THREADS / 32) {
-      double ss = 0.0;
-      for (int j = lane; j < H4; j += 32) {
-        float4 v = xs4[t * H4 + j];
-        ss += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
+    // sum of squares of every token (one warp per token), then 1 / rms
+    for (int t = warp; t < T; t += RT_WARPS) {
+      const float *zt = zs + (size_t)t * HP;
+      const double ss = canon::warp_sumsq(
+          [&](int c) { return canon::slice_sumsq([&](int i) { return zt[zpos(c * canon::SLICE + i)]; }); }, nsl);
+      if (lane == 0) {
+        const double r = canon::norm_rinv(ss, H, a.eps);
+        rinv_s[t] = r;
+        inv_s[t] = __double2float_rn(r);
       }
-      ss = warp_sum_d(ss);
-      if (lane == 0) inv_rms[t] = (float)(1.0 / sqrt(ss / (double)H + (double)a.eps));
     }
     __syncthreads();
-    float4 *xo4 = reinterpret_cast<float4 *>(a.x_out);
-    for (int i = tid; i < T * H4; i += RT_THREADS) {
-      float s = inv_rms[i / H4];
-      float4 v = xs4[i];
-      v.x *= s; v.y *= s; v.z *= s; v.w *= s;
-      xs4[i] = v;
-      if (blockIdx.x == 0) xo4[i] = v;
+    if (blockIdx.x == 0) {
+      float4 *xo4 = reinterpret_cast<float4 *>(a.x_out);
+      const int H4 = H / 4;
+      for (int i = tid; i < T * H4; i += RT_THREADS) {
+        const int t = i / H4, h = 4 * (i % H4);
+        const float s = inv_s[t];
+        const float *zt = zs + (size_t)t * HP;
+        xo4[i] = make_float4(__fmul_rn(zt[zpos(h)], s), __fmul_rn(zt[zpos(h + 1)], s), __fmul_rn(zt[zpos(h + 2)], s),
+                             __fmul_rn(zt[zpos(h + 3)], s));
+      }
     }
+  } else {
+    if (tid < RT_MAXT) rinv_s[tid] = 1.0;
     __syncthreads();
   }
 
-  // logits: one warp per router row, float64 accumulation of exact products
+  // logits: one warp per router row; slice partials split into exact integers
   if (e_row < E) {
     const float4 *w4 = reinterpret_cast<const float4 *>(a.Wr + (size_t)e_row * H);
     const double b = a.bias ? (double)a.bias[e_row] : 0.0;
+    bool ok = true;
 #pragma unroll 1
     for (int t = 0; t < T; ++t) {
-      double s = 0.0;
+      const float *zt = zs + (size_t)t * HP;
+      long long hi = 0, lo = 0;
 #pragma unroll
-      for (int jj = 0; jj < RT_PREFETCH; ++jj) {
-        const int j = lane + 32 * jj;
-        if (j < H4) {
-          const float4 w = wpre[jj], v = xs4[t * H4 + j];
-          s = fma((double)w.x, (double)v.x, s);
-          s = fma((double)w.y, (double)v.y, s);
-          s = fma((double)w.z, (double)v.z, s);
-          s = fma((double)w.w, (double)v.w, s);
+      for (int j = 0; j < RT_PRE; ++j) {
+        const int c = lane + 32 * j;
+        if (c < nsl) {
+          const float *zc = zt + zpos(c * canon::SLICE);   // a slice never crosses a pad
+          const double p = canon::slice_dot(
+              [&](int i) {
+                const float4 v = wpre[j][i >> 2];
+                return (i & 3) == 0 ? v.x : (i & 3) == 1 ? v.y : (i & 3) == 2 ? v.z : v.w;
+              },
+              [&](int i) { return zc[i]; });
+          long long h1, l1;
+          ok &= canon::split(p, h1, l1);
+          hi += h1;
+          lo += l1;
         }
       }
-      for (int j = lane + 32 * RT_PREFETCH; j < H4; j += 32) {
-        const float4 w = __ldg(w4 + j), v = xs4[t * H4 + j];
-        s = fma((double)w.x, (double)v.x, s);
-        s = fma((double)w.y, (double)v.y, s);
-        s = fma((double)w.z, (double)v.z, s);
-        s = fma((double)w.w, (double)v.w, s);
+      for (int c = lane + 32 * RT_PRE; c < nsl; c += 32) {   // larger H only
+        const float *zc = zt + zpos(c * canon::SLICE);
+        const float *wc = reinterpret_cast<const float *>(w4 + c * 4);
+        long long h1, l1;
+        ok &= canon::split(canon::slice_dot([&](int i) { return __ldg(wc + i); }, [&](int i) { return zc[i]; }), h1,
+                           l1);
+        hi += h1;
+        lo += l1;
       }
-      s = warp_sum_d(s);
-      if (lane == 0) a.logits[(size_t)t * E + e_row] = s + b;
+      canon::warp_sum_fix(hi, lo);
+      if (lane == 0) a.logits[(size_t)t * E + e_row] = canon::logit(canon::join(hi, lo), rinv_s[t], b);
     }
+    if (!ok) range_bad = 1;
   }
 
-  // the last CTA to finish selects the experts of every token
+  // the last CTA to finish selects the experts of every token (one warp each)
   __threadfence();
   __syncthreads();
-  if (tid == 0) is_last = (atomicAdd(a.ticket, 1u) == gridDim.x - 1u) ? 1u : 0u;
+  if (tid == 0) {
+    if (range_bad) set_status(a.status, DEV_RANGE);
+    is_last = (atomicAdd(a.ticket, 1u) == gridDim.x - 1u) ? 1u : 0u;
+  }
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  for (int t = warp; t < T; t += RT_THREADS / 32)
+  for (int t = warp; t < T; t += RT_WARPS)
     warp_topk_gates(a.logits + (size_t)t * E, E, a.k, a.idx + t * a.k, a.gate + t * a.k, &topk_sc[warp]);
   __syncthreads();
   if (tid == 0) atomicExch(a.ticket, 0u);
 }
 
-__global__ void rmsnorm_residual_kernel(const float *x, const float *y, float eps, float *out, int H) {
-  __shared__ double part[32];
+// x_out = RMSNorm(x + y), one CTA per token, with the sum of squares of
+// decode_canon.cuh (warp 0).
+__global__ void __launch_bounds__(256) rmsnorm_residual_kernel(const float *x, const float *y, float eps, float *out,
+                                                               int H) {
   __shared__ float inv;
-  const int t = blockIdx.x;
+  const int t = blockIdx.x, tid = threadIdx.x;
   const float *xr = x + (size_t)t * H;
   const float *yr = y + (size_t)t * H;
-  double ss = 0.0;
-  for (int h = threadIdx.x; h < H; h += blockDim.x) {
-    float z = xr[h] + yr[h];
-    ss += (double)z * z;
-  }
-  ss = warp_sum_d(ss);
-  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    double v = threadIdx.x < blockDim.x / 32 ? part[threadIdx.x] : 0.0;
-    v = warp_sum_d(v);
-    if (threadIdx.x == 0) inv = (float)(1.0 / sqrt(v / (double)H + (double)eps));
+  if (tid < 32) {
+    const double ss = canon::warp_sumsq(
+        [&](int c) {
+          const int b = c * canon::SLICE;
+          return canon::slice_sumsq([&](int i) { return __fadd_rn(xr[b + i], yr[b + i]); });
+        },
+        H / canon::SLICE);
+    if (tid == 0) inv = __double2float_rn(canon::norm_rinv(ss, H, eps));
   }
   __syncthreads();
-  for (int h = threadIdx.x; h < H; h += blockDim.x) out[(size_t)t * H + h] = (xr[h] + yr[h]) * inv;
+  for (int h = tid; h < H; h += 256) out[(size_t)t * H + h] = __fmul_rn(__fadd_rn(xr[h], yr[h]), inv);
 }
 
 size_t decode_ws_bytes(int T, int E) { return (((size_t)T * E * sizeof(double) + 255) & ~(size_t)255) + 256; }
 
 qmoe_status launch_route_decode(const RouteArgs &a, bool resid, cudaStream_t s) {
-  size_t smem = (size_t)a.T * a.H * sizeof(float);
-  int grid = (a.E + RT_THREADS / 32 - 1) / (RT_THREADS / 32);
+  const size_t smem = route_smem_bytes(a.T, a.H);
   const void *fn = resid ? (const void *)route_decode_kernel<true> : (const void *)route_decode_kernel<false>;
-  if (smem > 48 * 1024 &&
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) return QMOE_ERR_CUDA;
+  // static + dynamic shared memory must fit one SM's opt-in limit; above the
+  // default 48 KB the kernel's dynamic limit has to be raised
+  if (smem + fa.sharedSizeBytes > max_smem_optin()) return QMOE_ERR_UNSUPPORTED;
+  if (smem + fa.sharedSizeBytes > 48 * 1024 &&
       cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return QMOE_ERR_CUDA;
+  const int grid = (a.E + RT_WARPS - 1) / RT_WARPS;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(RT_THREADS);
@@ -274,20 +340,23 @@ constexpr int FIXED_MAX_DEVICES = 64;
 std::mutex g_fixed_mutex;
 void *g_fixed_ptr[FIXED_MAX_DEVICES];
 
-// First call on a device: look up the array's address and zero it
-// (synchronous; no allocation). Later calls reuse the address.
+// Every call looks the array's address up again (cudaGetSymbolAddress
+// allocates nothing): after a device reset, or in another context on the same
+// device, the module is loaded afresh and the array may sit elsewhere. The
+// first call that sees an address on a device zeroes the array there
+// (synchronous; the ticket must start at zero).
 qmoe_status fixed_scratch(void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return QMOE_ERR_CUDA;
   if (dev < 0 || dev >= FIXED_MAX_DEVICES) return QMOE_ERR_UNSUPPORTED;
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) return QMOE_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_fixed_mutex);
-  if (!g_fixed_ptr[dev]) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) return QMOE_ERR_CUDA;
+  if (g_fixed_ptr[dev] != p) {
     if (cudaMemset(p, 0, QMOE_ROUTE_FIXED_SCRATCH_BYTES) != cudaSuccess) return QMOE_ERR_CUDA;
     g_fixed_ptr[dev] = p;
   }
-  *out = g_fixed_ptr[dev];
+  *out = p;
   return QMOE_OK;
 }
 
@@ -322,6 +391,7 @@ extern "C" qmoe_status qmoe_rmsnorm_residual(const float *x_in, const float *y, 
   if (!x_in || !y || !x_out || T < 1 || H < 1) return QMOE_ERR_INVALID_ARG;
   if (!aligned16(x_in) || !aligned16(y) || !aligned16(x_out)) return QMOE_ERR_INVALID_ARG;
   if (!(eps >= 0.0f)) return QMOE_ERR_INVALID_ARG;
+  if (H % canon::SLICE) return QMOE_ERR_UNSUPPORTED;
   rmsnorm_residual_kernel<<<T, 256, 0, (cudaStream_t)stream>>>(x_in, y, eps, x_out, H);
   note_launch();
   return cuda_status(cudaGetLastError());

@@ -34,6 +34,10 @@ __device__ __forceinline__ bool ranks_above(double va, int ea, double vb, int eb
   return va > vb || (va == vb && ea < eb);
 }
 
+// A NaN logit ranks as -infinity, so the ranking is a total order and the k
+// selected slots are always k distinct valid experts.
+__device__ __forceinline__ double rank_value(double v) { return isnan(v) ? -INFINITY : v; }
+
 // One warp; get(e) returns the token's float64 logit of expert e (global
 // memory written by other CTAs and read through L2, or shared memory).
 // M = values per lane = ceil(E / 32).
@@ -46,7 +50,7 @@ __device__ inline void warp_topk_gates_m(Get get, int E, int k, int32_t *idx_out
 #pragma unroll
   for (int j = 0; j < M; ++j) {
     const int e = lane + 32 * j;
-    val[j] = e < E ? get(e) : 0.0;
+    val[j] = e < E ? rank_value(get(e)) : 0.0;
   }
 #pragma unroll
   for (int j = 0; j < M; ++j) {
@@ -108,7 +112,7 @@ __device__ inline void warp_topk_gates_m(Get get, int E, int k, int32_t *idx_out
         const int e = lane + 32 * j;
         const double v = val[j];
         int rank = 0;
-        for (int e2 = 0; e2 < E && rank < k; ++e2) rank += ranks_above(get(e2), e2, v, e) ? 1 : 0;
+        for (int e2 = 0; e2 < E && rank < k; ++e2) rank += ranks_above(rank_value(get(e2)), e2, v, e) ? 1 : 0;
         if (rank < k) {
           sc->sel_e[rank] = e;
           sc->sel_v[rank] = v;

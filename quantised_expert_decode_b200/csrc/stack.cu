@@ -1,5 +1,6 @@
 // Layer stack: L x (route -> decode FFN) + residual RMSNorm, captured once into
 // one CUDA graph whose arguments are fixed-address buffers in caller workspace.
+#include <algorithm>
 #include <new>
 #include <vector>
 
@@ -33,6 +34,8 @@ struct qmoe_stack {
   qmoe::FusedPlan fplan;
   qmoe::FusedBufs fbufs;
   std::vector<cudaEvent_t> events;  // 2L + 1 when timing
+  long long *trace;                 // fused path with timing: [L][G][points] SM clock stamps
+  int trace_ctas;
 };
 
 namespace {
@@ -40,7 +43,7 @@ namespace {
 size_t al(size_t b) { return (b + 255) & ~(size_t)255; }
 
 struct Layout {
-  size_t x, idx, gate, status, route, ffn, fused, total;
+  size_t x, idx, gate, status, route, ffn, fused, trace, total;
   bool use_fused;
   qmoe::FusedPlan fplan;
 };
@@ -51,13 +54,16 @@ Layout layout_of(const qmoe_stack_desc *d) {
   l.use_fused = d->T == 1 && !(d->flags & QMOE_STACK_LAYERWISE) &&
                 qmoe::fused_stack_plan(e.fmt, e.E, e.H, e.I, d->k, &l.fplan);
   l.fused = l.use_fused ? al(qmoe::fused_stack_ws_bytes(d->L, e.E, e.H, e.I, d->k)) : 0;
+  l.trace = (l.use_fused && (d->flags & QMOE_STACK_TIMING))
+                ? al((size_t)d->L * qmoe::num_sms() * qmoe::fused_trace_points() * sizeof(long long))
+                : 0;
   l.x = al((size_t)d->T * e.H * 4);
   l.idx = al((size_t)d->L * d->T * d->k * 4);
   l.gate = l.idx;
   l.status = 256;
   l.route = al(qmoe_route_workspace_bytes(d->T, e.E));
   l.ffn = al(qmoe_decode_workspace_bytes(d->T, d->k, e.H, e.I));
-  l.total = 5 * l.x + l.idx + l.gate + l.status + l.route + l.ffn + l.fused;
+  l.total = 5 * l.x + l.idx + l.gate + l.status + l.route + l.ffn + l.fused + l.trace;
   return l;
 }
 
@@ -113,7 +119,7 @@ qmoe_status record_fused(qmoe_stack *s, cudaStream_t cs, bool coop) {
   const bool timing = !s->events.empty();
   if (timing && cudaEventRecordWithFlags(s->events[0], cs, cudaEventRecordExternal) != cudaSuccess) return QMOE_ERR_CUDA;
   qmoe_status st = qmoe::fused_launch(s->fbufs, s->fplan, s->fmt, s->L, s->E, s->H, s->I, s->k, s->eps, s->x_in,
-                                      s->x_out, s->idx, s->gate, s->status, cs, coop);
+                                      s->x_out, s->idx, s->gate, s->status, s->trace, cs, coop);
   if (st != QMOE_OK) return st;
   if (timing && cudaEventRecordWithFlags(s->events[1], cs, cudaEventRecordExternal) != cudaSuccess) return QMOE_ERR_CUDA;
   s->kernels = 1;
@@ -196,7 +202,16 @@ extern "C" qmoe_status qmoe_stack_create(const qmoe_stack_desc *d, void *workspa
   s->ffn_ws = p; s->ffn_ws_bytes = lo.ffn; p += lo.ffn;
   s->path = lo.use_fused ? QMOE_PATH_FUSED : QMOE_PATH_LAYERWISE;
   s->fplan = lo.fplan;
-  if (lo.use_fused) s->fbufs = qmoe::fused_carve(p, d->L, s->E, s->H, s->I, s->k);
+  s->trace = nullptr;
+  s->trace_ctas = 0;
+  if (lo.use_fused) {
+    s->fbufs = qmoe::fused_carve(p, d->L, s->E, s->H, s->I, s->k);
+    p += lo.fused;
+    if (lo.trace) {
+      s->trace = reinterpret_cast<long long *>(p);
+      s->trace_ctas = qmoe::num_sms();
+    }
+  }
   if (cudaMemsetAsync(workspace, 0, lo.total, (cudaStream_t)stream) != cudaSuccess ||
       cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) {
     delete s;
@@ -242,6 +257,10 @@ extern "C" qmoe_status qmoe_stack_buffers(const qmoe_stack *s, float **x_in, flo
 
 extern "C" int qmoe_stack_kernels_per_replay(const qmoe_stack *s) { return s ? s->kernels : 0; }
 
+extern "C" uint32_t *qmoe_stack_barrier_word(const qmoe_stack *s) {
+  return (s && s->path == QMOE_PATH_FUSED) ? s->fbufs.bar : nullptr;
+}
+
 extern "C" int qmoe_stack_path(const qmoe_stack *s) { return s ? s->path : -1; }
 
 extern "C" qmoe_status qmoe_stack_decode(qmoe_stack *s, qmoe_stream_t stream) {
@@ -267,13 +286,39 @@ extern "C" qmoe_status qmoe_stack_layer_times(const qmoe_stack *s, float *route_
   if (!s) return QMOE_ERR_INVALID_ARG;
   if (s->events.empty()) return QMOE_ERR_UNSUPPORTED;
   if (s->path == QMOE_PATH_FUSED) {
+    // the kernel's event-timed duration, split over the layers in proportion
+    // to each layer's median CTA clock span (start to start); route_ms is the
+    // median span from a layer's start to its top-k
     float ms = 0.f;
     if (cudaEventSynchronize(s->events[1]) != cudaSuccess ||
         cudaEventElapsedTime(&ms, s->events[0], s->events[1]) != cudaSuccess)
       return QMOE_ERR_CUDA;
+    const int P = qmoe::fused_trace_points(), G = s->trace_ctas;
+    std::vector<long long> tr((size_t)s->L * G * P);
+    if (cudaMemcpy(tr.data(), s->trace, tr.size() * sizeof(long long), cudaMemcpyDeviceToHost) != cudaSuccess)
+      return QMOE_ERR_CUDA;
+    auto median = [](std::vector<double> v) {
+      std::nth_element(v.begin(), v.begin() + v.size() / 2, v.end());
+      return v[v.size() / 2];
+    };
+    std::vector<double> span(s->L), topk(s->L);
+    double total = 0.0;
     for (int l = 0; l < s->L; ++l) {
-      if (route_ms) route_ms[l] = 0.f;
-      if (ffn_ms) ffn_ms[l] = ms / s->L;
+      std::vector<double> a(G), b(G);
+      for (int c = 0; c < G; ++c) {
+        const long long *t = &tr[((size_t)l * G + c) * P];
+        a[c] = (double)(t[6] - t[0]);   // layer start -> second grid barrier passed
+        b[c] = (double)(t[1] - t[0]);   // layer start -> top-k done
+      }
+      span[l] = median(a);
+      topk[l] = median(b);
+      total += span[l];
+    }
+    for (int l = 0; l < s->L; ++l) {
+      const double layer_ms = total > 0 ? ms * span[l] / total : ms / s->L;
+      const double route = span[l] > 0 ? layer_ms * topk[l] / span[l] : 0.0;
+      if (route_ms) route_ms[l] = (float)route;
+      if (ffn_ms) ffn_ms[l] = (float)(layer_ms - route);
     }
     return QMOE_OK;
   }
@@ -286,5 +331,20 @@ extern "C" qmoe_status qmoe_stack_layer_times(const qmoe_stack *s, float *route_
     if (route_ms) route_ms[l] = a;
     if (ffn_ms) ffn_ms[l] = b;
   }
+  return QMOE_OK;
+}
+
+extern "C" qmoe_status qmoe_stack_trace(const qmoe_stack *s, int64_t *cycles_host, size_t count, int *ctas,
+                                        int *points) {
+  if (!s || !cycles_host) return QMOE_ERR_INVALID_ARG;
+  if (!s->trace) return QMOE_ERR_UNSUPPORTED;
+  const int P = qmoe::fused_trace_points();
+  const size_t n = (size_t)s->L * s->trace_ctas * P;
+  if (count < n) return QMOE_ERR_WORKSPACE;
+  if (cudaDeviceSynchronize() != cudaSuccess ||
+      cudaMemcpy(cycles_host, s->trace, n * sizeof(long long), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return QMOE_ERR_CUDA;
+  if (ctas) *ctas = s->trace_ctas;
+  if (points) *points = P;
   return QMOE_OK;
 }

@@ -11,18 +11,20 @@
 //      renormalised gates (one warp, identical in every CTA); then the producer
 //      warp issues this layer's weight copies.
 //   C  gate/up tiles (selected expert j, 16-row tile r, gate or up), one ring
-//      item each: a_g = Wg x or a_u = Wu x for those 16 rows -> global; the
-//      warp that completes the last of the four tiles of a 32-row block
-//      forms h = silu(a_g) * a_u for the block, quantises it into limbs and
-//      writes them to global (one block quantised once, by one warp)
+//      item each: a_g = Wg x or a_u = Wu x for those 16 rows -> shared
+//      memory. A CTA holds whole 32-row blocks of h (the four tiles gate and
+//      up of rows 32b..32b+31), so the warp that completes a block's fourth
+//      tile forms h = silu(a_g) * a_u from shared memory, quantises it into
+//      limbs and writes them to global (one block quantised once, by one warp)
 //      ---- grid barrier (h limbs complete) ----
 //   D  row owners: the limbs of every h_j in one bulk copy, down tiles of rows R_c for every selected
 //      expert (prefetched during C), y[R_c] = sum_j g_j * (Wd_j h_j)[R_c] in
 //      slot order, z_{l+1}[R_c] = x_l[R_c] + y[R_c]; then, from the rows
 //      R_c of the next layer's transposed router (prefetched), partial logits
 //      sum_{h in R_c} Wr_{l+1}[e][h] z[h] for every expert and the partial sum of
-//      squares of z, both added as fixed-point integers (scale 2^40) so the
-//      totals are exact and independent of the order of the additions.
+//      squares of z; R_c is one 16-element slice, so both are the slice
+//      partials of decode_canon.cuh, added as pairs of integers so the totals
+//      are exact and independent of the order of the additions.
 //      ---- grid barrier (z, logit and norm partials complete) ----
 // The router logit of the next layer is Wr (z / rms) = (Wr z) / rms, which is
 // why the partial logits can be formed before the norm is known. Layer 0 uses
@@ -30,6 +32,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "decode_canon.cuh"
 #include "decode_tile.cuh"
 #include "layout.cuh"
 #include "route_common.cuh"
@@ -42,9 +45,14 @@ using namespace tile;
 constexpr int SK_NCW = 7;  // consumer warps; with the producer 256 threads, so up to 255 registers
 constexpr int SK_THREADS = 32 * (SK_NCW + 1);
 constexpr int SK_MAXK = 16;
-constexpr int CONS_BAR = 1;
-constexpr double FIX_SCALE = 1099511627776.0;  // 2^40
-constexpr double FIX_INV = 1.0 / 1099511627776.0;
+constexpr int TRACE_POINTS = 8;
+// Trace points of a layer (SM clock of the CTA's consumer thread 0): layer
+// start; top-k done; gate/up tiles start; gate/up tiles done (all consumer
+// warps); first grid barrier passed; down tiles and partials done; second
+// grid barrier passed.
+enum { TP_START = 0, TP_TOPK, TP_TILES, TP_TILES_DONE, TP_BAR1, TP_DOWN_DONE, TP_BAR2 };
+constexpr int CONS_BAR = 1;   // the consumer warps
+constexpr int PLAN_BAR = 2;   // consumer warp 0 and the producer warp
 
 struct StackArgs {
   int L, E, H, I, k;
@@ -58,21 +66,21 @@ struct StackArgs {
   int32_t *idx_rec;           // [L][k]
   float *gate_rec;            // [L][k]
   float *zbuf;                // [2][H]
-  unsigned long long *lacc;   // [2][E] fixed-point partial-logit sums (two's complement)
-  unsigned long long *ssacc;  // [2] fixed-point sum of squares
-  float *hbuf;                // [2][k][I]: a_g, a_u
+  unsigned long long *lacc;   // [2 parity][2 hi|lo][E] integer partial-logit sums (two's complement)
+  double *ssq;                // [2 parity][H/16] slice sums of squares
   uint8_t *lbuf;              // [k][I/32][LIMB_REC]: limbs of h
   float2 *lscg;               // [k][I/32]: (s, s * sum X) of h's blocks
-  unsigned *qcnt;             // [k][I/32]: tiles of the block completed this layer
   unsigned *bar;
   int32_t *status;
+  long long *trace;           // [L][G][TRACE_POINTS] SM clock stamps (consumer thread 0), or null
   int nslots, slot_bytes;
+  int ncons;                  // consumer warps that take ring items; nslots is a multiple of it
   int w_rows, w_free;         // gate/up work weights of CTAs with / without output rows
 };
 
 struct SkState {
   int abort;
-  int turn;  // next ring item whose arrival a consumer warp may wait for
+  int acq;   // gate/up ring items acquired by the consumer warps so far (all layers)
   int idx[SK_MAXK];
   float gate[SK_MAXK];
   float ztmp[16];
@@ -81,12 +89,18 @@ struct SkState {
 };
 
 struct SkLayout {
-  size_t ring, dnbuf, wrtbuf, xs, limbs, lsc, logits, ytmp, bars, state, total;
+  size_t ring, dnbuf, wrtbuf, xs, limbs, lsc, logits, ytmp, hloc, bars, state, total;
 };
+
+// Blocks of h a CTA of a G-CTA grid holds at most (each: a_g and a_u of 32 rows,
+// then a completion counter).
+__host__ __device__ inline int sk_max_local_blocks(int k, int I, int G) { return (k * (I / 32) + G - 1) / G; }
+constexpr int HLOC_BYTES = 2 * 32 * 4 + 16;
 
 __host__ __device__ inline size_t al128(size_t v) { return (v + 127) & ~(size_t)127; }
 
-__host__ __device__ inline SkLayout sk_layout(int bits, int E, int H, int I, int k, int nslots, int slot_bytes) {
+__host__ __device__ inline SkLayout sk_layout(int bits, int E, int H, int I, int k, int nslots, int slot_bytes,
+                                               int G) {
   SkLayout o;
   const size_t tdn = (size_t)tile_bytes(bits, I);
   const size_t vecs = (size_t)((H / 32) > k * (I / 32) ? (H / 32) : k * (I / 32));  // limb records
@@ -98,27 +112,43 @@ __host__ __device__ inline SkLayout sk_layout(int bits, int E, int H, int I, int
   o.lsc = al128(o.limbs + vecs * LIMB_REC);
   o.logits = al128(o.lsc + vecs * 8);
   o.ytmp = al128(o.logits + (size_t)E * 8);
-  o.bars = al128(o.ytmp + (size_t)k * 16 * 4);
+  o.hloc = al128(o.ytmp + (size_t)k * 16 * 4);
+  o.bars = al128(o.hloc + (size_t)sk_max_local_blocks(k, I, G) * HLOC_BYTES);
   o.state = al128(o.bars + (size_t)(2 * nslots + 3) * 8);
   o.total = o.state + sizeof(SkState);
   return o;
 }
 
-__device__ __forceinline__ unsigned long long to_fixed(double v) {
-  return (unsigned long long)__double2ll_rn(v * FIX_SCALE);
+// Adds one slice partial to an exact (hi, lo) integer total; false when the
+// partial is out of the range the split covers.
+__device__ __forceinline__ bool add_fixed(unsigned long long *hi, unsigned long long *lo, double p) {
+  long long h, l;
+  const bool ok = canon::split(p, h, l);
+  atomicAdd(hi, (unsigned long long)h);
+  atomicAdd(lo, (unsigned long long)l);
+  return ok;
 }
-__device__ __forceinline__ double from_fixed(unsigned long long v) { return (double)(long long)v * FIX_INV; }
+__device__ __forceinline__ double read_fixed(const unsigned long long *hi, const unsigned long long *lo) {
+  return canon::join((long long)__ldcg(hi), (long long)__ldcg(lo));
+}
 
 // Consumer-side grid barrier: the 256 consumer threads meet, one thread joins
 // the grid, the consumers meet again. Returns false once the CTA has aborted.
-__device__ __forceinline__ bool cons_grid_barrier(const StackArgs &a, SkState *st, int tid) {
+__device__ __forceinline__ void trace_point(const StackArgs &a, int l, int p) {
+  if (a.trace) a.trace[((size_t)l * gridDim.x + blockIdx.x) * TRACE_POINTS + p] = clock64();
+}
+
+__device__ __forceinline__ bool cons_grid_barrier(const StackArgs &a, SkState *st, int tid, int l = -1,
+                                                  int p_before = 0) {
   named_barrier_sync(CONS_BAR, SK_NCW * 32);
   if (tid == 0) {
+    if (l >= 0) trace_point(a, l, p_before);
     if (!*(volatile int *)&st->abort && !grid_barrier_one_thread(a.bar, gridDim.x)) {
       set_status(a.status, DEV_TIMEOUT);
       *(volatile int *)&st->abort = 1;
     }
     __threadfence();
+    if (l >= 0) trace_point(a, l, p_before + 1);
   }
   named_barrier_sync(CONS_BAR, SK_NCW * 32);
   return !*(volatile int *)&st->abort;
@@ -131,24 +161,17 @@ __device__ __noinline__ void topk_smem(const double *logits, int E, int k, int32
 }
 
 // One warp: h = silu(a_g) * a_u for the 32 rows of block b of selected
-// expert j (lane i: row 32b + i), quantised exactly as quant_chunk_inl does a
-// 32-element block, limbs and scales written to global; the block's tile
-// counter is reset for the next layer.
-__device__ __noinline__ void quant_h_block(const StackArgs &a, int j, int b, int lane) {
-  // the other tiles' a_g / a_u are visible: their warps released them with
-  // the block counter's increments, which lane 0 acquired with its own
+// expert j (lane i: row 32b + i) from the block's a_g / a_u in shared memory,
+// quantised exactly as every decode path quantises a 32-element block; limbs
+// and scales go to global for the row owners.
+__device__ __noinline__ void quant_h_block(const StackArgs &a, const float *hl, int j, int b, int lane) {
   const int nblkI = a.I / 32;
-  const float gv = __ldcg(a.hbuf + (size_t)j * a.I + b * 32 + lane);
-  const float uv = __ldcg(a.hbuf + ((size_t)a.k + j) * a.I + b * 32 + lane);
-  const float h = silu_f(gv) * uv;
+  const float h = canon::hval(hl[lane], hl[32 + lane]);
   float m = fabsf(h);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  float sc = 0.0f, inv = 0.0f;
-  if (m > 0.0f) {
-    sc = m * (1.0f / QMAX);
-    inv = __frcp_rn(sc);
-  }
+  float sc, inv;
+  block_scale(m, sc, inv);
   const int X = quant_one(h, inv);
   int l[3];
   limbs3(X, l[0], l[1], l[2]);
@@ -163,10 +186,7 @@ __device__ __noinline__ void quant_h_block(const StackArgs &a, int j, int b, int
   int sx = X;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, o);
-  if (lane == 0) {
-    a.lscg[(size_t)j * nblkI + b] = make_float2(sc, sc * (float)sx);
-    a.qcnt[(size_t)j * nblkI + b] = 0u;
-  }
+  if (lane == 0) a.lscg[(size_t)j * nblkI + b] = make_float2(sc, __fmul_rn(sc, (float)sx));
 }
 
 template <int BITS>
@@ -174,7 +194,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
   extern __shared__ __align__(128) uint8_t smem[];
   const int S = a.nslots;
   const int H = a.H, I = a.I, E = a.E, k = a.k, L = a.L;
-  const SkLayout lay = sk_layout(BITS, E, H, I, k, S, a.slot_bytes);
+  const SkLayout lay = sk_layout(BITS, E, H, I, k, S, a.slot_bytes, (int)gridDim.x);
   uint8_t *ring = smem + lay.ring;
   uint8_t *dnbuf = smem + lay.dnbuf;
   float *wrtbuf = reinterpret_cast<float *>(smem + lay.wrtbuf);
@@ -183,6 +203,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
   float2 *lsc = reinterpret_cast<float2 *>(smem + lay.lsc);
   double *logits = reinterpret_cast<double *>(smem + lay.logits);
   float *ytmp = reinterpret_cast<float *>(smem + lay.ytmp);
+  uint8_t *hloc = smem + lay.hloc;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.bars);
   uint64_t *empty = full + S;
   uint64_t *dnbar = empty + S;
@@ -197,18 +218,18 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
   const bool rows = c < H16;
   const int r0 = 16 * c;
   // gate/up items (selected expert j, matrix gate or up, 16-row tile r) of this
-  // CTA, balanced by bytes. Items, not (gate, up) pairs, are the unit of
-  // assignment: the two halves of a pair meet through the per-block counters
-  // in global memory, and a CTA then holds at most ceil(2 k I16 / G) items (7
-  // for 960 items on 148 CTAs), one per consumer warp, where pairs gave some
-  // CTAs 8 items and one warp two tiles in a row.
+  // CTA: item i = 2 (j I16 + r) + matrix, so the four items 4B..4B+3 are the
+  // gate and up tiles of the 32-row block B = j (I/32) + b of h. A CTA takes
+  // whole blocks (1 or 2 of the 240 at the 512-expert shape), so each block
+  // of h is formed and quantised where its tiles were computed.
   auto wcum = [&](int cc) -> long long {
     const int nr = cc < H16 ? cc : H16;
     return (long long)nr * a.w_rows + (long long)(cc - nr) * a.w_free;
   };
-  const int NI = 2 * k * I16;   // item i: unit i >> 1 = (j, r), matrix i & 1
+  const int NBLK = k * nblkI;
   const long long WT = wcum(G);
-  const int ilo = (int)(wcum(c) * NI / WT), ihi = (int)(wcum(c + 1) * NI / WT);
+  const int blo = (int)(wcum(c) * NBLK / WT), bhi = (int)(wcum(c + 1) * NBLK / WT);
+  const int ilo = 4 * blo, ihi = 4 * bhi;
   const int nitems = ihi - ilo;
   const int nth = SK_NCW * 32;
   const bool producer = warp == SK_NCW;
@@ -223,7 +244,9 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
     mbar_init(hbar, 1);
     fence_mbar_init();
     st->abort = 0;
-    st->turn = 0;
+    st->acq = 0;
+    for (int q = 0; q < sk_max_local_blocks(k, I, G); ++q)
+      *reinterpret_cast<int *>(hloc + q * HLOC_BYTES + 256) = 0;
     for (int j = 0; j < SK_MAXK; ++j) st->vid[j] = j;
   }
   __syncthreads();
@@ -244,95 +267,103 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
       set_status(a.status, DEV_TIMEOUT);
       st->abort = 1;
     } else {
-      for (int e = tid; e < E; e += nth) {
-        double p = 0.0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) p = fma((double)wrtbuf[i * E + e], (double)st->ztmp[i], p);
-        atomicAdd(&a.lacc[e], to_fixed(p));
-      }
+      bool ok = true;
+      for (int e = tid; e < E; e += nth)
+        ok &= add_fixed(&a.lacc[e], &a.lacc[E + e],
+                        canon::slice_dot([&](int i) { return wrtbuf[i * E + e]; }, [&](int i) { return st->ztmp[i]; }));
+      if (!ok) set_status(a.status, DEV_RANGE);
     }
   }
   if (!producer) cons_grid_barrier(a, st, tid);
 
   // Ring bookkeeping shared by producer and consumers (same sequence of items).
+  // Item n goes to slot n % S; within a layer the m-th item of the CTA goes
+  // to consumer warp m % NA, and S is a multiple of NA, so a slot's phases of
+  // one layer are taken in order by one warp (and its phase of the previous
+  // layer completed before the layer's grid barriers): when a warp waits for
+  // item n the slot's barrier is in the phase of item n, and the parity wait
+  // is exact.
   int nring = 0;
-  // Consumers take arrival waits in ring order; see the per-layer FFN kernel.
+  const int NA = a.ncons;
   auto wait_full = [&](int n) -> bool {
     const long long dl = clock64() + WAIT_BUDGET_CYCLES;
-    bool ok = true;
-    while (*(volatile int *)&st->turn != n) {
+    const uint32_t par = (uint32_t)((n / S) & 1);
+    while (!mbar_try_wait(&full[n % S], par)) {
       if (*(volatile int *)&st->abort) return false;
       if (clock64() > dl) {
-        ok = false;
-        break;
+        set_status(a.status, DEV_TIMEOUT);
+        *(volatile int *)&st->abort = 1;
+        return false;
       }
     }
-    if (ok) ok = mbar_wait(&full[n % S], (uint32_t)((n / S) & 1), dl);
-    if (!ok) {
-      set_status(a.status, DEV_TIMEOUT);
-      *(volatile int *)&st->abort = 1;
-      return false;
-    }
     __syncwarp();
-    if (lane == 0) {
-      __threadfence_block();
-      *(volatile int *)&st->turn = n + 1;
-    }
+    if (lane == 0) atomicAdd(&st->acq, 1);
     return true;
   };
 
   for (int l = 0; l < L; ++l) {
     const int par = l & 1;
+    if (tid == 0) trace_point(a, l, TP_START);
     // ------------------------------------------------------------------ A --
     if (!producer && !*(volatile int *)&st->abort) {
       // one batch of loads: sum of squares, z, partial logits, bias
       const float4 *zb = reinterpret_cast<const float4 *>(a.zbuf + (size_t)par * H);
       const float *b = a.bias[l];
-      const unsigned long long *la = a.lacc + (size_t)par * E;
-      const unsigned long long ssv = __ldcg(&a.ssacc[par]);
+      const unsigned long long *la = a.lacc + (size_t)par * 2 * E;
       float4 zv[4];
-      unsigned long long lv[4];
+      unsigned long long lh[4], ll[4];
       float bv[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int q = tid + i * nth;
         if (q < H / 4) zv[i] = __ldcg(zb + q);
         if (q < E) {
-          lv[i] = __ldcg(la + q);
+          lh[i] = __ldcg(la + q);
+          ll[i] = __ldcg(la + E + q);
           bv[i] = b ? __ldg(b + q) : 0.0f;
         }
       }
-      const double rms = l > 0 ? sqrt(from_fixed(ssv) / (double)H + (double)a.eps) : 1.0;
-      const double rinv = 1.0 / rms;
-      const float inv = (float)rinv;
+      // every warp adds the slice sums of squares itself (same order, same value)
+      const double *sq = a.ssq + (size_t)par * H16;
+      const double rinv =
+          l > 0 ? canon::norm_rinv(canon::warp_sumsq([&](int cc) { return __ldcg(sq + cc); }, H16), H, a.eps) : 1.0;
+      const float inv = __double2float_rn(rinv);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int q = tid + i * nth;
         if (q < H / 4) {
           float4 v = zv[i];
           if (l > 0) {
-            v.x *= inv; v.y *= inv; v.z *= inv; v.w *= inv;
+            v.x = __fmul_rn(v.x, inv); v.y = __fmul_rn(v.y, inv); v.z = __fmul_rn(v.z, inv); v.w = __fmul_rn(v.w, inv);
           }
           reinterpret_cast<float4 *>(xs)[q] = v;
         }
-        if (q < E) logits[q] = from_fixed(lv[i]) * rinv + (double)bv[i];
+        if (q < E) logits[q] = canon::logit(canon::join((long long)lh[i], (long long)ll[i]), rinv, (double)bv[i]);
       }
       for (int q = tid + 4 * nth; q < H / 4; q += nth) {   // larger geometries only
         float4 v = __ldcg(zb + q);
         if (l > 0) {
-          v.x *= inv; v.y *= inv; v.z *= inv; v.w *= inv;
+          v.x = __fmul_rn(v.x, inv); v.y = __fmul_rn(v.y, inv); v.z = __fmul_rn(v.z, inv); v.w = __fmul_rn(v.w, inv);
         }
         reinterpret_cast<float4 *>(xs)[q] = v;
       }
-      for (int q = tid + 4 * nth; q < E; q += nth) logits[q] = from_fixed(__ldcg(la + q)) * rinv + (b ? (double)b[q] : 0.0);
+      for (int q = tid + 4 * nth; q < E; q += nth)
+        logits[q] = canon::logit(read_fixed(la + q, la + E + q), rinv, b ? (double)b[q] : 0.0);
       // clear the other parity's accumulators for the next layer (read last by
       // every CTA before the previous barriers)
-      unsigned long long *lz = a.lacc + (size_t)(par ^ 1) * E;
-      for (int e = c * nth + tid; e < E; e += G * nth) lz[e] = 0ull;
-      if (c == 0 && tid == 0) a.ssacc[par ^ 1] = 0ull;
+      unsigned long long *lz = a.lacc + (size_t)(par ^ 1) * 2 * E;
+      for (int e = c * nth + tid; e < 2 * E; e += G * nth) lz[e] = 0ull;
       named_barrier_sync(CONS_BAR, nth);
       if (warp == 0) {
         topk_smem(logits, E, k, st->idx, st->gate, &st->tks);
+        if (lane == 0) trace_point(a, l, TP_TOPK);
+        // the selection always names k distinct experts in [0, E) (NaN logits
+        // rank lowest); checked anyway before any address is formed from it
+        if (lane < k && (unsigned)st->idx[lane] >= (unsigned)E) {
+          set_status(a.status, DEV_BAD_INDEX);
+          *(volatile int *)&st->abort = 1;
+        }
+        __syncwarp();
         if (c == 0 && lane < k) {
           a.idx_rec[l * k + lane] = st->idx[lane];
           a.gate_rec[l * k + lane] = st->gate[lane];
@@ -346,8 +377,11 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
         }
       }
     }
-    // plan ready (includes the producer warp); every thread sees one abort value
-    if (__syncthreads_or(*(volatile int *)&st->abort)) break;
+    // Warp 0 hands the selection to the producer as soon as its top-k is done,
+    // while the other consumer warps still quantise x. Both sides read one
+    // abort value: nothing sets it between here and the consumer barrier below.
+    if (warp == 0 || producer) named_barrier_sync(PLAN_BAR, 64);
+    if (producer && *(volatile int *)&st->abort) break;
 
     if (producer) {
       // -------------------------------------------------------------- B --
@@ -383,7 +417,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
         const int want = nring + nitems;
         const long long dl = clock64() + WAIT_BUDGET_CYCLES;
         bool ok = true;
-        while (*(volatile int *)&st->turn < want) {
+        while (*(volatile int *)&st->acq < want) {
           if (*(volatile int *)&st->abort) {
             ok = false;
             break;
@@ -412,39 +446,52 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
       continue;
     }
 
+    named_barrier_sync(CONS_BAR, nth);   // x limbs complete
+    if (*(volatile int *)&st->abort) break;
+    if (tid == 0) trace_point(a, l, TP_TILES);
+
     // -------------------------------------------------------------------- C --
     // Each consumer warp first asks L2 for its own items with ordinary
     // prefetches. They travel the load path beside the producer's bulk copies
     // of the same bytes, so more of the layer's weights are in flight per SM.
-    for (int m = warp; m < nitems; m += SK_NCW) {
+    for (int m = warp; warp < NA && m < nitems; m += NA) {
       const int i = ilo + m, u = i >> 1, mat = i & 1, j = u / I16, r = u % I16;
       const uint8_t *src = a.gu[l] + (((size_t)st->idx[j] * 2 + mat) * I16 + r) * (size_t)tgu;
       for (int off = lane * 128; off < tgu; off += 32 * 128)
         asm volatile("prefetch.global.L2 [%0];" ::"l"(src + off));
     }
-    for (int m = warp; m < nitems; m += SK_NCW) {
+    for (int m = warp; warp < NA && m < nitems; m += NA) {
       const int n = nring + m;
       if (!wait_full(n)) break;
       const int i = ilo + m, u = i >> 1, mat = i & 1, j = u / I16, r = u % I16;
       const float2 o = tile_dot1<BITS, 4>(ring + (size_t)(n % S) * a.slot_bytes, nblkH, limbs, lsc);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[n % S]);
+      // this tile's 16 rows into the local block: a_g / a_u of rows 16 (r & 1) ..
+      float *hl = reinterpret_cast<float *>(hloc + ((i >> 2) - blo) * HLOC_BYTES);
       if ((lane & 3) == 0) {   // lanes of quad g hold rows g and g+8 of the tile
         const int g = lane >> 2;
-        float *dst = a.hbuf + ((size_t)mat * k + j) * I + r * 16;
-        dst[g] = o.x;
-        dst[g + 8] = o.y;
+        hl[mat * 32 + (r & 1) * 16 + g] = o.x;
+        hl[mat * 32 + (r & 1) * 16 + g + 8] = o.y;
       }
-      // four tiles (gate and up of rows 32b..32b+31) make a block of h; the
-      // warp that completes the fourth quantises the block
+      // the warp that completes the block's fourth tile quantises the block
       __syncwarp();
-      unsigned last = 0;
-      if (lane == 0)   // release this tile's values; the fourth arriver acquires all four
-        last = atom_add_acq_rel_gpu(a.qcnt + (size_t)j * nblkI + (r >> 1), 1u) == 3u;
-      if (__shfl_sync(0xffffffffu, last, 0)) quant_h_block(a, j, r >> 1, lane);
+      int last = 0;
+      if (lane == 0) {
+        __threadfence_block();
+        last = atomicAdd(reinterpret_cast<int *>(hl + 64), 1) == 3;
+        if (last) {
+          __threadfence_block();
+          *reinterpret_cast<volatile int *>(hl + 64) = 0;   // for the next layer
+        }
+      }
+      if (__shfl_sync(0xffffffffu, last, 0)) {
+        __syncwarp();
+        quant_h_block(a, hl, j, r >> 1, lane);
+      }
     }
     nring += nitems;
-    if (!cons_grid_barrier(a, st, tid)) continue;
+    if (!cons_grid_barrier(a, st, tid, l, TP_TILES_DONE)) continue;
 
     // -------------------------------------------------------------------- D --
     if (rows) {
@@ -481,35 +528,33 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
       }
       named_barrier_sync(CONS_BAR, nth);
       if (ok && warp == 0) {
-        double ssp = 0.0;
         if (lane < 16) {
           float y = 0.0f;
-          for (int j = 0; j < k; ++j) y = fmaf(st->gate[j], ytmp[j * 16 + lane], y);  // slot order
-          const float z = xs[r0 + lane] + y;
+          for (int j = 0; j < k; ++j) y = canon::combine_step(y, st->gate[j], ytmp[j * 16 + lane]);  // slot order
+          const float z = __fadd_rn(xs[r0 + lane], y);
           st->ztmp[lane] = z;
           a.zbuf[(size_t)(par ^ 1) * H + r0 + lane] = z;
-          ssp = (double)z * (double)z;
         }
-        ssp = warp_sum_d(ssp);
-        if (lane == 0) atomicAdd(&a.ssacc[par ^ 1], to_fixed(ssp));
+        __syncwarp();
+        if (lane == 0) a.ssq[(size_t)(par ^ 1) * H16 + c] = canon::slice_sumsq([&](int i) { return st->ztmp[i]; });
       }
       named_barrier_sync(CONS_BAR, nth);
       if (ok && l + 1 < L) {
         if (mbar_wait(wrtbar, (uint32_t)((l + 1) & 1), clock64() + WAIT_BUDGET_CYCLES)) {
-          unsigned long long *la = a.lacc + (size_t)(par ^ 1) * E;
-          for (int e = tid; e < E; e += nth) {
-            double p = 0.0;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) p = fma((double)wrtbuf[i * E + e], (double)st->ztmp[i], p);
-            atomicAdd(la + e, to_fixed(p));
-          }
+          unsigned long long *la = a.lacc + (size_t)(par ^ 1) * 2 * E;
+          bool rok = true;
+          for (int e = tid; e < E; e += nth)
+            rok &= add_fixed(la + e, la + E + e,
+                             canon::slice_dot([&](int i) { return wrtbuf[i * E + e]; },
+                                              [&](int i) { return st->ztmp[i]; }));
+          if (!rok) set_status(a.status, DEV_RANGE);
         } else {
           set_status(a.status, DEV_TIMEOUT);
           *(volatile int *)&st->abort = 1;
         }
       }
     }
-    cons_grid_barrier(a, st, tid);
+    cons_grid_barrier(a, st, tid, l, TP_DOWN_DONE);
   }
 
   if (producer) {
@@ -525,14 +570,15 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
   }
   if (*(volatile int *)&st->abort) return;
   // ---------------------------------------------------------------- output --
-  if (rows && tid < 16) {
-    const double ss = from_fixed(__ldcg(&a.ssacc[L & 1]));
-    const float inv = (float)(1.0 / sqrt(ss / (double)H + (double)a.eps));
-    a.x_out[r0 + tid] = __ldcg(a.zbuf + (size_t)(L & 1) * H + r0 + tid) * inv;
+  if (rows && warp == 0) {
+    const double *sq = a.ssq + (size_t)(L & 1) * H16;
+    const double ss = canon::warp_sumsq([&](int cc) { return __ldcg(sq + cc); }, H16);
+    const float inv = __double2float_rn(canon::norm_rinv(ss, H, a.eps));
+    if (lane < 16) a.x_out[r0 + lane] = __fmul_rn(__ldcg(a.zbuf + (size_t)(L & 1) * H + r0 + lane), inv);
   }
   // leave lacc[0] clear for the next launch's layer-0 partials (its last
   // reader finished long before the last barrier)
-  for (int e = c * nth + tid; e < E; e += G * nth) a.lacc[e] = 0ull;
+  for (int e = c * nth + tid; e < 2 * E; e += G * nth) a.lacc[e] = 0ull;
 }
 
 }  // namespace
@@ -541,25 +587,32 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
 // Can the fused kernel run this stack? Fills the launch plan when it can.
 bool fused_stack_plan(int fmt, int E, int H, int I, int k, FusedPlan *p) {
   if (k > SK_MAXK || E > 1024 || H / 16 > num_sms() || H % 128 || I % 128) return false;
+  // As many consumer warps taking ring items as possible (the ring depth a
+  // multiple of their number), then the deepest ring that fits.
   const int slot = (int)al128((size_t)tile_bytes(fmt, H));
   const size_t cap = max_smem_optin();
-  for (int S = 12; S >= 4; --S) {
-    const SkLayout o = sk_layout(fmt, E, H, I, k, S, slot);
-    if (o.total <= cap) {
+  int best_na = 0;
+  for (int S = 14; S >= 4; --S) {
+    const SkLayout o = sk_layout(fmt, E, H, I, k, S, slot, num_sms());
+    if (o.total > cap) continue;
+    int na = SK_NCW;
+    while (S % na) --na;
+    if (na > best_na) {
+      best_na = na;
       p->smem = o.total;
       p->nslots = S;
+      p->ncons = na;
       p->slot_bytes = slot;
-      return true;
     }
   }
-  return false;
+  return best_na > 0;
 }
 
 size_t fused_stack_ws_bytes(int L, int E, int H, int I, int k) {
   auto a = [](size_t v) { return (v + 255) & ~(size_t)255; };
   const size_t nb = (size_t)k * (I / 32);
-  return a((size_t)L * H * E * 4) + a(2 * (size_t)E * 8) + 256 + a(2 * (size_t)H * 4) + a(2 * (size_t)k * I * 4) +
-         a(nb * LIMB_REC) + a(nb * 8) + a(nb * 4) + 256 + 3 * a((size_t)L * 8);
+  return a((size_t)L * H * E * 4) + a(4 * (size_t)E * 8) + a(2 * (size_t)(H / 16) * 8) + a(2 * (size_t)H * 4) +
+         a(nb * LIMB_REC) + a(nb * 8) + 256 + 3 * a((size_t)L * 8);
 }
 
 
@@ -568,14 +621,12 @@ FusedBufs fused_carve(void *ws, int L, int E, int H, int I, int k) {
   char *p = static_cast<char *>(ws);
   FusedBufs b;
   b.wrt = reinterpret_cast<float *>(p); p += a((size_t)L * H * E * 4);
-  b.lacc = reinterpret_cast<unsigned long long *>(p); p += a(2 * (size_t)E * 8);
-  b.ssacc = reinterpret_cast<unsigned long long *>(p); p += 256;
+  b.lacc = reinterpret_cast<unsigned long long *>(p); p += a(4 * (size_t)E * 8);
+  b.ssq = reinterpret_cast<double *>(p); p += a(2 * (size_t)(H / 16) * 8);
   b.zbuf = reinterpret_cast<float *>(p); p += a(2 * (size_t)H * 4);
-  b.hbuf = reinterpret_cast<float *>(p); p += a(2 * (size_t)k * I * 4);
   const size_t nb = (size_t)k * (I / 32);
   b.lbuf = reinterpret_cast<uint8_t *>(p); p += a(nb * LIMB_REC);
   b.lscg = reinterpret_cast<float2 *>(p); p += a(nb * 8);
-  b.qcnt = reinterpret_cast<unsigned *>(p); p += a(nb * 4);
   b.bar = reinterpret_cast<unsigned *>(p); p += 256;
   b.gu = reinterpret_cast<const uint8_t **>(p); p += a((size_t)L * 8);
   b.dn = reinterpret_cast<const uint8_t **>(p); p += a((size_t)L * 8);
@@ -619,14 +670,15 @@ qmoe_status fused_prepare(const FusedBufs &b, int L, int E, int H, const float *
 
 qmoe_status fused_launch(const FusedBufs &b, const FusedPlan &p, int fmt, int L, int E, int H, int I, int k, float eps,
                          const float *x_in, float *x_out, int32_t *idx_rec, float *gate_rec, int32_t *status,
-                         cudaStream_t s, bool cooperative) {
+                         long long *trace, cudaStream_t s, bool cooperative) {
   StackArgs a{};
   a.L = L; a.E = E; a.H = H; a.I = I; a.k = k; a.eps = eps;
   a.gu = b.gu; a.dn = b.dn; a.bias = b.bias; a.wrt = b.wrt;
   a.x_in = x_in; a.x_out = x_out; a.idx_rec = idx_rec; a.gate_rec = gate_rec;
-  a.zbuf = b.zbuf; a.lacc = b.lacc; a.ssacc = b.ssacc; a.hbuf = b.hbuf; a.bar = b.bar; a.status = status;
-  a.lbuf = b.lbuf; a.lscg = b.lscg; a.qcnt = b.qcnt;
-  a.nslots = p.nslots; a.slot_bytes = p.slot_bytes;
+  a.zbuf = b.zbuf; a.lacc = b.lacc; a.ssq = b.ssq; a.bar = b.bar; a.status = status;
+  a.lbuf = b.lbuf; a.lscg = b.lscg;
+  a.trace = trace;
+  a.nslots = p.nslots; a.slot_bytes = p.slot_bytes; a.ncons = p.ncons;
   // Gate/up units are split evenly: the h barrier waits for the slowest CTA's
   // gate/up tiles, while the row owners' down tiles and router rows are only
   // needed after it and stream in behind the gate/up work.
@@ -652,4 +704,8 @@ qmoe_status fused_launch(const FusedBufs &b, const FusedPlan &p, int fmt, int L,
   return cuda_status(e);
 }
 
+}  // namespace qmoe
+
+namespace qmoe {
+int fused_trace_points() { return TRACE_POINTS; }
 }  // namespace qmoe

@@ -13,16 +13,17 @@ namespace qmoe {
 struct FusedPlan {
   size_t smem;
   int nslots, slot_bytes;
+  int ncons;   // consumer warps that take ring items (nslots is a multiple of it)
 };
 
 // Device buffers of the fused path, carved from the stack's workspace.
 struct FusedBufs {
   float *wrt;                      // [L][H][E] transposed routers
-  unsigned long long *lacc, *ssacc;
-  float *zbuf, *hbuf;
+  unsigned long long *lacc;         // [2][2][E] integer partial-logit sums
+  double *ssq;                     // [2][H/16] slice sums of squares
+  float *zbuf;
   uint8_t *lbuf;                   // limbs of h, [k][I/32][96]
   float2 *lscg;                    // block scales of h, [k][I/32]
-  unsigned *qcnt;                  // per-block tile counters, [k][I/32]
   unsigned *bar;
   const uint8_t **gu, **dn;
   const float **bias;
@@ -33,8 +34,12 @@ size_t fused_stack_ws_bytes(int L, int E, int H, int I, int k);
 FusedBufs fused_carve(void *ws, int L, int E, int H, int I, int k);
 qmoe_status fused_prepare(const FusedBufs &b, int L, int E, int H, const float *const *Wr,
                           const qmoe_experts *layers, const float *const *bias, cudaStream_t s);
+// trace: null, or [L][grid][fused_trace_points()] int64 SM-clock stamps per
+// layer and CTA (layer start, top-k done, gate/up tiles start and done, first
+// grid barrier passed, down tiles done, second grid barrier passed).
 qmoe_status fused_launch(const FusedBufs &b, const FusedPlan &p, int fmt, int L, int E, int H, int I, int k, float eps,
                          const float *x_in, float *x_out, int32_t *idx_rec, float *gate_rec, int32_t *status,
-                         cudaStream_t s, bool cooperative);
+                         long long *trace, cudaStream_t s, bool cooperative);
+int fused_trace_points();
 
 }  // namespace qmoe

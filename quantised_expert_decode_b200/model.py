@@ -86,6 +86,11 @@ class DecodeStack:
         """(route_ms, ffn_ms) per layer of the last completed replay (timing stacks)."""
         return L.qmoe_stack_layer_times(self.handle, self.L)
 
+    def phase_trace(self):
+        """Per-layer phase stamps of the last replay (fused timing stacks):
+        int64 SM cycles [L, CTAs, points]."""
+        return L.qmoe_stack_trace(self.handle, self.L)
+
     def status(self) -> int:
         return L.qmoe_read_status(self.dev_status)
 

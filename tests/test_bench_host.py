@@ -54,6 +54,16 @@ def test_clock_summary_median_max_and_reasons(tmp_path):
     assert s["reasons"] == ["hw_slowdown", "sw_power_cap"]
 
 
+def test_nvml_sample_summary_reasons_from_the_bitmask():
+    # bits: sw_power_cap 0x4, hw_slowdown 0x8, sw_thermal 0x20, hw_thermal 0x40; idle (0x1) is not a reason
+    s = bench.summarize_clock_samples([(1965.0, 0x0), (1950.0, 0x4), (1965.0, 0x1)], 1965.0)
+    assert s["sm_mhz"] == 1965.0 and s["sm_mhz_min"] == 1950.0 and s["samples"] == 3
+    assert s["reasons"] == ["sw_power_cap"]
+    s = bench.summarize_clock_samples([(1200.0, 0x8 | 0x40), (1965.0, 0x20)], 1965.0)
+    assert s["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"]
+    assert bench.summarize_clock_samples([], 1965.0)["sm_mhz"] is None
+
+
 def test_clock_summary_without_samples(tmp_path):
     s = _clock_summary(tmp_path, [])
     assert s["sm_mhz"] is None and s["reasons"] == ["nvidia-smi unavailable"]

@@ -61,3 +61,22 @@ def test_recombined_columns_equal_the_code_activation_product():
         d2, d1, d0 = (q * l2).sum(1), (q * l1).sum(1), (q * l0).sum(1)
         hi = (256 * d2 + d1) * 256
         assert np.array_equal(hi + d0, (q * X).sum(1)), bits
+
+
+def test_limb_pair_recombination_is_exact_for_4_bit_codes():
+    """The epilogue forms hi * 256 + lo as fma(f(hi), 256, f(lo)) from the two
+    block sums of a limb pair. For 4-bit codes each sum is at most
+    32 * 15 * 128 = 61,440 in magnitude: both convert exactly through the magic
+    number, f(hi) * 256 is exact, and the exact result stays below 2^24, so the
+    fused multiply-add's single rounding is no rounding at all."""
+    bound = 32 * 15 * 128
+    rs = np.random.default_rng(2)
+    hi = np.concatenate([[-bound, bound, 0, -1, 1], rs.integers(-bound, bound + 1, 100000)])
+    lo = np.concatenate([[bound, -bound, 0, 1, -1], rs.integers(-bound, bound + 1, 100000)])
+    exact = hi.astype(np.int64) * 256 + lo
+    assert np.abs(exact).max() < 2 ** 24
+    assert np.array_equal(i2f_small(hi).astype(np.int64), hi) and np.array_equal(i2f_small(lo).astype(np.int64), lo)
+    # fma in float32 of exactly representable operands whose exact result fits
+    # 24 bits: the float64 evaluation is the exact value, and it survives float32
+    fused = i2f_small(hi).astype(np.float64) * 256.0 + i2f_small(lo).astype(np.float64)
+    assert np.array_equal(fused.astype(np.float32).astype(np.int64), exact)

@@ -150,18 +150,22 @@ def _prefill(layer, x, idx, gate, k, check=True):
 
 
 def _oracle_rows(cfg, x64, idx, g, rows):
-    """Oracle outputs of the given token rows, one expert at a time (no cache)."""
+    """Oracle outputs of the given token rows on their given routes
+    (``moe.moe_layer``), each expert generated once and not kept."""
     Lyr = W.Layer(SEED, cfg, 0)
-    y = np.zeros((len(rows), cfg.H), dtype=np.float64)
-    experts = sorted(set(int(e) for r in rows for e in idx[r]))
-    for e in experts:
-        Wg, Wu, Wd = Lyr.expert(e)
-        for n, r in enumerate(rows):
-            for j in range(idx.shape[1]):
-                if idx[r, j] == e:
-                    y[n] += g[r, j] * moe.expert_ffn(x64[r:r + 1], Wg, Wu, Wd)[0]
+
+    def get(e):
+        w = Lyr.expert(e)
         Lyr.drop()
-    return y
+        return w
+    rows = np.asarray(rows)
+    return moe.moe_layer(x64[rows], idx[rows], g[rows], get)
+
+
+def _row_errors(y, ref):
+    """Relative error of every token row: ||y_t - ref_t|| / ||ref_t||."""
+    y = np.asarray(y, dtype=np.float64)
+    return np.sqrt(np.sum((y - ref) ** 2, axis=1)) / np.sqrt(np.sum(ref * ref, axis=1))
 
 
 SMALL = configs.get(4).with_(E=64, H=512, I=256, k=4, T=300)
@@ -186,8 +190,9 @@ def test_prefill_small_layer_matches_oracle(small_layer):
     y, _ = _prefill(layer, x, idx, gate, SMALL.k)
     idx_np, g_np = to_np(idx), to_np(gate).astype(np.float64)
     ref = W.run_layer(SEED, SMALL, x64)[0]
-    err = moe.rel_rms(to_np(y), ref)
-    assert err < PREFILL_TOL, err
+    # every token row on its own: one wrong row cannot hide in an average
+    errs = _row_errors(to_np(y), ref)
+    assert errs.max() < PREFILL_TOL, (int(errs.argmax()), errs.max())
     # the route itself is the oracle's
     oi, og, _ = moe.route(x64, gen.router(SEED, SMALL, 0), gen.bias(SEED, SMALL, 0), SMALL.k)
     assert np.array_equal(idx_np, oi)
@@ -209,8 +214,8 @@ def test_prefill_crafted_routes(small_layer, T):
     y, _ = _prefill(layer, x, torch.from_numpy(idx_np).cuda(), torch.from_numpy(g_np).cuda(), k)
     rows = list(range(T)) if T <= 17 else list(range(0, T, 37))
     ref = _oracle_rows(SMALL, x64, idx_np, g_np.astype(np.float64), rows)
-    err = moe.rel_rms(to_np(y)[rows], ref)
-    assert err < PREFILL_TOL, err
+    errs = _row_errors(to_np(y)[rows], ref)
+    assert errs.max() < PREFILL_TOL, (rows[int(errs.argmax())], errs.max())
 
 
 def test_prefill_zero_activation_and_bad_routes(small_layer):
@@ -229,9 +234,13 @@ def test_prefill_zero_activation_and_bad_routes(small_layer):
     assert q.qmoe_read_status(st) == 7
 
 
-def test_prefill_full_size_sampled_rows():
+def test_prefill_full_size_rows_of_the_heaviest_expert():
     """The 4096-token chunk through one 512-expert Q4 layer with the biased
-    router; the oracle checks a sample of rows one expert at a time."""
+    router. The oracle checks, row by row, every token routed to the most
+    loaded expert (its pairs span several 256-token chunks, so every chunk
+    boundary of the grouped GEMMs is crossed) and 256 further random tokens.
+    The routes fed to the oracle are the GPU's; the router's own parity is
+    checked bit for bit in test_prefill_router_matches_oracle_at_full_size."""
     cfg = configs.get(4)
     layers, routers, biases = device_layers(SEED, cfg, 1)
     x = device_tokens(SEED, cfg, 0)
@@ -241,8 +250,35 @@ def test_prefill_full_size_sampled_rows():
     counts = np.bincount(idx_np.ravel(), minlength=cfg.E)
     assert counts.max() > 512          # the skewed load spans several 256-token chunks
     x64 = W.x_float(SEED, cfg)
-    rows = [0, 1, 2, 1000, 2047, 3001, 4094, 4095]
+    heavy = int(counts.argmax())
+    rows = set(np.nonzero((idx_np == heavy).any(axis=1))[0].tolist())
+    rows |= set(np.random.default_rng(7).choice(cfg.T, size=256, replace=False).tolist())
+    rows = sorted(rows | {0, cfg.T - 1})
     ref = _oracle_rows(cfg, x64, idx_np, g_np, rows)
-    err = moe.rel_rms(to_np(y)[rows], ref)
-    assert err < PREFILL_TOL, err
+    errs = _row_errors(to_np(y)[rows], ref)
+    assert errs.max() < PREFILL_TOL, (rows[int(errs.argmax())], errs.max())
     assert np.isfinite(to_np(y)).all()
+
+
+def test_prefill_combine_is_reproducible_and_matches_the_atomic_form(small_layer):
+    """The slot-ordered combine gives the same bits on every run; the earlier
+    atomic combine (kept behind a flag of the timed entry point) agrees to fp32
+    rounding of the order of its additions."""
+    layer, Wr, bias = small_layer
+    x, x64 = _small_inputs(SMALL.T, step=1)
+    idx, gate = route(Wr, bias, x, SMALL.k, L.BF16)
+    y1, _ = _prefill(layer, x, idx, gate, SMALL.k)
+    y2, _ = _prefill(layer, x, idx, gate, SMALL.k)
+    assert torch.equal(y1, y2)
+    T, k = SMALL.T, SMALL.k
+    ya = torch.full((T, layer.H), float("nan"), dtype=torch.float32, device="cuda")
+    ws = torch.empty(q.qmoe_prefill_workspace_bytes(T, k, layer.E, layer.H, layer.I), dtype=torch.uint8,
+                     device="cuda")
+    st = status_word()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    q.qmoe_ffn_prefill_timed(layer.handle(), x, T, idx, gate, k, ya, ws, st, ev, flags=L.PREFILL_ATOMIC_COMBINE)
+    torch.cuda.synchronize()
+    assert q.qmoe_read_status(st) == 0
+    assert moe.rel_rms(to_np(ya), to_np(y1)) < 1e-6
+    ref = W.run_layer(SEED, SMALL, x64)[0]
+    assert _row_errors(to_np(y1), ref).max() < PREFILL_TOL

@@ -1,11 +1,13 @@
 """GPU parity of the captured layer stack (route -> FFN -> residual RMSNorm per
-layer, one CUDA graph) against the float64 oracle run free from the same x_0."""
+layer, one CUDA graph) against the float64 oracle run free from the same x_0,
+and bit-for-bit agreement between the decode paths."""
 import numpy as np
 import pytest
 import torch
 
 from oracle import moe
 from oracle import workload as W
+from quantised_expert_decode_b200 import _lib as L
 from quantised_expert_decode_b200.model import DecodeStack
 from synth import configs, gen
 from synth.workload import device_layers
@@ -15,14 +17,34 @@ pytestmark = pytest.mark.gpu
 SEED = 0
 
 
-# Beyond the first layer the GPU and the oracle route slightly different
-# activations (fp32 vs float64 arithmetic, 16-bit activation limbs), so two
-# logits closer than this may legitimately order differently. A differing
-# expert SET is accepted only as a reported near-tie below this gap.
-NEAR_TIE = 1e-4
+def _flip_bound(cfg, built, x0, l, layerwise, x_oracle):
+    """Certified bound on how far a GPU logit of layer l can sit from the
+    oracle's own logit, from the actual input difference of that layer.
+
+    The GPU's input to layer l is the output of the first l layers (a stack of
+    l layers from the same x_0). A logit moves by at most
+    ||Wr_e||_2 * ||x_gpu - x_oracle||_2 when its input moves, plus the GPU's own
+    rounding of the normalised activations (2^-23 of sum_h |Wr_eh x_h|); two
+    logits can swap only if their oracle gap is below twice that."""
+    layers, routers, biases = built
+    if l == 0:
+        x_gpu = x0.astype(np.float64)
+    else:
+        part = DecodeStack(layers[:l], routers[:l], None if biases is None else biases[:l], cfg.T, cfg.k, cfg.eps,
+                           layerwise=layerwise)
+        part.x_in.copy_(torch.from_numpy(x0))
+        part.decode()
+        torch.cuda.synchronize()
+        x_gpu = to_np(part.x_out).astype(np.float64)
+        part.close()
+    Wr = gen.router(SEED, cfg, l).astype(np.float64)
+    delta = np.sqrt(np.sum((x_gpu - x_oracle) ** 2, axis=1))                     # per token
+    rows = np.sqrt(np.sum(Wr * Wr, axis=1)).max()
+    rnd = 2.0 ** -23 * (np.abs(x_gpu) @ np.abs(Wr).T).max(axis=1)
+    return 2.0 * (rows * delta + rnd)
 
 
-def _compare(cfg, stack, x0_np, n_layers):
+def _compare(cfg, stack, x0_np, n_layers, built, layerwise=False):
     xo, recs = W.run_stack(SEED, cfg, x0_np.astype(np.float64), n_layers)
     idx = to_np(stack.idx)
     gate = to_np(stack.gate)
@@ -30,41 +52,42 @@ def _compare(cfg, stack, x0_np, n_layers):
         if np.array_equal(idx[l], oi):
             assert np.max(np.abs(gate[l] - og)) < 50 * GATE_TOL, l
             continue
+        # A differing route is accepted only where the oracle's own top-k gap
+        # lies below the bound derived from this layer's input difference;
+        # the layers after it then follow another route, so the run stops here.
         L_ = W.Layer(SEED, cfg, l)
         lg = moe.logits(x_in, L_.Wr, L_.bias, cfg.k)
+        bound = _flip_bound(cfg, built, x0_np, l, layerwise, x_in)
         for t in range(cfg.T):
-            if set(idx[l, t].tolist()) != set(oi[t].tolist()):
-                gap = gap_report(lg[t], cfg.k)
-                if gap < NEAR_TIE:
-                    pytest.xfail(f"layer {l} token {t}: near-tie route flip, oracle top-k gap {gap:.3g}")
-                pytest.fail(f"layer {l} token {t}: expert sets differ; oracle top-k gap {gap:.3g}")
-            for a, b in zip(idx[l, t], oi[t]):
-                if a != b:
-                    assert abs(lg[t, a] - lg[t, b]) < NEAR_TIE, (l, t, a, b)
-            gm = dict(zip(idx[l, t].tolist(), gate[l, t].tolist()))
-            for e, gv in zip(oi[t].tolist(), og[t].tolist()):
-                assert abs(gm[e] - gv) < 50 * GATE_TOL, (l, t, e)
+            if np.array_equal(idx[l, t], oi[t]):
+                continue
+            gap = gap_report(lg[t], cfg.k)
+            if gap >= bound[t]:
+                pytest.fail(f"layer {l} token {t}: routes differ; oracle top-k gap {gap:.3g} "
+                            f">= certified bound {bound[t]:.3g}")
+        pytest.xfail(f"layer {l}: near-tie route flip within the certified input bound {bound.max():.3g}")
     err = moe.rel_rms(to_np(stack.x_out), xo)
     assert err < DECODE_TOL, err
     return err
 
 
-def _run(cfg, n_layers, step=0, layerwise=False, built=None):
-    layers, routers, biases = built if built else device_layers(SEED, cfg, n_layers)
+def _run(cfg, n_layers, step=0, layerwise=False, built=None, scale=1.0):
+    built = built if built else device_layers(SEED, cfg, n_layers)
+    layers, routers, biases = built
     stack = DecodeStack(layers, routers, biases, cfg.T, cfg.k, cfg.eps, layerwise=layerwise)
-    x0 = gen.tokens(SEED, cfg, step)
+    x0 = (gen.tokens(SEED, cfg, step) * np.float32(scale)).astype(np.float32)
     stack.x_in.copy_(torch.from_numpy(x0))
     stack.decode()
     torch.cuda.synchronize()
     assert stack.status() == 0
-    return stack, x0, layers
+    return stack, x0, built
 
 
 @pytest.mark.parametrize("layerwise", [False, True])
 def test_stack_small_geometry(layerwise):
     cfg = configs.get(0).with_(L=6, residual=True)
-    stack, x0, _ = _run(cfg, 6, layerwise=layerwise)
-    _compare(cfg, stack, x0, 6)
+    stack, x0, built = _run(cfg, 6, layerwise=layerwise)
+    _compare(cfg, stack, x0, 6, built, layerwise)
     assert stack.path == (0 if layerwise else 1)
     assert stack.kernels_per_replay == (13 if layerwise else 1)
     # host-buffer entry point gives the same answer as the device-buffer replay
@@ -77,11 +100,19 @@ def test_stack_small_geometry(layerwise):
     stack.close()
 
 
+def _same_bits(a, b):
+    assert a.path != b.path
+    assert torch.equal(a.idx, b.idx)
+    assert torch.equal(a.gate, b.gate)
+    assert torch.equal(a.x_out, b.x_out)
+
+
 def test_stack_48_layers_q2_single_token():
     cfg = configs.get(2)
-    stack, x0, layers = _run(cfg, cfg.L)
+    stack, x0, built = _run(cfg, cfg.L)
+    layers = built[0]
     assert sum(l.nbytes for l in layers) == cfg.L * cfg.E * cfg.expert_bytes()
-    _compare(cfg, stack, x0, cfg.L)
+    _compare(cfg, stack, x0, cfg.L, built)
     # replays are deterministic
     first = stack.x_out.clone()
     stack.decode()
@@ -92,38 +123,54 @@ def test_stack_48_layers_q2_single_token():
     stack.x_in.copy_(torch.from_numpy(x1))
     stack.decode()
     torch.cuda.synchronize()
-    _compare(cfg, stack, x1, cfg.L)
-    # the per-layer kernel path routes identically and agrees to fp32 roundoff
+    _compare(cfg, stack, x1, cfg.L, built)
+    # the per-layer kernel path gives the same bits as the fused kernel
     lw = DecodeStack(layers, stack.routers, None, cfg.T, cfg.k, cfg.eps, layerwise=True)
     lw.x_in.copy_(torch.from_numpy(x1))
     lw.decode()
     torch.cuda.synchronize()
-    assert stack.path == 1 and lw.path == 0
-    assert torch.equal(lw.idx, stack.idx)
-    assert moe.rel_rms(to_np(lw.x_out), to_np(stack.x_out)) < 1e-5
+    assert stack.path == L.PATH_FUSED and lw.path == L.PATH_LAYERWISE
+    _same_bits(stack, lw)
     lw.close()
     stack.close()
 
 
+@pytest.mark.parametrize("scale", [1e3, 1e-4])
+def test_stack_input_scale(scale):
+    """x_0 scaled far from unit RMS (the first layer sees it raw): both paths
+    match the oracle and each other bit for bit."""
+    cfg = configs.get(2).with_(L=4)
+    built = device_layers(SEED, cfg, 4)
+    fused, x0, _ = _run(cfg, 4, built=built, scale=scale)
+    assert fused.path == L.PATH_FUSED
+    _compare(cfg, fused, x0, 4, built)
+    lw, _, _ = _run(cfg, 4, built=built, scale=scale, layerwise=True)
+    _same_bits(fused, lw)
+    fused.close()
+    lw.close()
+
+
 def test_stack_48_layers_q4_verify_batch():
     cfg = configs.get(3)
-    stack, x0, _ = _run(cfg, cfg.L)
-    _compare(cfg, stack, x0, cfg.L)
+    stack, x0, built = _run(cfg, cfg.L)
+    _compare(cfg, stack, x0, cfg.L, built, layerwise=True)
     stack.close()
 
 
 def test_verify_batch_equals_single_token_decoding_bit_for_bit():
-    """A verify batch (8 correlated tokens, Q4 experts, per-layer path) reproduces
-    every token decoded alone through the same per-layer path bit for bit:
-    routes, gates and the final activations. A token's arithmetic (exact
-    integer block sums, then one fixed floating-point order) does not depend on
-    which other tokens of the batch share its experts."""
+    """A verify batch (8 correlated tokens, Q4 experts) reproduces every token
+    decoded alone bit for bit - routes, gates and the final activations -
+    against both single-token paths: the default one (the fused kernel) and
+    the per-layer kernels. A token's arithmetic (exact integer block sums and
+    router partials, then one fixed floating-point order) does not depend on
+    which other tokens of the batch share its experts, nor on the path."""
     cfg = configs.get(3)
     n_layers = 8
     layers, routers, biases = device_layers(SEED, cfg, n_layers)
-    batch = DecodeStack(layers, routers, biases, cfg.T, cfg.k, cfg.eps, layerwise=True)
-    one = DecodeStack(layers, routers, biases, 1, cfg.k, cfg.eps, layerwise=True)
-    assert batch.path == 0 and one.path == 0
+    batch = DecodeStack(layers, routers, biases, cfg.T, cfg.k, cfg.eps)
+    one = DecodeStack(layers, routers, biases, 1, cfg.k, cfg.eps)
+    one_lw = DecodeStack(layers, routers, biases, 1, cfg.k, cfg.eps, layerwise=True)
+    assert batch.path == L.PATH_LAYERWISE and one.path == L.PATH_FUSED and one_lw.path == L.PATH_LAYERWISE
     x0 = torch.from_numpy(gen.tokens(SEED, cfg, 0)).cuda()
     batch.x_in.copy_(x0)
     batch.decode()
@@ -133,12 +180,40 @@ def test_verify_batch_equals_single_token_decoding_bit_for_bit():
     idx = to_np(batch.idx)
     assert min(len(np.unique(idx[l])) for l in range(n_layers)) < cfg.T * cfg.k
     for t in range(cfg.T):
-        one.x_in.copy_(x0[t:t + 1])
-        one.decode()
-        torch.cuda.synchronize()
-        assert one.status() == 0
-        assert torch.equal(one.idx[:, 0], batch.idx[:, t]), t
-        assert torch.equal(one.gate[:, 0], batch.gate[:, t]), t
-        assert torch.equal(one.x_out[0], batch.x_out[t]), t
+        for s in (one, one_lw):
+            s.x_in.copy_(x0[t:t + 1])
+            s.decode()
+            torch.cuda.synchronize()
+            assert s.status() == 0
+            assert torch.equal(s.idx[:, 0], batch.idx[:, t]), (t, s.path)
+            assert torch.equal(s.gate[:, 0], batch.gate[:, t]), (t, s.path)
+            assert torch.equal(s.x_out[0], batch.x_out[t]), (t, s.path)
     one.close()
+    one_lw.close()
     batch.close()
+
+
+def test_fused_phase_trace_is_ordered_and_layer_times_add_up():
+    """The fused kernel's phase stamps come in program order in every CTA and
+    layer, and the per-layer times derived from them add up to the kernel's
+    event-timed duration."""
+    cfg = configs.get(0).with_(L=4, residual=True)
+    layers, routers, _ = device_layers(SEED, cfg, 4)
+    st = DecodeStack(layers, routers, None, 1, cfg.k, cfg.eps, timing=True)
+    assert st.path == L.PATH_FUSED
+    st.x_in.copy_(torch.from_numpy(gen.tokens(SEED, cfg, 0)))
+    st.decode()
+    torch.cuda.synchronize()
+    assert st.status() == 0
+    tr = st.phase_trace()
+    assert tr.shape[0] == 4 and tr.shape[2] == 8
+    assert (np.diff(tr[:, :, :7], axis=2) >= 0).all()
+    route_ms, ffn_ms = st.layer_times()
+    assert all(r >= 0 for r in route_ms) and all(f > 0 for f in ffn_ms)
+    plain = DecodeStack(layers, routers, None, 1, cfg.k, cfg.eps)
+    plain.x_in.copy_(st.x_in)
+    plain.decode()
+    torch.cuda.synchronize()
+    assert torch.equal(plain.x_out, st.x_out)     # stamping changes no result
+    plain.close()
+    st.close()
