@@ -484,9 +484,10 @@ def measure_stack(args, cfg, seed=SEED, full=True):
         # start, averaged over the layers of the last replay (in microseconds
         # at the sampled SM clock)
         tr = tstack.phase_trace().astype(np.float64)                     # [L, CTAs, points]
-        rel = np.median(tr[:, :, 1:7] - tr[:, :, :1], axis=1).mean(axis=0)
+        rel = np.median(tr[:, :, 1:8] - tr[:, :, :1], axis=1).mean(axis=0)
         mhz = clk.get("sm_mhz") or clk.get("sm_max_mhz") or 1965.0
-        names = ["topk_done", "tiles_start", "tiles_done", "barrier1_passed", "down_done", "barrier2_passed"]
+        names = ["topk_done", "tiles_start", "tiles_done", "barrier1_passed", "down_done", "barrier2_passed",
+                 "logits_ready"]
         phases = {n: float(v) / mhz for n, v in zip(names, rel)}
     tstack.close()
     del layers, routers, biases, xs
@@ -501,7 +502,7 @@ def measure_stack(args, cfg, seed=SEED, full=True):
         # one persistent kernel per token: it streams every expert and router byte
         kernel = "stack_decode_kernel (fused decode stack, one launch per token)"
         launch_bytes = float(expert_bytes_step + router_bytes_step)
-        launch_s = float(ffn_ms.sum()) / 1e3
+        launch_s = float(route_ms.sum() + ffn_ms.sum()) / 1e3       # the whole kernel
         achieved = launch_bytes / launch_s / 1e9
     else:
         kernel = "ffn_decode_kernel (one launch per layer)"
@@ -587,7 +588,7 @@ def run_layer(args, cfg):
         # read then evicts the dirty lines the write left, so their write-back
         # to HBM happens here and not inside the timed kernels
         flush.fill_(i & 255)
-        torch.sum(flush_rd, out=flush_sink)
+        torch.sum(flush_rd, dim=0, keepdim=True, out=flush_sink)
         if e:
             e[0].record(stream)
         q.qmoe_route(Wr, None, xs[i], q.F32, T, cfg.H, cfg.E, cfg.k, idx, gate, rws, st, stream)

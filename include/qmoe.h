@@ -55,7 +55,7 @@ typedef enum {
   QMOE_ERR_TIMEOUT = 6,       /* a device-side wait exceeded its budget */
   QMOE_ERR_DEVICE_STATUS = 7, /* invalid routed index seen on the device */
   QMOE_ERR_RANGE = 8          /* decode activations too large for the exact router sums:
-                                 a 16-element slice's partial logit reached 2^33 */
+                                 a 16-element slice's partial logit reached 2^31 */
 } qmoe_status;
 
 enum { QMOE_Q2 = 2, QMOE_Q4 = 4 };        /* block formats (bits per code) */
@@ -318,8 +318,8 @@ qmoe_status qmoe_stack_layer_times(const qmoe_stack *stack, float *route_ms, flo
  * stack: SM clock cycles (clock64 of each CTA's first consumer thread, so
  * compare only stamps of one CTA), int64 [L][*ctas][*points]: layer start,
  * top-k done, gate/up tiles start, gate/up tiles done, first grid barrier
- * passed, down tiles and router partials done, second grid barrier passed
- * (slot 7 unused). count is the capacity of cycles_host in entries (WORKSPACE
+ * passed, down tiles and router partials done, second grid barrier passed,
+ * logits and normalised x ready (recorded between the first and second). count is the capacity of cycles_host in entries (WORKSPACE
  * if too small). UNSUPPORTED on the per-layer path or without the flag.
  * Synchronises the device. */
 qmoe_status qmoe_stack_trace(const qmoe_stack *stack, int64_t *cycles_host, size_t count, int *ctas, int *points);

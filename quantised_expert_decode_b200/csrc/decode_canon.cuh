@@ -11,9 +11,10 @@
 //   partials   a slice's router partial sum_i Wr[e][16c+i] z[16c+i] and its
 //              sum of squares sum_i z[16c+i]^2 are float64 fma chains in
 //              element order i = 0..15;
-//   logits     each router partial is split into two integers (hi at 2^-20,
-//              lo at 2^-60); integers add exactly in any order, so a row summed
-//              by one warp and a row summed over 128 CTAs with atomics agree;
+//   logits     each router partial is split into two integers (hi in units
+//              of 2^-20, lo in units of 2^-60); integers add exactly in any
+//              order, so a row summed by one warp and a row summed over 128
+//              CTAs with atomics agree;
 //   squares    the slice sums of squares are added in one fixed order: lane l
 //              of a warp adds slices l, l + 32, l + 64, ... in turn, then the
 //              32 lane sums meet in a butterfly (xor 16, 8, 4, 2, 1); the fused
@@ -25,7 +26,7 @@
 //   combine    y = sum_j gate_j * r_j in slot order, one rounding per multiply
 //              and per add; z_next = x + y.
 //
-// A router partial of magnitude 2^33 or more (or NaN) cannot be split exactly;
+// A router partial of magnitude 2^31 or more (or NaN) cannot be split exactly;
 // it is reported through the device status (DEV_RANGE) instead.
 #pragma once
 
@@ -38,32 +39,52 @@ namespace canon {
 namespace {
 
 constexpr int SLICE = 16;
-constexpr double FIX_HI = 1048576.0;                        // 2^20
 constexpr double FIX_HI_INV = 1.0 / 1048576.0;              // 2^-20
 constexpr double FIX_LO = 1152921504606846976.0;            // 2^60
 constexpr double FIX_LO_INV = 1.0 / 1152921504606846976.0;  // 2^-60
-constexpr double FIX_RANGE = 8589934592.0;                  // 2^33
+constexpr double FIX_RANGE = 2147483648.0;                  // 2^31
+constexpr double MAGIC_HI = 6442450944.0;                   // 1.5 * 2^32: its ulp is 2^-20
+constexpr double MAGIC_LO = 6755399441055744.0;             // 1.5 * 2^52: its ulp is 1
 
-// p -> (hi, lo) with p = hi 2^-20 + lo 2^-60 up to the rounding of lo.
-// hi 2^-20 is the multiple of 2^-20 nearest p; the remainder r is a multiple
-// of min(ulp(p), 2^-20) below 2^-21 in magnitude, so p - hi 2^-20 is exact.
-// Returns false (and zeros) when |p| >= 2^33 or p is NaN.
+// p -> (hi, lo) with p = hi 2^-20 + lo 2^-60 up to the rounding of lo, in
+// float64 adds and integer subtractions only (no conversion instruction):
+//   t = p + 1.5 * 2^32 rounds p to the nearest multiple of 2^-20 (the ulp of
+//     t, which stays in [2^32, 2^33) for |p| < 2^31), and the integer hi sits
+//     in t's low mantissa bits: hi = bits(t) - bits(1.5 * 2^32);
+//   r = p - (t - 1.5 * 2^32) is exact (a multiple of min(ulp(p), 2^-20) below
+//     2^-21 in magnitude);
+//   u = r * 2^60 + 1.5 * 2^52 rounds r * 2^60 (exact, below 2^39) to an
+//     integer, lo = bits(u) - bits(1.5 * 2^52).
+// Both roundings are to nearest, ties to even. Returns false (and zeros) when
+// |p| >= 2^31 or p is NaN.
 __device__ __forceinline__ bool split(double p, long long &hi, long long &lo) {
   if (!(fabs(p) < FIX_RANGE)) {
     hi = 0;
     lo = 0;
     return false;
   }
-  hi = __double2ll_rn(__dmul_rn(p, FIX_HI));
-  const double r = __dsub_rn(p, __dmul_rn((double)hi, FIX_HI_INV));
-  lo = __double2ll_rn(__dmul_rn(r, FIX_LO));
+  const double t = __dadd_rn(p, MAGIC_HI);
+  const double r = __dsub_rn(p, __dsub_rn(t, MAGIC_HI));
+  const double u = __fma_rn(r, FIX_LO, MAGIC_LO);
+  hi = __double_as_longlong(t) - __double_as_longlong(MAGIC_HI);
+  lo = __double_as_longlong(u) - __double_as_longlong(MAGIC_LO);
   return true;
 }
 
+// int64 -> float64 without a conversion instruction: each 32-bit half goes
+// through the 2^52 magic number (exact), then hi * 2^32 + lo, exact below 2^53
+// and rounded once (to nearest) above.
+__device__ __forceinline__ double i64_to_f64(long long v) {
+  const double h = __dsub_rn(__hiloint2double(0x43300000, (int)(((unsigned long long)v >> 32) ^ 0x80000000u)),
+                             4503601774854144.0);          // 2^52 + 2^31
+  const double l = __dsub_rn(__hiloint2double(0x43300000, (int)(unsigned)v), 4503599627370496.0);   // 2^52
+  return __fma_rn(h, 4294967296.0, l);
+}
+
 // Exact integer totals -> float64 (two exact scalings, one rounding in the add;
-// (double)HI is exact below 2^53).
+// each total is exact in float64 below 2^53).
 __device__ __forceinline__ double join(long long hi, long long lo) {
-  return __dadd_rn(__dmul_rn((double)hi, FIX_HI_INV), __dmul_rn((double)lo, FIX_LO_INV));
+  return __dadd_rn(__dmul_rn(i64_to_f64(hi), FIX_HI_INV), __dmul_rn(i64_to_f64(lo), FIX_LO_INV));
 }
 
 // Router partial of one slice: w(i), z(i) for i = 0..15.

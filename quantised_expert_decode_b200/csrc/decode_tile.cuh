@@ -159,42 +159,63 @@ __device__ __noinline__ Acc tile_dot(const uint8_t *tile, int nblk, const uint8_
       w[0] = q0.x; w[1] = q0.y; w[2] = q0.z; w[3] = q0.w;
       w[4] = q1.x; w[5] = q1.y; w[6] = q1.z; w[7] = q1.w;
     }
+    // all MMAs of the chunk first, into separate accumulators, then their
+    // epilogues in the same (sb, q) order as before: the MMA latency overlaps
+    // (a warp keeps NSET x NQ x BS of them in flight instead of one) and the
+    // floating-point order of the results is unchanged
+    uint32_t bq[NSET][NQ][2];
 #pragma unroll
-    for (int sb = 0; sb < NSET; ++sb) {
+    for (int sb = 0; sb < NSET; ++sb)
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
-        uint32_t b0 = 0u, b1 = 0u;
-        if (pv[q] >= 0) {
-          const int blk = c * 4 + sb * BS + pbeta;
-          const uint8_t *lp = limbs + ((size_t)pv[q] * nblk + blk) * LIMB_REC + ploff + 4 * t;
-          b0 = *reinterpret_cast<const uint32_t *>(lp);
-          b1 = *reinterpret_cast<const uint32_t *>(lp + 16);
-        }
-        int d0 = 0, d1 = 0, d2 = 0, d3 = 0;
+        // lanes without a token (or on the zero limb column) read vector 0's
+        // record, in bounds, and pass zeros
+        const int blk = c * 4 + sb * BS + pbeta;
+        const int pvs = pv[q] >= 0 ? pv[q] : vid[0];
+        const uint8_t *lp = limbs + ((size_t)pvs * nblk + blk) * LIMB_REC + ploff + 4 * t;
+        const uint32_t x0 = *reinterpret_cast<const uint32_t *>(lp);
+        const uint32_t x1 = *reinterpret_cast<const uint32_t *>(lp + 16);
+        bq[sb][q][0] = pv[q] >= 0 ? x0 : 0u;
+        bq[sb][q][1] = pv[q] >= 0 ? x1 : 0u;
+      }
+    int D[NSET][NQ][4];
 #pragma unroll
-        for (int beta = 0; beta < BS; ++beta) {
-          const int bb = sb * BS + beta;
-          uint32_t a0, a1, a2, a3;
-          if (BITS == 2) {
-            const uint32_t x = w[bb];
-            a0 = x & 0x03030303u;
-            a1 = (x >> 2) & 0x03030303u;
-            a2 = (x >> 4) & 0x03030303u;
-            a3 = (x >> 6) & 0x03030303u;
-          } else {
-            const uint32_t x0 = w[2 * bb], x1 = w[2 * bb + 1];
-            a0 = x0 & 0x0F0F0F0Fu;
-            a1 = (x0 >> 4) & 0x0F0F0F0Fu;
-            a2 = x1 & 0x0F0F0F0Fu;
-            a3 = (x1 >> 4) & 0x0F0F0F0Fu;
-          }
-          const bool on = (pbeta == beta);
-          mma_u8s8(d0, d1, d2, d3, a0, a1, a2, a3, on ? b0 : 0u, on ? b1 : 0u);
+    for (int sb = 0; sb < NSET; ++sb)
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) D[sb][q][0] = D[sb][q][1] = D[sb][q][2] = D[sb][q][3] = 0;
+#pragma unroll
+    for (int beta = 0; beta < BS; ++beta)
+#pragma unroll
+      for (int sb = 0; sb < NSET; ++sb) {
+        const int bb = sb * BS + beta;
+        uint32_t a0, a1, a2, a3;
+        if (BITS == 2) {
+          const uint32_t x = w[bb];
+          a0 = x & 0x03030303u;
+          a1 = (x >> 2) & 0x03030303u;
+          a2 = (x >> 4) & 0x03030303u;
+          a3 = (x >> 6) & 0x03030303u;
+        } else {
+          const uint32_t x0 = w[2 * bb], x1 = w[2 * bb + 1];
+          a0 = x0 & 0x0F0F0F0Fu;
+          a1 = (x0 >> 4) & 0x0F0F0F0Fu;
+          a2 = x1 & 0x0F0F0F0Fu;
+          a3 = (x1 >> 4) & 0x0F0F0F0Fu;
         }
+        const bool on = (pbeta == beta);
+#pragma unroll
+        for (int q = 0; q < NQ; ++q)
+          mma_u8s8(D[sb][q][0], D[sb][q][1], D[sb][q][2], D[sb][q][3], a0, a1, a2, a3, on ? bq[sb][q][0] : 0u,
+                   on ? bq[sb][q][1] : 0u);
+      }
+#pragma unroll
+    for (int sb = 0; sb < NSET; ++sb)
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
         if (ov[q] >= 0) {
           const int bo = c * 4 + sb * BS + obeta;
-          const float v0 = limb_pair(d0, d1);
-          const float v1 = limb_pair(d2, d3);
+          const float v0 = limb_pair(D[sb][q][0], D[sb][q][1]);
+          const float v1 = limb_pair(D[sb][q][2], D[sb][q][3]);
           const float2 ss = lsc[(size_t)ov[q] * nblk + bo];
           const uint2 dm = *reinterpret_cast<const uint2 *>(sbase + (bo * 8 + g) * 8);
           const float sw = ss.x * wgt;
@@ -208,7 +229,6 @@ __device__ __noinline__ Acc tile_dot(const uint8_t *tile, int nblk, const uint8_
           }
         }
       }
-    }
   }
   // combine the lanes that share a token: the two halves of a pair, then even
   // + odd blocks (for NP == 1 the other pair of lanes, else acc_odd)

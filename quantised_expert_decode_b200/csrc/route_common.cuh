@@ -2,10 +2,12 @@
 // logits (used by the decode and prefill routers).
 //
 // Selection order: logit descending, expert index ascending on equal logits.
-// 1. Every logit gets an fp32 key (round-to-nearest of the float64 value, -0
-//    taken as +0, made order-preserving as an unsigned integer). Rounding is
-//    monotone and equal logits get equal keys, so the k largest float64
-//    logits are among the k largest keys, counted with multiplicity.
+// 1. Every logit gets a 32-bit key: the top half of the float64 value's bits
+//    made order-preserving as an unsigned integer (-0 taken as +0). Dropping
+//    the low bits is monotone and equal logits get equal keys, so the k
+//    largest float64 logits are among the k largest keys, counted with
+//    multiplicity. (Integer operations only: a float64 -> float32 rounding
+//    would issue on the conversion unit, which runs at a fraction of the rate.)
 // 2. Threshold: the k-th largest of the 32 per-lane maximum keys (ties by
 //    lane). At least k keys (those lane maxima) are >= it, so it is at most
 //    the k-th largest key and every key >= threshold is a candidate: a
@@ -29,6 +31,12 @@ struct TopkScratch {
   int sel_e[TOPK_MAX_K];
   double sel_v[TOPK_MAX_K];
 };
+
+__device__ __forceinline__ unsigned double_key(double v) {
+  const long long b = __double_as_longlong(v == 0.0 ? 0.0 : v);
+  const unsigned long long o = b < 0 ? ~(unsigned long long)b : ((unsigned long long)b | 0x8000000000000000ull);
+  return (unsigned)(o >> 32);
+}
 
 __device__ __forceinline__ bool ranks_above(double va, int ea, double vb, int eb) {
   return va > vb || (va == vb && ea < eb);
@@ -56,8 +64,7 @@ __device__ inline void warp_topk_gates_m(Get get, int E, int k, int32_t *idx_out
   for (int j = 0; j < M; ++j) {
     const int e = lane + 32 * j;
     // -0 and +0 are equal logits (ranked by index), so they share one key
-    const float f = __double2float_rn(val[j]);
-    key[j] = e < E ? float_key(f == 0.0f ? 0.0f : f) : 0u;
+    key[j] = e < E ? double_key(val[j]) : 0u;
   }
   unsigned lmax = 0;
 #pragma unroll
@@ -84,7 +91,35 @@ __device__ inline void warp_topk_gates_m(Get get, int E, int k, int32_t *idx_out
     if (lane >= o) incl += v;
   }
   const int total = __shfl_sync(0xffffffffu, incl, 31);
-  if (total <= TOPK_CAND) {
+  if (total <= 32) {
+    // one candidate per lane (in lane order of the keys), ranked against the
+    // others through shuffles
+    int pos = incl - mine, ce = 0;
+    double cv = 0.0;
+#pragma unroll
+    for (int j = 0; j < M; ++j)
+      if (key[j] != 0u && key[j] >= thr) {
+        sc->cand[pos] = lane + 32 * j;
+        sc->cand_v[pos] = val[j];
+        ++pos;
+      }
+    __syncwarp();
+    if (lane < total) {
+      ce = sc->cand[lane];
+      cv = sc->cand_v[lane];
+    }
+    int rank = 0;
+#pragma unroll
+    for (int i2 = 0; i2 < 32; ++i2) {   // all 32 shuffles independent; lanes past `total` hold no candidate
+      const double v2 = __shfl_sync(0xffffffffu, cv, i2);
+      const int e2 = __shfl_sync(0xffffffffu, ce, i2);
+      rank += (i2 < total && ranks_above(v2, e2, cv, ce)) ? 1 : 0;
+    }
+    if (lane < total && rank < k) {
+      sc->sel_e[rank] = ce;
+      sc->sel_v[rank] = cv;
+    }
+  } else if (total <= TOPK_CAND) {
     int pos = incl - mine;
 #pragma unroll
     for (int j = 0; j < M; ++j)

@@ -42,15 +42,20 @@ namespace qmoe {
 namespace {
 using namespace tile;
 
-constexpr int SK_NCW = 7;  // consumer warps; with the producer 256 threads, so up to 255 registers
+// Consumer warps. With the producer, 12 warps: three per SM sub-partition, so
+// up to 168 registers a thread. The legacy integer MMA issues at a fraction of
+// the tcgen05 rate and one warp keeps only a couple in flight, so the tile
+// dot products want warps more than registers: with 11 consumers a CTA's 8
+// gate/up tiles and 10 down tiles each get a warp of their own.
+constexpr int SK_NCW = 11;
 constexpr int SK_THREADS = 32 * (SK_NCW + 1);
 constexpr int SK_MAXK = 16;
 constexpr int TRACE_POINTS = 8;
 // Trace points of a layer (SM clock of the CTA's consumer thread 0): layer
 // start; top-k done; gate/up tiles start; gate/up tiles done (all consumer
 // warps); first grid barrier passed; down tiles and partials done; second
-// grid barrier passed.
-enum { TP_START = 0, TP_TOPK, TP_TILES, TP_TILES_DONE, TP_BAR1, TP_DOWN_DONE, TP_BAR2 };
+// grid barrier passed; logits and normalised x ready (before the top-k).
+enum { TP_START = 0, TP_TOPK, TP_TILES, TP_TILES_DONE, TP_BAR1, TP_DOWN_DONE, TP_BAR2, TP_LOGITS };
 constexpr int CONS_BAR = 1;   // the consumer warps
 constexpr int PLAN_BAR = 2;   // consumer warp 0 and the producer warp
 
@@ -354,6 +359,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
       unsigned long long *lz = a.lacc + (size_t)(par ^ 1) * 2 * E;
       for (int e = c * nth + tid; e < 2 * E; e += G * nth) lz[e] = 0ull;
       named_barrier_sync(CONS_BAR, nth);
+      if (tid == 0) trace_point(a, l, TP_LOGITS);
       if (warp == 0) {
         topk_smem(logits, E, k, st->idx, st->gate, &st->tks);
         if (lane == 0) trace_point(a, l, TP_TOPK);
@@ -464,7 +470,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
       const int n = nring + m;
       if (!wait_full(n)) break;
       const int i = ilo + m, u = i >> 1, mat = i & 1, j = u / I16, r = u % I16;
-      const float2 o = tile_dot1<BITS, 4>(ring + (size_t)(n % S) * a.slot_bytes, nblkH, limbs, lsc);
+      const float2 o = tile_dot1<BITS, 1>(ring + (size_t)(n % S) * a.slot_bytes, nblkH, limbs, lsc);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[n % S]);
       // this tile's 16 rows into the local block: a_g / a_u of rows 16 (r & 1) ..
@@ -514,7 +520,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
       bool ok = mbar_wait(dnbar, (uint32_t)(l & 1), clock64() + WAIT_BUDGET_CYCLES);
       if (ok) {
         for (int j = warp; j < k; j += SK_NCW) {
-          const float2 o = tile_dot1<BITS, 4>(dnbuf + (size_t)j * tdn, nblkI, limbs + (size_t)j * nblkI * LIMB_REC,
+          const float2 o = tile_dot1<BITS, 1>(dnbuf + (size_t)j * tdn, nblkI, limbs + (size_t)j * nblkI * LIMB_REC,
                                            lsc + (size_t)j * nblkI);
           if ((lane & 3) == 0) {
             const int g = lane >> 2;

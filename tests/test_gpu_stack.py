@@ -208,6 +208,7 @@ def test_fused_phase_trace_is_ordered_and_layer_times_add_up():
     tr = st.phase_trace()
     assert tr.shape[0] == 4 and tr.shape[2] == 8
     assert (np.diff(tr[:, :, :7], axis=2) >= 0).all()
+    assert ((tr[:, :, 0] <= tr[:, :, 7]) & (tr[:, :, 7] <= tr[:, :, 1])).all()   # logits ready, then the top-k
     route_ms, ffn_ms = st.layer_times()
     assert all(r >= 0 for r in route_ms) and all(f > 0 for f in ffn_ms)
     plain = DecodeStack(layers, routers, None, 1, cfg.k, cfg.eps)

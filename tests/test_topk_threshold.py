@@ -1,9 +1,9 @@
 """The candidate threshold of the warp top-k, checked on the CPU with its rule
 restated.
 
-Expert e sits on lane e % 32 of a warp. Every float64 logit gets an fp32 key
-(round to nearest, -0 taken as +0, made order-preserving as an unsigned
-integer). The threshold is the k-th largest of the 32 per-lane maximum keys
+Expert e sits on lane e % 32 of a warp. Every float64 logit gets a 32-bit key:
+the top 32 bits of its float64 pattern (-0 taken as +0), made order-preserving
+as an unsigned integer. The threshold is the k-th largest of the 32 per-lane maximum keys
 (ties by lane); every key at or above it is a candidate, and the exact ranking
 (logit descending, lower index on ties) runs on the candidates only. The
 candidate set must contain the exact top-k for any logits; it should stay small
@@ -13,10 +13,11 @@ import pytest
 
 
 def keys(logits):
-    f = np.asarray(logits, dtype=np.float64).astype(np.float32)
-    f = np.where(f == 0, np.float32(0), f).astype(np.float32)
-    b = f.view(np.uint32).astype(np.uint64)
-    return np.where(b & 0x80000000, (~b) & 0xFFFFFFFF, b | 0x80000000)
+    f = np.asarray(logits, dtype=np.float64)
+    f = np.where(f == 0, 0.0, f)
+    b = f.view(np.uint64)
+    o = np.where(b & np.uint64(1 << 63), ~b, b | np.uint64(1 << 63))
+    return o >> np.uint64(32)
 
 
 def candidates(logits, k):
