@@ -484,11 +484,17 @@ def measure_stack(args, cfg, seed=SEED, full=True):
         # start, averaged over the layers of the last replay (in microseconds
         # at the sampled SM clock)
         tr = tstack.phase_trace().astype(np.float64)                     # [L, CTAs, points]
-        rel = np.median(tr[:, :, 1:8] - tr[:, :, :1], axis=1).mean(axis=0)
+        rows = np.arange(tr.shape[1]) < cfg.H // 16                     # CTAs with a phase D
+        busy = tr[:, :, 8] != 0                                          # CTAs with gate/up tiles
+        first = np.array([[np.median((tr[l, :, 8] - tr[l, :, 0])[busy[l]])] for l in range(tr.shape[0])])
+        rel = np.concatenate([np.median(tr[:, :, 1:8] - tr[:, :, :1], axis=1), first,
+                              np.median(tr[:, rows, 9:] - tr[:, rows, :1], axis=1)], axis=1).mean(axis=0)
         mhz = clk.get("sm_mhz") or clk.get("sm_max_mhz") or 1965.0
         names = ["topk_done", "tiles_start", "tiles_done", "barrier1_passed", "down_done", "barrier2_passed",
-                 "logits_ready"]
+                 "logits_ready", "first_tile_landed", "h_limbs_landed", "down_tiles_done", "z_written"]
         phases = {n: float(v) / mhz for n, v in zip(names, rel)}
+        # the slowest CTA's gate/up tiles hold the first grid barrier
+        phases["tiles_done_max_cta"] = float(np.max(tr[:, :, 3] - tr[:, :, 0], axis=1).mean()) / mhz
     tstack.close()
     del layers, routers, biases, xs
     free_device()

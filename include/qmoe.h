@@ -119,10 +119,15 @@ qmoe_status qmoe_pack(int fmt, int kind, int E, int H, int I,
  * gate fp32 [T,k]. Workspace: qmoe_route_workspace_bytes(T, E) bytes, zeroed
  * once before first use (it is left zeroed by every completed call).
  * Limits: 1 <= k <= 16, k <= E <= 1024, H multiple of 128, T >= 1.
- * T <= 8 with fp32 x runs the single-pass decode router (float64 GEMV); larger
- * T or bf16 x runs the prefill router (a float64 logit GEMM over register
- * tiles into the workspace, then one warp per token for the selection). Both
- * form every product exactly in float64 and sum in float64. */
+ * T <= 8 with fp32 x runs the decode router: every 16-element slice partial
+ * sum_h x*Wr is a float64 fused multiply-add chain, split into two exact
+ * integers and summed exactly, so the logit does not depend on how the work is
+ * split (the fused layer stack forms the same logits); one warp per token then
+ * selects from shared memory. Larger T or bf16 x runs the prefill router:
+ * approximate logits on the integer tensor cores (16-bit fixed point in two
+ * 8-bit limbs) with a proven error bound pick a few candidates per token,
+ * whose float64 logits (exact products, float64 sums) decide the selection
+ * and the gates. */
 size_t qmoe_route_workspace_bytes(int T, int E);
 qmoe_status qmoe_route(const float *Wr, const float *bias, const void *x, int x_dtype,
                        int T, int H, int E, int k, int32_t *idx, float *gate,
@@ -153,9 +158,9 @@ qmoe_status qmoe_rmsnorm_residual(const float *x_in, const float *y, float eps, 
  * synchronise the device). This entry point has no counterpart in the
  * method's sources; it is an interface convenience of this library.
  * It runs the same single-pass decode router as qmoe_route with fp32 x, with
- * its scratch (float64 logits and a 256-byte completion ticket) held in one
- * fixed device array of QMOE_ROUTE_FIXED_SCRATCH_BYTES bytes inside the
- * library; nothing is allocated.
+ * its scratch (the exact integer partial-logit sums and a 256-byte completion
+ * ticket) held in one fixed device array of QMOE_ROUTE_FIXED_SCRATCH_BYTES
+ * bytes inside the library; nothing is allocated.
  * Limits: 1 <= T <= QMOE_ROUTE_FIXED_MAX_T, E <= QMOE_ROUTE_FIXED_MAX_E,
  * 1 <= k <= 16, H a multiple of 128; larger requests return UNSUPPORTED.
  * The first call on each device looks up the array's address and zeroes it
@@ -166,7 +171,7 @@ qmoe_status qmoe_rmsnorm_residual(const float *x_in, const float *y, float eps, 
  * them on one stream. */
 #define QMOE_ROUTE_FIXED_MAX_T 8
 #define QMOE_ROUTE_FIXED_MAX_E 1024
-#define QMOE_ROUTE_FIXED_SCRATCH_BYTES (QMOE_ROUTE_FIXED_MAX_T * QMOE_ROUTE_FIXED_MAX_E * 8 + 256)
+#define QMOE_ROUTE_FIXED_SCRATCH_BYTES (QMOE_ROUTE_FIXED_MAX_T * 2 * QMOE_ROUTE_FIXED_MAX_E * 8 + 256)
 qmoe_status qmoe_route_fixed(const float *Wr, const float *bias, const float *x, int T, int H, int E, int k,
                              int32_t *idx, float *gate, int32_t *dev_status, qmoe_stream_t stream);
 
@@ -319,8 +324,11 @@ qmoe_status qmoe_stack_layer_times(const qmoe_stack *stack, float *route_ms, flo
  * compare only stamps of one CTA), int64 [L][*ctas][*points]: layer start,
  * top-k done, gate/up tiles start, gate/up tiles done, first grid barrier
  * passed, down tiles and router partials done, second grid barrier passed,
- * logits and normalised x ready (recorded between the first and second). count is the capacity of cycles_host in entries (WORKSPACE
- * if too small). UNSUPPORTED on the per-layer path or without the flag.
+ * logits and normalised x ready (recorded between the first and second),
+ * first gate/up tile landed (0 in a CTA without gate/up tiles), h limbs
+ * landed, down tiles done, z written (these three 0 in CTAs that own no
+ * output rows). count is the
+ * capacity of cycles_host in entries (WORKSPACE if too small). UNSUPPORTED on the per-layer path or without the flag.
  * Synchronises the device. */
 qmoe_status qmoe_stack_trace(const qmoe_stack *stack, int64_t *cycles_host, size_t count, int *ctas, int *points);
 /* One graph replay on `stream`: reads the stack's input buffer, writes its

@@ -232,7 +232,7 @@ def qmoe_stack_kernels_per_replay(stack: int) -> int:
     return lib().qmoe_stack_kernels_per_replay(stack)
 
 
-def qmoe_stack_trace(stack: int, L: int, max_ctas: int = 1024, points: int = 8):
+def qmoe_stack_trace(stack: int, L: int, max_ctas: int = 1024, points: int = 16):
     """Phase stamps (SM cycles) of the last replay: numpy int64 [L, ctas, points]."""
     import numpy as np
     buf = np.zeros(L * max_ctas * points, dtype=np.int64)

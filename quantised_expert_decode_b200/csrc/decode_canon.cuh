@@ -87,12 +87,26 @@ __device__ __forceinline__ double join(long long hi, long long lo) {
   return __dadd_rn(__dmul_rn(i64_to_f64(hi), FIX_HI_INV), __dmul_rn(i64_to_f64(lo), FIX_LO_INV));
 }
 
+// float -> float64, exactly, for normal numbers by moving the bits (IEEE 754
+// binary32 -> binary64: the exponent rebiased by 1023 - 127, the 23 mantissa
+// bits placed at the top of the 52); zero, subnormals, infinities and NaN go
+// through the conversion instruction. Integer operations only on the common
+// path: the conversion unit issues at a small fraction of the integer rate and
+// was the bottleneck of the router's dot products.
+__device__ __forceinline__ double f2d(float f) {
+  const unsigned u = __float_as_uint(f);
+  const unsigned a = u & 0x7fffffffu;
+  if (a - 0x00800000u < 0x7f000000u)
+    return __hiloint2double((int)((u & 0x80000000u) | ((a >> 3) + 0x38000000u)), (int)(a << 29));
+  return (double)f;
+}
+
 // Router partial of one slice: w(i), z(i) for i = 0..15.
 template <class W, class Z>
 __device__ __forceinline__ double slice_dot(W w, Z z) {
   double p = 0.0;
 #pragma unroll
-  for (int i = 0; i < SLICE; ++i) p = fma((double)w(i), (double)z(i), p);
+  for (int i = 0; i < SLICE; ++i) p = fma(f2d(w(i)), f2d(z(i)), p);
   return p;
 }
 
@@ -102,7 +116,7 @@ __device__ __forceinline__ double slice_sumsq(Z z) {
   double p = 0.0;
 #pragma unroll
   for (int i = 0; i < SLICE; ++i) {
-    const double v = (double)z(i);
+    const double v = f2d(z(i));
     p = fma(v, v, p);
   }
   return p;
@@ -112,12 +126,11 @@ __device__ __forceinline__ double slice_sumsq(Z z) {
 // order above; every lane of the calling warp returns the same value.
 // Up to PRE slice sums per lane are fetched before any is added, so slice sums
 // read from global memory cost one round trip, not one per slice.
-template <int PRE = 4, class Q>
-__device__ __forceinline__ double warp_sumsq(Q q, int nsl) {
+// The same order with the lane's first PRE slice sums v[m] (slice lane + 32 m)
+// already formed; slices from 32 PRE on come from q(c).
+template <int PRE, class Q>
+__device__ __forceinline__ double warp_sum_slices(const double (&v)[PRE], Q q, int nsl) {
   const int lane = threadIdx.x & 31;
-  double v[PRE];
-#pragma unroll
-  for (int m = 0; m < PRE; ++m) v[m] = lane + 32 * m < nsl ? q(lane + 32 * m) : 0.0;
   double s = 0.0;
 #pragma unroll
   for (int m = 0; m < PRE; ++m)
@@ -126,6 +139,15 @@ __device__ __forceinline__ double warp_sumsq(Q q, int nsl) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, o));
   return s;
+}
+
+template <int PRE = 4, class Q>
+__device__ __forceinline__ double warp_sumsq(Q q, int nsl) {
+  const int lane = threadIdx.x & 31;
+  double v[PRE];
+#pragma unroll
+  for (int m = 0; m < PRE; ++m) v[m] = lane + 32 * m < nsl ? q(lane + 32 * m) : 0.0;
+  return warp_sum_slices<PRE>(v, q, nsl);
 }
 
 // 1 / rms from the sum of squares of H elements.

@@ -3,6 +3,19 @@
 // expert index, renormalised gates; optionally preceded by the residual
 // RMSNorm of the previous layer's output. The arithmetic is the one of
 // decode_canon.cuh, shared with the fused layer-stack kernel.
+//
+// Work split. CTA (g, s) owns the 32 experts 32g .. 32g+31 (one per lane) and
+// the s-th of ns ranges of 16-element slices of the hidden axis; its warps
+// take the range's slices in turn. A lane streams its expert's weights of a
+// slice into registers and forms the slice partial of every token at once:
+// the activations of the range sit in shared memory as float64 [h][token], so
+// one broadcast load serves the whole warp. The slice partials are split into
+// exact integers (decode_canon.cuh), summed over the CTA's warps and added
+// into the workspace with integer atomics; integer sums do not depend on the
+// order, so the logits are the same for any split. The CTA that finishes last
+// forms the logits (partial sum / rms + bias), selects every token's experts
+// (one warp per token, from shared memory) and clears the sums for the next
+// call.
 #include <mutex>
 
 #include "common.cuh"
@@ -12,10 +25,13 @@
 namespace qmoe {
 namespace {
 
-constexpr int RT_WARPS = 8;                // one router row per warp; one token per warp for the top-k
+constexpr int RT_WARPS = 8;
 constexpr int RT_THREADS = 32 * RT_WARPS;
 constexpr int RT_MAXT = 8;
-constexpr int RT_PRE = 4;                  // slices per lane held in registers (all of H <= 2048)
+constexpr int RT_GROUP = 32;               // experts per CTA, one per lane
+constexpr int RT_CHUNK = 16;               // slices staged in shared memory at a time
+constexpr int RT_PRE = 2;                  // slices per warp whose weights are fetched before the wait
+static_assert(RT_CHUNK * 16 == 32 * RT_WARPS, "a whole chunk is one element per thread and token");
 
 struct RouteArgs {
   const float *Wr;
@@ -25,166 +41,263 @@ struct RouteArgs {
   float *x_out;        // normalised activations (RESID only)
   float eps;
   int T, H, E, k;
+  int ns;              // hidden-axis ranges per expert group
   int32_t *idx;
   float *gate;
-  double *logits;      // workspace [T, E]
-  unsigned *ticket;    // workspace
+  unsigned long long *lacc;   // workspace [T][2 hi|lo][E] exact partial-logit sums (two's complement)
+  unsigned *ticket;           // workspace
   int32_t *status;
 };
 
-// z = x (+ y) of every token sits in shared memory with one pad float after
-// every 32: element h of token t at t * HP + h + h / 32 (HP = H + H / 32). A
-// lane reads the 16 elements of one slice, lanes 16 elements apart; the pad
-// spreads the 32 lanes of a warp over the 32 banks.
-__host__ __device__ inline int route_hp(int H) { return H + H / 32; }
-__device__ __forceinline__ int zpos(int h) { return h + (h >> 5); }
-inline size_t route_smem_bytes(int T, int H) { return (size_t)T * route_hp(H) * 4; }
+// Dynamic shared memory of one CTA: the largest of the staged activations
+// (float64 [RT_CHUNK * 16][TT]), the per-warp integer sums
+// ([RT_WARPS][TT][2][32]) and, in the last CTA, the logits ([T][E]).
+inline size_t route_smem_bytes(int TT, int E) {
+  size_t z = (size_t)RT_CHUNK * canon::SLICE * TT * 8;
+  size_t r = (size_t)RT_WARPS * TT * 2 * RT_GROUP * 8;
+  size_t l = (size_t)TT * E * 8;
+  size_t m = z > r ? z : r;
+  return m > l ? m : l;
+}
 
-template <bool RESID>
+// One warp: token t's 1 / rms from z = x + y (decode_canon.cuh's order) and
+// x_out[t] = z * (float)(1 / rms). Up to H = 2048 a lane keeps its four
+// slices of z in registers, so x and y are read once, all loads in flight.
+__device__ __forceinline__ float4 add4(float4 u, float4 v) {
+  return make_float4(__fadd_rn(u.x, v.x), __fadd_rn(u.y, v.y), __fadd_rn(u.z, v.z), __fadd_rn(u.w, v.w));
+}
+__device__ __forceinline__ float4 scale4(float4 u, float s) {
+  return make_float4(__fmul_rn(u.x, s), __fmul_rn(u.y, s), __fmul_rn(u.z, s), __fmul_rn(u.w, s));
+}
+__device__ __forceinline__ float comp4(const float4 &u, int i) { return i == 0 ? u.x : i == 1 ? u.y : i == 2 ? u.z : u.w; }
+
+__device__ double resid_norm_token(const RouteArgs &a, int t) {
+  const int lane = threadIdx.x & 31, H = a.H, nsl = H / canon::SLICE;
+  const float4 *x4 = reinterpret_cast<const float4 *>(a.x + (size_t)t * H);
+  const float4 *y4 = reinterpret_cast<const float4 *>(a.y + (size_t)t * H);
+  float4 *o4 = reinterpret_cast<float4 *>(a.x_out + (size_t)t * H);
+  auto zslice = [&](int c) {
+    return canon::slice_sumsq([&](int i) {
+      return __fadd_rn(__ldcg(a.x + (size_t)t * H + c * canon::SLICE + i), __ldcg(a.y + (size_t)t * H + c * canon::SLICE + i));
+    });
+  };
+  if (nsl <= 128) {
+    float4 z[4][4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int c = lane + 32 * m;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) z[m][q] = c < nsl ? add4(__ldcg(x4 + 4 * c + q), __ldcg(y4 + 4 * c + q))
+                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    double v[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) v[m] = canon::slice_sumsq([&](int i) { return comp4(z[m][i >> 2], i & 3); });
+    const double r = canon::norm_rinv(canon::warp_sum_slices<4>(v, zslice, nsl), H, a.eps);
+    const float inv = __double2float_rn(r);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int c = lane + 32 * m;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (c < nsl) o4[4 * c + q] = scale4(z[m][q], inv);
+    }
+    return r;
+  }
+  const double r = canon::norm_rinv(canon::warp_sumsq(zslice, nsl), H, a.eps);
+  const float inv = __double2float_rn(r);
+  for (int h4 = lane; h4 < H / 4; h4 += 32) o4[h4] = scale4(add4(__ldcg(x4 + h4), __ldcg(y4 + h4)), inv);
+  return r;
+}
+
+// One warp: token t's logits from the exact sums (lane l: experts l + 32 j),
+// written to lg (shared memory) for the candidates' values, keys kept in
+// registers; the sums are cleared for the next call; then the selection.
+template <int M>
+__device__ __forceinline__ void route_token_select(const RouteArgs &a, int t, double rinv, double *lg,
+                                                   TopkScratch *sc) {
+  const int lane = threadIdx.x & 31, E = a.E;
+  unsigned long long *ph = a.lacc + (size_t)t * 2 * E;
+  unsigned long long hv[M], lv[M];
+  float bv[M];
+#pragma unroll
+  for (int j = 0; j < M; ++j) {
+    const int e = lane + 32 * j;
+    hv[j] = lv[j] = 0ull;
+    bv[j] = 0.0f;
+    if (e < E) {
+      hv[j] = __ldcg(ph + e);
+      lv[j] = __ldcg(ph + E + e);
+      if (a.bias) bv[j] = __ldg(a.bias + e);
+    }
+  }
+  unsigned key[M];
+#pragma unroll
+  for (int j = 0; j < M; ++j) {
+    const int e = lane + 32 * j;
+    key[j] = 0u;
+    if (e < E) {
+      const double v = canon::logit(canon::join((long long)hv[j], (long long)lv[j]), rinv,
+                                    a.bias ? canon::f2d(bv[j]) : 0.0);
+      lg[e] = v;
+      key[j] = logit_key(v);
+      ph[e] = 0ull;
+      ph[E + e] = 0ull;
+    }
+  }
+  __syncwarp();
+  warp_topk_keys<M>(key, [&](int e) { return lg[e]; }, E, a.k, a.idx + t * a.k, a.gate + t * a.k, sc);
+}
+
+template <int TT, bool RESID>
 __global__ void __launch_bounds__(RT_THREADS, 1) route_decode_kernel(RouteArgs a) {
-  extern __shared__ __align__(16) float zs[];  // [T][HP], padded
-  __shared__ double rinv_s[RT_MAXT];
-  __shared__ float inv_s[RT_MAXT];
+  extern __shared__ __align__(16) double rsm[];
   __shared__ unsigned is_last;
   __shared__ int range_bad;
   __shared__ TopkScratch topk_sc[RT_WARPS];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int T = a.T, H = a.H, E = a.E, nsl = H / canon::SLICE, HP = route_hp(H);
-  const int e_row = blockIdx.x * RT_WARPS + warp;
+  const int T = a.T, H = a.H, E = a.E, nsl = H / canon::SLICE;
+  const int g = blockIdx.x / a.ns, sp = blockIdx.x % a.ns;
+  const int e = g * RT_GROUP + lane;
+  const bool live = e < E;
+  const int c0 = (int)((long long)sp * nsl / a.ns), c1 = (int)((long long)(sp + 1) * nsl / a.ns);
+  const float4 *wrow = reinterpret_cast<const float4 *>(a.Wr + (size_t)(live ? e : 0) * H);
 
-  // This warp's router row does not depend on the previous kernel: fetch the
-  // lane's slices (c = lane + 32 j) into registers before waiting for it.
+  // The first slices' weights do not depend on the previous kernel: fetch
+  // them before waiting for it.
   float4 wpre[RT_PRE][4];
-  if (e_row < E) {
-    const float4 *w4 = reinterpret_cast<const float4 *>(a.Wr + (size_t)e_row * H);
 #pragma unroll
-    for (int j = 0; j < RT_PRE; ++j) {
-      const int c = lane + 32 * j;
+  for (int m = 0; m < RT_PRE; ++m) {
+    const int c = c0 + warp + RT_WARPS * m;
 #pragma unroll
-      for (int m = 0; m < 4; ++m)
-        if (c < nsl) wpre[j][m] = __ldg(w4 + c * 4 + m);
-    }
+    for (int q = 0; q < 4; ++q)
+      wpre[m][q] = (live && c < c1 && c < c0 + RT_CHUNK) ? __ldg(wrow + c * 4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   if (tid == 0) range_bad = 0;
   pdl_wait();
   pdl_launch_dependents();
 
-  // z = x (+ y) into the padded layout; eight float4 of each input in flight
-  // per thread
-  {
-    const float4 *x4 = reinterpret_cast<const float4 *>(a.x);
-    const float4 *y4 = reinterpret_cast<const float4 *>(a.y);
-    const int n4 = T * H / 4, H4 = H / 4;
-    constexpr int B = 8;
-    for (int i0 = tid; i0 < n4; i0 += B * RT_THREADS) {
-      float4 xv[B], yv[B];
+  long long hi[TT], lo[TT];
 #pragma unroll
-      for (int u = 0; u < B; ++u) {
-        const int i = i0 + u * RT_THREADS;
-        if (i < n4) {
-          xv[u] = __ldcg(x4 + i);
-          if (RESID) yv[u] = __ldcg(y4 + i);
-        }
-      }
+  for (int t = 0; t < TT; ++t) hi[t] = lo[t] = 0;
+  bool ok = true;
+  double *zd = rsm;   // [RT_CHUNK * 16][TT]
+  int cc = c0;
+  // slice c of the staged chunk: every token's partial, split and summed
+  auto slice = [&](int c, const float4 (&w4)[4]) {
+    double p[TT];
 #pragma unroll
-      for (int u = 0; u < B; ++u) {
-        const int i = i0 + u * RT_THREADS;
-        if (i < n4) {
-          float4 v = xv[u];
-          if (RESID) {
-            v.x = __fadd_rn(v.x, yv[u].x); v.y = __fadd_rn(v.y, yv[u].y);
-            v.z = __fadd_rn(v.z, yv[u].z); v.w = __fadd_rn(v.w, yv[u].w);
-          }
-          const int t = i / H4, h = 4 * (i % H4);
-          float *zt = zs + (size_t)t * HP;
-          zt[zpos(h)] = v.x; zt[zpos(h + 1)] = v.y; zt[zpos(h + 2)] = v.z; zt[zpos(h + 3)] = v.w;
+    for (int t = 0; t < TT; ++t) p[t] = 0.0;
+    const double *zc = zd + (size_t)(c - cc) * canon::SLICE * TT;
+#pragma unroll
+    for (int i = 0; i < canon::SLICE; ++i) {
+      const float4 v = w4[i >> 2];
+      const double w = canon::f2d((i & 3) == 0 ? v.x : (i & 3) == 1 ? v.y : (i & 3) == 2 ? v.z : v.w);
+      if (TT == 1) {
+        p[0] = fma(w, zc[i], p[0]);
+      } else {
+#pragma unroll
+        for (int t = 0; t < TT; t += 2) {
+          const double2 z2 = *reinterpret_cast<const double2 *>(zc + i * TT + t);
+          p[t] = fma(w, z2.x, p[t]);
+          p[t + 1] = fma(w, z2.y, p[t + 1]);
         }
       }
     }
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+      long long h1, l1;
+      ok &= canon::split(p[t], h1, l1);
+      hi[t] += h1;
+      lo[t] += l1;
+    }
+  };
+  for (; cc < c1; cc += RT_CHUNK) {
+    const int ncs = min(RT_CHUNK, c1 - cc), nh = ncs * canon::SLICE, h0 = cc * canon::SLICE;
+    __syncthreads();   // the previous chunk is no longer read
+    if (nh == RT_THREADS) {
+      // a whole chunk: element h0 + tid of every token, all loads in flight at once
+      float xv[TT], yv[TT];
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        xv[t] = yv[t] = 0.0f;
+        if (t < T) {
+          xv[t] = __ldcg(a.x + (size_t)t * H + h0 + tid);
+          if (RESID) yv[t] = __ldcg(a.y + (size_t)t * H + h0 + tid);
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < TT; ++t) zd[tid * TT + t] = canon::f2d(RESID ? __fadd_rn(xv[t], yv[t]) : xv[t]);
+    } else {
+      for (int i = tid; i < TT * nh; i += RT_THREADS) {
+        const int t = i / nh, hh = i % nh;
+        float z = 0.0f;
+        if (t < T) {
+          z = __ldcg(a.x + (size_t)t * H + h0 + hh);
+          if (RESID) z = __fadd_rn(z, __ldcg(a.y + (size_t)t * H + h0 + hh));
+        }
+        zd[hh * TT + t] = canon::f2d(z);
+      }
+    }
+    __syncthreads();
+    if (cc == c0) {
+      if (warp < ncs) slice(cc + warp, wpre[0]);
+      if (warp + RT_WARPS < ncs) slice(cc + warp + RT_WARPS, wpre[1]);
+    }
+    for (int m = cc == c0 ? RT_PRE : 0; warp + RT_WARPS * m < ncs; ++m) {
+      const int c = cc + warp + RT_WARPS * m;
+      float4 w4[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) w4[q] = live ? __ldg(wrow + c * 4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+      slice(c, w4);
+    }
+  }
+  if (!ok && live) range_bad = 1;
+
+  // sum the warps' integers, then one pair of atomics per (token, expert)
+  __syncthreads();
+  unsigned long long *red = reinterpret_cast<unsigned long long *>(rsm);   // [warp][TT][2][32]
+#pragma unroll
+  for (int t = 0; t < TT; ++t) {
+    red[((warp * TT + t) * 2 + 0) * RT_GROUP + lane] = (unsigned long long)hi[t];
+    red[((warp * TT + t) * 2 + 1) * RT_GROUP + lane] = (unsigned long long)lo[t];
   }
   __syncthreads();
-  if (RESID) {
-    // sum of squares of every token (one warp per token), then 1 / rms
-    for (int t = warp; t < T; t += RT_WARPS) {
-      const float *zt = zs + (size_t)t * HP;
-      const double ss = canon::warp_sumsq(
-          [&](int c) { return canon::slice_sumsq([&](int i) { return zt[zpos(c * canon::SLICE + i)]; }); }, nsl);
-      if (lane == 0) {
-        const double r = canon::norm_rinv(ss, H, a.eps);
-        rinv_s[t] = r;
-        inv_s[t] = __double2float_rn(r);
-      }
-    }
-    __syncthreads();
-    if (blockIdx.x == 0) {
-      float4 *xo4 = reinterpret_cast<float4 *>(a.x_out);
-      const int H4 = H / 4;
-      for (int i = tid; i < T * H4; i += RT_THREADS) {
-        const int t = i / H4, h = 4 * (i % H4);
-        const float s = inv_s[t];
-        const float *zt = zs + (size_t)t * HP;
-        xo4[i] = make_float4(__fmul_rn(zt[zpos(h)], s), __fmul_rn(zt[zpos(h + 1)], s), __fmul_rn(zt[zpos(h + 2)], s),
-                             __fmul_rn(zt[zpos(h + 3)], s));
-      }
-    }
-  } else {
-    if (tid < RT_MAXT) rinv_s[tid] = 1.0;
-    __syncthreads();
-  }
-
-  // logits: one warp per router row; slice partials split into exact integers
-  if (e_row < E) {
-    const float4 *w4 = reinterpret_cast<const float4 *>(a.Wr + (size_t)e_row * H);
-    const double b = a.bias ? (double)a.bias[e_row] : 0.0;
-    bool ok = true;
-#pragma unroll 1
-    for (int t = 0; t < T; ++t) {
-      const float *zt = zs + (size_t)t * HP;
-      long long hi = 0, lo = 0;
+  for (int i = tid; i < TT * 2 * RT_GROUP; i += RT_THREADS) {
+    const int t = i / (2 * RT_GROUP), which = (i / RT_GROUP) & 1, ln = i % RT_GROUP;
+    const int ee = g * RT_GROUP + ln;
+    if (t < T && ee < E) {
+      unsigned long long v = 0;
 #pragma unroll
-      for (int j = 0; j < RT_PRE; ++j) {
-        const int c = lane + 32 * j;
-        if (c < nsl) {
-          const float *zc = zt + zpos(c * canon::SLICE);   // a slice never crosses a pad
-          const double p = canon::slice_dot(
-              [&](int i) {
-                const float4 v = wpre[j][i >> 2];
-                return (i & 3) == 0 ? v.x : (i & 3) == 1 ? v.y : (i & 3) == 2 ? v.z : v.w;
-              },
-              [&](int i) { return zc[i]; });
-          long long h1, l1;
-          ok &= canon::split(p, h1, l1);
-          hi += h1;
-          lo += l1;
-        }
-      }
-      for (int c = lane + 32 * RT_PRE; c < nsl; c += 32) {   // larger H only
-        const float *zc = zt + zpos(c * canon::SLICE);
-        const float *wc = reinterpret_cast<const float *>(w4 + c * 4);
-        long long h1, l1;
-        ok &= canon::split(canon::slice_dot([&](int i) { return __ldg(wc + i); }, [&](int i) { return zc[i]; }), h1,
-                           l1);
-        hi += h1;
-        lo += l1;
-      }
-      canon::warp_sum_fix(hi, lo);
-      if (lane == 0) a.logits[(size_t)t * E + e_row] = canon::logit(canon::join(hi, lo), rinv_s[t], b);
+      for (int w = 0; w < RT_WARPS; ++w) v += red[((w * TT + t) * 2 + which) * RT_GROUP + ln];
+      atomicAdd(a.lacc + ((size_t)t * 2 + which) * E + ee, v);
     }
-    if (!ok) range_bad = 1;
   }
 
-  // the last CTA to finish selects the experts of every token (one warp each)
-  __threadfence();
+  // the last CTA to finish selects the experts of every token
   __syncthreads();
   if (tid == 0) {
     if (range_bad) set_status(a.status, DEV_RANGE);
+    __threadfence();
     is_last = (atomicAdd(a.ticket, 1u) == gridDim.x - 1u) ? 1u : 0u;
   }
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  for (int t = warp; t < T; t += RT_WARPS)
-    warp_topk_gates(a.logits + (size_t)t * E, E, a.k, a.idx + t * a.k, a.gate + t * a.k, &topk_sc[warp]);
+  // one warp per token: 1 / rms (RESID), the logits from the exact sums (which
+  // are cleared for the next call), the selection
+  double *lg = rsm;   // [T][E]
+  for (int t = warp; t < T; t += RT_WARPS) {
+    const double rinv = RESID ? resid_norm_token(a, t) : 1.0;
+    double *lt = lg + (size_t)t * E;
+    switch (topk_m(E)) {
+      case 4: route_token_select<4>(a, t, rinv, lt, &topk_sc[warp]); break;
+      case 8: route_token_select<8>(a, t, rinv, lt, &topk_sc[warp]); break;
+      case 16: route_token_select<16>(a, t, rinv, lt, &topk_sc[warp]); break;
+      default: route_token_select<32>(a, t, rinv, lt, &topk_sc[warp]); break;
+    }
+  }
+  __syncthreads();
   __syncthreads();
   if (tid == 0) atomicExch(a.ticket, 0u);
 }
@@ -210,11 +323,14 @@ __global__ void __launch_bounds__(256) rmsnorm_residual_kernel(const float *x, c
   for (int h = tid; h < H; h += 256) out[(size_t)t * H + h] = __fmul_rn(__fadd_rn(xr[h], yr[h]), inv);
 }
 
-size_t decode_ws_bytes(int T, int E) { return (((size_t)T * E * sizeof(double) + 255) & ~(size_t)255) + 256; }
+// Workspace: the exact sums [T][2][E] int64, then a 256-byte ticket block.
+size_t decode_lacc_bytes(int T, int E) { return (((size_t)T * 2 * E * sizeof(unsigned long long)) + 255) & ~(size_t)255; }
+size_t decode_ws_bytes(int T, int E) { return decode_lacc_bytes(T, E) + 256; }
 
-qmoe_status launch_route_decode(const RouteArgs &a, bool resid, cudaStream_t s) {
-  const size_t smem = route_smem_bytes(a.T, a.H);
-  const void *fn = resid ? (const void *)route_decode_kernel<true> : (const void *)route_decode_kernel<false>;
+template <int TT>
+qmoe_status launch_route_tt(RouteArgs a, bool resid, cudaStream_t s) {
+  const void *fn = resid ? (const void *)route_decode_kernel<TT, true> : (const void *)route_decode_kernel<TT, false>;
+  const size_t smem = route_smem_bytes(TT, a.E);
   cudaFuncAttributes fa{};
   if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) return QMOE_ERR_CUDA;
   // static + dynamic shared memory must fit one SM's opt-in limit; above the
@@ -223,9 +339,17 @@ qmoe_status launch_route_decode(const RouteArgs &a, bool resid, cudaStream_t s) 
   if (smem + fa.sharedSizeBytes > 48 * 1024 &&
       cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return QMOE_ERR_CUDA;
-  const int grid = (a.E + RT_WARPS - 1) / RT_WARPS;
+  // the largest shared-memory carve-out, as the FFN kernels around it use:
+  // an SM then need not be reconfigured between the two kernels
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+    return QMOE_ERR_CUDA;
+  const int ng = (a.E + RT_GROUP - 1) / RT_GROUP, nsl = a.H / canon::SLICE;
+  int ns = num_sms() / ng;
+  if (ns > nsl / 8) ns = nsl / 8;
+  if (ns < 1) ns = 1;
+  a.ns = ns;
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3((unsigned)grid);
+  cfg.gridDim = dim3((unsigned)(ng * ns));
   cfg.blockDim = dim3(RT_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
@@ -234,10 +358,17 @@ qmoe_status launch_route_decode(const RouteArgs &a, bool resid, cudaStream_t s) 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = resid ? cudaLaunchKernelEx(&cfg, route_decode_kernel<true>, a)
-                        : cudaLaunchKernelEx(&cfg, route_decode_kernel<false>, a);
+  cudaError_t e = resid ? cudaLaunchKernelEx(&cfg, route_decode_kernel<TT, true>, a)
+                        : cudaLaunchKernelEx(&cfg, route_decode_kernel<TT, false>, a);
   note_launch();
   return cuda_status(e);
+}
+
+qmoe_status launch_route_decode(const RouteArgs &a, bool resid, cudaStream_t s) {
+  if (a.T <= 1) return launch_route_tt<1>(a, resid, s);
+  if (a.T <= 2) return launch_route_tt<2>(a, resid, s);
+  if (a.T <= 4) return launch_route_tt<4>(a, resid, s);
+  return launch_route_tt<8>(a, resid, s);
 }
 
 }  // namespace
@@ -287,8 +418,8 @@ extern "C" qmoe_status qmoe_route(const float *Wr, const float *bias, const void
   a.T = T; a.H = H; a.E = E; a.k = k;
   a.idx = idx;
   a.gate = gate;
-  a.logits = static_cast<double *>(workspace);
-  a.ticket = reinterpret_cast<unsigned *>(static_cast<char *>(workspace) + decode_ws_bytes(T, E) - 256);
+  a.lacc = static_cast<unsigned long long *>(workspace);
+  a.ticket = reinterpret_cast<unsigned *>(static_cast<char *>(workspace) + decode_lacc_bytes(T, E));
   a.status = dev_status;
   return launch_route_decode(a, false, (cudaStream_t)stream);
 }
@@ -314,8 +445,8 @@ extern "C" qmoe_status qmoe_residual_route(const float *x_in, const float *y, fl
   a.T = T; a.H = H; a.E = E; a.k = k;
   a.idx = idx;
   a.gate = gate;
-  a.logits = static_cast<double *>(workspace);
-  a.ticket = reinterpret_cast<unsigned *>(static_cast<char *>(workspace) + decode_ws_bytes(T, E) - 256);
+  a.lacc = static_cast<unsigned long long *>(workspace);
+  a.ticket = reinterpret_cast<unsigned *>(static_cast<char *>(workspace) + decode_lacc_bytes(T, E));
   a.status = dev_status;
   return launch_route_decode(a, true, (cudaStream_t)stream);
 }
@@ -329,11 +460,12 @@ extern "C" qmoe_status qmoe_residual_route(const float *x_in, const float *y, fl
 namespace qmoe {
 namespace {
 
-constexpr size_t FIXED_LOGITS_BYTES = (size_t)QMOE_ROUTE_FIXED_MAX_T * QMOE_ROUTE_FIXED_MAX_E * sizeof(double);
-static_assert(QMOE_ROUTE_FIXED_SCRATCH_BYTES == FIXED_LOGITS_BYTES + 256, "fixed scratch layout");
+constexpr size_t FIXED_SUMS_BYTES = (size_t)QMOE_ROUTE_FIXED_MAX_T * 2 * QMOE_ROUTE_FIXED_MAX_E * 8;
+static_assert(QMOE_ROUTE_FIXED_SCRATCH_BYTES == FIXED_SUMS_BYTES + 256, "fixed scratch layout");
 
-// [0, FIXED_LOGITS_BYTES): float64 logits; then the 256-byte ticket block,
-// which must start at zero (each completed call leaves it at zero).
+// [0, FIXED_SUMS_BYTES): the exact partial-logit sums ([T][2][E] int64, laid
+// out for the call's own T and E); then the 256-byte ticket block. Both must
+// start at zero, and each completed call leaves them at zero.
 __device__ __align__(256) unsigned char g_route_scratch[QMOE_ROUTE_FIXED_SCRATCH_BYTES];
 
 constexpr int FIXED_MAX_DEVICES = 64;
@@ -380,8 +512,8 @@ extern "C" qmoe_status qmoe_route_fixed(const float *Wr, const float *bias, cons
   a.T = T; a.H = H; a.E = E; a.k = k;
   a.idx = idx;
   a.gate = gate;
-  a.logits = static_cast<double *>(scratch);
-  a.ticket = reinterpret_cast<unsigned *>(static_cast<char *>(scratch) + FIXED_LOGITS_BYTES);
+  a.lacc = static_cast<unsigned long long *>(scratch);
+  a.ticket = reinterpret_cast<unsigned *>(static_cast<char *>(scratch) + FIXED_SUMS_BYTES);
   a.status = dev_status;
   return launch_route_decode(a, false, (cudaStream_t)stream);
 }

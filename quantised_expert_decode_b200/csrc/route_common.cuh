@@ -166,6 +166,153 @@ __device__ inline void warp_topk_gates_m(Get get, int E, int k, int32_t *idx_out
   __syncwarp();
 }
 
+// Key of a float64 logit from its bits: the high word made order-preserving
+// as an unsigned integer. Every negative number whose high word is
+// 0x80000000 (-0 and the smallest subnormals) takes the key of +0, which keeps
+// the key monotone and gives -0 and +0 one key; NaN takes the key of
+// -infinity, its rank. Integer operations only; never 0 (0 marks "no logit").
+__device__ __forceinline__ unsigned logit_key(double v) {
+  unsigned hi = (unsigned)__double2hiint(v);
+  const unsigned ahi = hi & 0x7fffffffu;
+  if (ahi >= 0x7ff00000u && (ahi > 0x7ff00000u || (unsigned)__double2loint(v) != 0u)) hi = 0xfff00000u;
+  if (hi == 0x80000000u) hi = 0u;
+  return hi ^ ((unsigned)((int)hi >> 31) | 0x80000000u);
+}
+
+// Position of expert e's key in a per-lane key table of M keys a lane
+// (lane e % 32 holds the keys of experts e % 32 + 32 j, j < M, contiguously).
+__device__ __forceinline__ int key_slot(int e, int M) { return (e & 31) * M + (e >> 5); }
+
+// Keys per lane for E experts (a power of two, at least 4 so that a lane's
+// keys load as 16-byte vectors).
+__host__ __device__ constexpr int topk_m(int E) {
+  return E <= 128 ? 4 : E <= 256 ? 8 : E <= 512 ? 16 : 32;
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// The selection above with the keys already in registers: lane l holds
+// key[j] = key of expert l + 32 j (0 for e >= E), and val(e) returns expert
+// e's float64 logit (for the candidates only). Candidate positions come from
+// one ballot per key column, so no step waits on a chain of shuffles.
+template <int M, class Val>
+__device__ __forceinline__ void warp_topk_keys(const unsigned (&key)[M], Val val, int E, int k, int32_t *idx_out,
+                                               float *gate_out, TopkScratch *sc) {
+  const int lane = threadIdx.x & 31;
+  unsigned lmax = key[0];
+#pragma unroll
+  for (int j = 1; j < M; ++j) lmax = max(lmax, key[j]);
+  int rank = 0;
+#pragma unroll
+  for (int s2 = 0; s2 < 32; ++s2) {
+    const unsigned o = __shfl_sync(0xffffffffu, lmax, s2);
+    rank += (o > lmax || (o == lmax && s2 < lane)) ? 1 : 0;
+  }
+  // ranks are a permutation of 0..31; k <= TOPK_MAX_K <= 32. Lanes without a
+  // valid key have maximum 0, so with fewer than k such lanes thr is 0 and
+  // every valid key is a candidate.
+  const unsigned at = __ballot_sync(0xffffffffu, rank == k - 1);
+  const unsigned thr = __shfl_sync(0xffffffffu, lmax, __ffs(at) - 1);
+  const unsigned below = lanemask_lt();
+  int total = 0;
+#pragma unroll
+  for (int j = 0; j < M; ++j) {
+    const bool c = key[j] != 0u && key[j] >= thr;
+    const unsigned b = __ballot_sync(0xffffffffu, c);
+    const int pos = total + __popc(b & below);
+    if (c && pos < TOPK_CAND) sc->cand[pos] = lane + 32 * j;
+    total += __popc(b);
+  }
+  __syncwarp();
+  if (total <= 32) {
+    int ce = 0;
+    double cv = 0.0;
+    if (lane < total) {
+      ce = sc->cand[lane];
+      cv = rank_value(val(ce));
+    }
+    int r = 0;
+    if (total <= 16) {
+#pragma unroll
+      for (int i2 = 0; i2 < 16; ++i2) {
+        const double v2 = __shfl_sync(0xffffffffu, cv, i2);
+        const int e2 = __shfl_sync(0xffffffffu, ce, i2);
+        r += (i2 < total && ranks_above(v2, e2, cv, ce)) ? 1 : 0;
+      }
+    } else {
+#pragma unroll
+      for (int i2 = 0; i2 < 32; ++i2) {
+        const double v2 = __shfl_sync(0xffffffffu, cv, i2);
+        const int e2 = __shfl_sync(0xffffffffu, ce, i2);
+        r += (i2 < total && ranks_above(v2, e2, cv, ce)) ? 1 : 0;
+      }
+    }
+    if (lane < total && r < k) {
+      sc->sel_e[r] = ce;
+      sc->sel_v[r] = cv;
+    }
+  } else if (total <= TOPK_CAND) {
+    for (int i = lane; i < total; i += 32) sc->cand_v[i] = rank_value(val(sc->cand[i]));
+    __syncwarp();
+    for (int i = lane; i < total; i += 32) {
+      const int e = sc->cand[i];
+      const double v = sc->cand_v[i];
+      int r = 0;
+      for (int i2 = 0; i2 < total; ++i2) r += ranks_above(sc->cand_v[i2], sc->cand[i2], v, e) ? 1 : 0;
+      if (r < k) {
+        sc->sel_e[r] = e;
+        sc->sel_v[r] = v;
+      }
+    }
+  } else {
+    // many equal keys (degenerate router): rank the candidates against all logits
+#pragma unroll
+    for (int j = 0; j < M; ++j) {
+      if (key[j] != 0u && key[j] >= thr) {
+        const int e = lane + 32 * j;
+        const double v = rank_value(val(e));
+        int r = 0;
+        for (int e2 = 0; e2 < E && r < k; ++e2) r += ranks_above(rank_value(val(e2)), e2, v, e) ? 1 : 0;
+        if (r < k) {
+          sc->sel_e[r] = e;
+          sc->sel_v[r] = v;
+        }
+      }
+    }
+  }
+  __syncwarp();
+  float ex = 0.0f;
+  if (lane < k) ex = expf((float)(sc->sel_v[lane] - sc->sel_v[0]));
+  const float sum = warp_sum(ex);
+  if (lane < k) {
+    idx_out[lane] = sc->sel_e[lane];
+    gate_out[lane] = ex / sum;
+  }
+  __syncwarp();
+}
+
+// Selection from float64 logits lg[0, E) and their keys in a per-lane key
+// table (key_slot layout, M = topk_m(E) keys a lane), both in shared memory.
+template <int M>
+__device__ __forceinline__ void warp_topk_table_m(const double *lg, const unsigned *keys, int E, int k,
+                                                  int32_t *idx_out, float *gate_out, TopkScratch *sc) {
+  const int lane = threadIdx.x & 31;
+  unsigned key[M];
+#pragma unroll
+  for (int q = 0; q < M / 4; ++q) {
+    const uint4 v = reinterpret_cast<const uint4 *>(keys + lane * M)[q];
+    key[4 * q] = v.x; key[4 * q + 1] = v.y; key[4 * q + 2] = v.z; key[4 * q + 3] = v.w;
+  }
+#pragma unroll
+  for (int j = 0; j < M; ++j)
+    if (lane + 32 * j >= E) key[j] = 0u;
+  warp_topk_keys<M>(key, [&](int e) { return lg[e]; }, E, k, idx_out, gate_out, sc);
+}
+
 template <typename Get>
 __device__ inline void warp_topk_gates_get(Get get, int E, int k, int32_t *idx_out, float *gate_out,
                                            TopkScratch *sc) {

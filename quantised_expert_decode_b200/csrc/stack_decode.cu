@@ -50,12 +50,17 @@ using namespace tile;
 constexpr int SK_NCW = 11;
 constexpr int SK_THREADS = 32 * (SK_NCW + 1);
 constexpr int SK_MAXK = 16;
-constexpr int TRACE_POINTS = 8;
+constexpr int TRACE_POINTS = 12;
 // Trace points of a layer (SM clock of the CTA's consumer thread 0): layer
 // start; top-k done; gate/up tiles start; gate/up tiles done (all consumer
 // warps); first grid barrier passed; down tiles and partials done; second
-// grid barrier passed; logits and normalised x ready (before the top-k).
-enum { TP_START = 0, TP_TOPK, TP_TILES, TP_TILES_DONE, TP_BAR1, TP_DOWN_DONE, TP_BAR2, TP_LOGITS };
+// grid barrier passed; logits and normalised x ready (before the top-k);
+// first gate/up tile landed (consumer warp 0); h limbs landed; down tiles
+// done; z and its sum of squares written (before the next layer's partials).
+enum {
+  TP_START = 0, TP_TOPK, TP_TILES, TP_TILES_DONE, TP_BAR1, TP_DOWN_DONE, TP_BAR2, TP_LOGITS,
+  TP_FIRST_TILE, TP_LIMBS, TP_DOWN_TILES, TP_Z
+};
 constexpr int CONS_BAR = 1;   // the consumer warps
 constexpr int PLAN_BAR = 2;   // consumer warp 0 and the producer warp
 
@@ -94,7 +99,7 @@ struct SkState {
 };
 
 struct SkLayout {
-  size_t ring, dnbuf, wrtbuf, xs, limbs, lsc, logits, ytmp, hloc, bars, state, total;
+  size_t ring, dnbuf, wrtbuf, xs, limbs, lsc, logits, keys, ytmp, hloc, bars, state, total;
 };
 
 // Blocks of h a CTA of a G-CTA grid holds at most (each: a_g and a_u of 32 rows,
@@ -112,10 +117,15 @@ __host__ __device__ inline SkLayout sk_layout(int bits, int E, int H, int I, int
   o.ring = 0;
   o.dnbuf = al128(o.ring + (size_t)nslots * slot_bytes);
   o.wrtbuf = al128(o.dnbuf + (size_t)k * tdn);
-  o.xs = al128(o.wrtbuf + (size_t)16 * E * 4);
+  const size_t wrt_bytes = (size_t)16 * E * 4, key_bytes = (size_t)32 * topk_m(E) * 4;
+  o.xs = al128(o.wrtbuf + (wrt_bytes > key_bytes ? wrt_bytes : key_bytes));
   o.limbs = al128(o.xs + (size_t)H * 4);
   o.lsc = al128(o.limbs + vecs * LIMB_REC);
   o.logits = al128(o.lsc + vecs * 8);
+  // The key table of the top-k is live only in phase A, while the router-row
+  // buffer is idle (its last reads were in the previous layer's phase D, its
+  // next fill is issued after the layer's gate/up tiles): they share memory.
+  o.keys = o.wrtbuf;
   o.ytmp = al128(o.logits + (size_t)E * 8);
   o.hloc = al128(o.ytmp + (size_t)k * 16 * 4);
   o.bars = al128(o.hloc + (size_t)sk_max_local_blocks(k, I, G) * HLOC_BYTES);
@@ -161,8 +171,14 @@ __device__ __forceinline__ bool cons_grid_barrier(const StackArgs &a, SkState *s
 
 // Top-k of logits held in shared memory (kept out of line: it runs once per
 // layer and would otherwise add its registers to the kernel body's).
-__device__ __noinline__ void topk_smem(const double *logits, int E, int k, int32_t *idx, float *gate, TopkScratch *sc) {
-  warp_topk_gates_get([&](int e) { return logits[e]; }, E, k, idx, gate, sc);
+__device__ __noinline__ void topk_smem(const double *logits, const unsigned *keys, int E, int k, int32_t *idx,
+                                       float *gate, TopkScratch *sc) {
+  switch (topk_m(E)) {
+    case 4: warp_topk_table_m<4>(logits, keys, E, k, idx, gate, sc); break;
+    case 8: warp_topk_table_m<8>(logits, keys, E, k, idx, gate, sc); break;
+    case 16: warp_topk_table_m<16>(logits, keys, E, k, idx, gate, sc); break;
+    default: warp_topk_table_m<32>(logits, keys, E, k, idx, gate, sc); break;
+  }
 }
 
 // One warp: h = silu(a_g) * a_u for the 32 rows of block b of selected
@@ -207,6 +223,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
   uint8_t *limbs = smem + lay.limbs;
   float2 *lsc = reinterpret_cast<float2 *>(smem + lay.lsc);
   double *logits = reinterpret_cast<double *>(smem + lay.logits);
+  unsigned *keytab = reinterpret_cast<unsigned *>(smem + lay.keys);
+  const int MK = topk_m(E);
   float *ytmp = reinterpret_cast<float *>(smem + lay.ytmp);
   uint8_t *hloc = smem + lay.hloc;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.bars);
@@ -308,7 +326,13 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
 
   for (int l = 0; l < L; ++l) {
     const int par = l & 1;
-    if (tid == 0) trace_point(a, l, TP_START);
+    if (tid == 0) {
+      trace_point(a, l, TP_START);
+      // points of phases a CTA has no work in stay 0
+      if (a.trace && nitems == 0) a.trace[((size_t)l * gridDim.x + blockIdx.x) * TRACE_POINTS + TP_FIRST_TILE] = 0;
+      if (a.trace && !rows)
+        for (int q = TP_LIMBS; q <= TP_Z; ++q) a.trace[((size_t)l * gridDim.x + blockIdx.x) * TRACE_POINTS + q] = 0;
+    }
     // ------------------------------------------------------------------ A --
     if (!producer && !*(volatile int *)&st->abort) {
       // one batch of loads: sum of squares, z, partial logits, bias
@@ -343,7 +367,11 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
           }
           reinterpret_cast<float4 *>(xs)[q] = v;
         }
-        if (q < E) logits[q] = canon::logit(canon::join((long long)lh[i], (long long)ll[i]), rinv, (double)bv[i]);
+        if (q < E) {
+          const double lv = canon::logit(canon::join((long long)lh[i], (long long)ll[i]), rinv, canon::f2d(bv[i]));
+          logits[q] = lv;
+          keytab[key_slot(q, MK)] = logit_key(lv);
+        }
       }
       for (int q = tid + 4 * nth; q < H / 4; q += nth) {   // larger geometries only
         float4 v = __ldcg(zb + q);
@@ -352,8 +380,11 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
         }
         reinterpret_cast<float4 *>(xs)[q] = v;
       }
-      for (int q = tid + 4 * nth; q < E; q += nth)
-        logits[q] = canon::logit(read_fixed(la + q, la + E + q), rinv, b ? (double)b[q] : 0.0);
+      for (int q = tid + 4 * nth; q < E; q += nth) {
+        const double lv = canon::logit(read_fixed(la + q, la + E + q), rinv, b ? canon::f2d(b[q]) : 0.0);
+        logits[q] = lv;
+        keytab[key_slot(q, MK)] = logit_key(lv);
+      }
       // clear the other parity's accumulators for the next layer (read last by
       // every CTA before the previous barriers)
       unsigned long long *lz = a.lacc + (size_t)(par ^ 1) * 2 * E;
@@ -361,7 +392,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
       named_barrier_sync(CONS_BAR, nth);
       if (tid == 0) trace_point(a, l, TP_LOGITS);
       if (warp == 0) {
-        topk_smem(logits, E, k, st->idx, st->gate, &st->tks);
+        topk_smem(logits, keytab, E, k, st->idx, st->gate, &st->tks);
         if (lane == 0) trace_point(a, l, TP_TOPK);
         // the selection always names k distinct experts in [0, E) (NaN logits
         // rank lowest); checked anyway before any address is formed from it
@@ -469,6 +500,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
     for (int m = warp; warp < NA && m < nitems; m += NA) {
       const int n = nring + m;
       if (!wait_full(n)) break;
+      if (tid == 0 && m == 0) trace_point(a, l, TP_FIRST_TILE);
       const int i = ilo + m, u = i >> 1, mat = i & 1, j = u / I16, r = u % I16;
       const float2 o = tile_dot1<BITS, 1>(ring + (size_t)(n % S) * a.slot_bytes, nblkH, limbs, lsc);
       __syncwarp();
@@ -515,6 +547,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
           set_status(a.status, DEV_TIMEOUT);
           *(volatile int *)&st->abort = 1;
         }
+        if (tid == 0) trace_point(a, l, TP_LIMBS);
       }
       named_barrier_sync(CONS_BAR, nth);
       bool ok = mbar_wait(dnbar, (uint32_t)(l & 1), clock64() + WAIT_BUDGET_CYCLES);
@@ -533,6 +566,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
         *(volatile int *)&st->abort = 1;
       }
       named_barrier_sync(CONS_BAR, nth);
+      if (tid == 0) trace_point(a, l, TP_DOWN_TILES);
       if (ok && warp == 0) {
         if (lane < 16) {
           float y = 0.0f;
@@ -545,6 +579,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
         if (lane == 0) a.ssq[(size_t)(par ^ 1) * H16 + c] = canon::slice_sumsq([&](int i) { return st->ztmp[i]; });
       }
       named_barrier_sync(CONS_BAR, nth);
+      if (tid == 0) trace_point(a, l, TP_Z);
       if (ok && l + 1 < L) {
         if (mbar_wait(wrtbar, (uint32_t)((l + 1) & 1), clock64() + WAIT_BUDGET_CYCLES)) {
           unsigned long long *la = a.lacc + (size_t)(par ^ 1) * 2 * E;

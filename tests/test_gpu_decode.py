@@ -70,6 +70,42 @@ def test_route_multi_token_matches_oracle():
         assert np.max(np.abs(to_np(gate) - og)) < GATE_TOL
 
 
+def test_route_special_activation_values():
+    """Exact zeros, negative zeros, subnormals and large magnitudes in x: every
+    value the router widens to float64 keeps its exact value."""
+    cfg = configs.get(1)
+    Wr_np = gen.router(SEED, cfg, 0)
+    Wr = torch.from_numpy(Wr_np).cuda()
+    rs = np.random.default_rng(3)
+    for T in (1, 4, 8):
+        x_np = gen.tokens(SEED, cfg, 2, T=T).copy()
+        pick = rs.random(x_np.shape)
+        x_np[pick < 0.05] = 0.0
+        x_np[(pick >= 0.05) & (pick < 0.1)] = -0.0
+        sub = (pick >= 0.1) & (pick < 0.15)
+        x_np[sub] = np.float32(1e-40) * np.sign(rs.standard_normal(int(sub.sum()))).astype(np.float32)
+        x_np[(pick >= 0.15) & (pick < 0.16)] *= np.float32(1e4)
+        idx, gate = route(Wr, None, torch.from_numpy(x_np).cuda(), cfg.k)
+        oi, og, _ = moe.route(x_np.astype(np.float64), Wr_np, None, cfg.k)
+        assert np.array_equal(to_np(idx), oi), T
+        assert np.max(np.abs(to_np(gate) - og)) < GATE_TOL
+
+
+@pytest.mark.parametrize("E,H,T", [(100, 384, 3), (33, 128, 1), (1000, 640, 8)])
+def test_route_ragged_geometry_with_bias(E, H, T):
+    """Expert counts that leave lanes of the last 32-expert group idle and
+    hidden sizes whose 16-element slices do not split evenly over the CTAs."""
+    rs = np.random.default_rng(E + H + T)
+    Wr_np = (0.05 * rs.standard_normal((E, H))).astype(np.float32)
+    b_np = (0.1 * rs.standard_normal(E)).astype(np.float32)
+    x_np = rs.standard_normal((T, H)).astype(np.float32)
+    k = min(10, E)
+    idx, gate = route(torch.from_numpy(Wr_np).cuda(), torch.from_numpy(b_np).cuda(), torch.from_numpy(x_np).cuda(), k)
+    oi, og, _ = moe.route(x_np.astype(np.float64), Wr_np, b_np, k)
+    assert np.array_equal(to_np(idx), oi)
+    assert np.max(np.abs(to_np(gate) - og)) < GATE_TOL
+
+
 def test_route_exact_ties_go_to_lower_index():
     cfg = configs.get(0)
     Wr_np = gen.router(SEED, cfg, 0).copy()

@@ -206,9 +206,16 @@ def test_fused_phase_trace_is_ordered_and_layer_times_add_up():
     torch.cuda.synchronize()
     assert st.status() == 0
     tr = st.phase_trace()
-    assert tr.shape[0] == 4 and tr.shape[2] == 8
+    assert tr.shape[0] == 4 and tr.shape[2] == 12
     assert (np.diff(tr[:, :, :7], axis=2) >= 0).all()
     assert ((tr[:, :, 0] <= tr[:, :, 7]) & (tr[:, :, 7] <= tr[:, :, 1])).all()   # logits ready, then the top-k
+    busy = tr[:, :, 8] != 0                               # CTAs with gate/up tiles in the layer
+    assert busy.any()
+    assert ((tr[:, :, 2] <= tr[:, :, 8]) & (tr[:, :, 8] <= tr[:, :, 3]))[busy].all()   # a tile lands while C runs
+    rows = np.arange(tr.shape[1]) < cfg.H // 16          # CTAs that own output rows run phase D
+    d = tr[:, rows]
+    assert ((d[:, :, 4] <= d[:, :, 9]) & (d[:, :, 9] <= d[:, :, 10]) & (d[:, :, 10] <= d[:, :, 11])
+            & (d[:, :, 11] <= d[:, :, 5])).all()
     route_ms, ffn_ms = st.layer_times()
     assert all(r >= 0 for r in route_ms) and all(f > 0 for f in ffn_ms)
     plain = DecodeStack(layers, routers, None, 1, cfg.k, cfg.eps)

@@ -2,8 +2,10 @@
 restated.
 
 Expert e sits on lane e % 32 of a warp. Every float64 logit gets a 32-bit key:
-the top 32 bits of its float64 pattern (-0 taken as +0), made order-preserving
-as an unsigned integer. The threshold is the k-th largest of the 32 per-lane maximum keys
+the top 32 bits of its float64 pattern, made order-preserving as an unsigned
+integer; a high word of 0x80000000 (-0 and the smallest negative subnormals)
+is taken as that of +0, and NaN as -infinity (its rank). The threshold is the
+k-th largest of the 32 per-lane maximum keys
 (ties by lane); every key at or above it is a candidate, and the exact ranking
 (logit descending, lower index on ties) runs on the candidates only. The
 candidate set must contain the exact top-k for any logits; it should stay small
@@ -14,10 +16,15 @@ import pytest
 
 def keys(logits):
     f = np.asarray(logits, dtype=np.float64)
-    f = np.where(f == 0, 0.0, f)
-    b = f.view(np.uint64)
-    o = np.where(b & np.uint64(1 << 63), ~b, b | np.uint64(1 << 63))
-    return o >> np.uint64(32)
+    f = np.where(np.isnan(f), -np.inf, f)
+    hi = (f.view(np.uint64) >> np.uint64(32)).astype(np.uint64)
+    hi = np.where(hi == np.uint64(0x80000000), np.uint64(0), hi)
+    return np.where(hi & np.uint64(0x80000000), ~hi & np.uint64(0xFFFFFFFF), hi | np.uint64(0x80000000))
+
+
+def rank_key(v):
+    """Selection order: value descending (NaN lowest), index ascending."""
+    return -np.inf if np.isnan(v) else v
 
 
 def candidates(logits, k):
@@ -32,10 +39,10 @@ def candidates(logits, k):
 
 
 def exact_top_k(logits, k):
-    return sorted(range(len(logits)), key=lambda e: (-logits[e], e))[:k]
+    return sorted(range(len(logits)), key=lambda e: (-rank_key(logits[e]), e))[:k]
 
 
-@pytest.mark.parametrize("kind", ["router", "ties", "degenerate", "signed_zero", "one_lane"])
+@pytest.mark.parametrize("kind", ["router", "ties", "degenerate", "signed_zero", "one_lane", "tiny", "nan"])
 def test_candidates_contain_the_exact_top_k(kind):
     rs = np.random.default_rng(5)
     for trial in range(300):
@@ -51,6 +58,13 @@ def test_candidates_contain_the_exact_top_k(kind):
         elif kind == "signed_zero":
             v = np.where(rs.random(E) < 0.5, -0.0, 0.0)
             v[rs.integers(0, E, 2)] = -1.0
+        elif kind == "tiny":
+            # negative subnormals whose high word is 0x80000000 share +0's key
+            v = np.where(rs.random(E) < 0.5, -5e-324 * rs.integers(1, 1000, E), 0.0)
+            v[rs.integers(0, E, 3)] = 1e-310
+        elif kind == "nan":
+            v = rs.standard_normal(E)
+            v[rs.integers(0, E, max(1, E // 4))] = np.nan
         else:
             v = rs.standard_normal(E)
             v[np.arange(0, E, 32)] += 10.0       # the largest logits all on lane 0
