@@ -81,6 +81,25 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       : "memory");
 }
 
+// L2 policy for bytes read once per pass (expert and router weights): evicted
+// first, so that the streamed weights do not push the kernels' code, the
+// activations and the small shared buffers out of L2.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// bulk_g2s with an L2 cache policy (l2_evict_first for streamed weights).
+__device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                              uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
 // Integer tensor-core MMA: D[16x8] += A[16x32] (u8 codes) * B[32x8] (s8 limbs).
 // Fragments per lane (g = lane/4, t = lane%4):
 //   a0: A[g][4t..4t+3]   a1: A[g+8][4t..4t+3]   a2: A[g][16+4t..]   a3: A[g+8][16+4t..]

@@ -401,6 +401,13 @@ __device__ __forceinline__ void quant_chunk_inl(float4 v, uint8_t *limbs_vec, fl
   if ((lane & 7) == 0) lsc_vec[blk] = make_float2(s, __fmul_rn(s, (float)sx));
 }
 
+// Two chunks (see quant_chunk) in one call.
+__device__ __noinline__ void quant_chunk2(float4 v0, uint8_t *limbs0, float2 *lsc0, int chunk0, float4 v1,
+                                          uint8_t *limbs1, float2 *lsc1, int chunk1, int lane) {
+  quant_chunk_inl(v0, limbs0, lsc0, chunk0, lane);
+  quant_chunk_inl(v1, limbs1, lsc1, chunk1, lane);
+}
+
 // Quantise activation vectors of 128-element chunks; task = vec * nch + chunk.
 // Each warp first issues the loads of up to MB tasks, then quantises them, so a
 // warp pays one memory latency per MB tasks.
@@ -414,12 +421,15 @@ __device__ __forceinline__ void quant_tasks(int ntask, int nch, int nblk, uint8_
       const int task = base + i * NW;
       if (task < ntask) v[i] = load(task / nch, task % nch);
     }
+    // two chunks a call, so that their shuffle chains overlap
 #pragma unroll
-    for (int i = 0; i < MB; ++i) {
-      const int task = base + i * NW;
-      if (task < ntask) {
-        const int vec = task / nch;
-        quant_chunk(v[i], limbs + (size_t)vec * nblk * LIMB_REC, lsc + (size_t)vec * nblk, task % nch, lane);
+    for (int i = 0; i < MB; i += 2) {
+      const int t0 = base + i * NW, t1 = base + (i + 1) * NW;
+      if (t0 < ntask) {
+        const int u1 = t1 < ntask ? t1 : t0;   // a lone chunk is quantised twice into the same place
+        quant_chunk2(v[i], limbs + (size_t)(t0 / nch) * nblk * LIMB_REC, lsc + (size_t)(t0 / nch) * nblk, t0 % nch,
+                     t1 < ntask ? v[i + 1] : v[i], limbs + (size_t)(u1 / nch) * nblk * LIMB_REC,
+                     lsc + (size_t)(u1 / nch) * nblk, u1 % nch, lane);
       }
     }
   }

@@ -30,6 +30,8 @@ constexpr int FD_THREADS = 32 * (NCW + 1); // + one producer warp
 constexpr int FD_MAXT = 8;
 constexpr int FD_MAXK = 16;
 constexpr int FD_MAXP = FD_MAXT * FD_MAXK; // (token, slot) pairs
+constexpr int FD_MAXE = 1024;              // experts a layer
+static_assert(FD_MAXP % 32 == 0 && FD_MAXT <= 8, "plan layout: 32-pair rows, one byte of tokens an expert");
 constexpr int CONSUMER_BAR = 1;            // named barrier id for the consumer warps
 struct Plan {
   int err;
@@ -41,30 +43,164 @@ struct Plan {
   int ptok[FD_MAXP];
   int pslot[FD_MAXP];
   float pgate[FD_MAXP];
-  int sidx[FD_MAXP];
-  float sgate[FD_MAXP];
-  unsigned bm[32];
-  int vids[NCW][FD_MAXT];  // per consumer warp: limb-region vectors of the current item
-  int lo1, hi1, lo2, hi2;  // this CTA's gate/up and down item ranges
+  int cw[FD_MAXP + 1];      // exclusive prefix of tile_cost(nt[u])
+  unsigned tm[FD_MAXE / 4]; // per expert, one byte: the tokens (bits) routed to it
+  int wbase[32];            // experts in the bitmap words before word w
+  unsigned bm[32];          // bitmap of the routed experts
+  int vids[NCW][FD_MAXT];   // per consumer warp: limb-region vectors of the current item
+  int lo1, hi1, lo2, hi2;   // this CTA's gate/up and down item ranges
 };
 
-// Relative cost of a tile whose expert serves n tokens: the bytes (the same
-// for every tile) plus the tensor-core and epilogue work of the tile-dot
-// variant for n vectors (1, 2, 4 or 8), which grows about linearly above two.
-__device__ __forceinline__ int tile_cost(int n) { return n <= 1 ? 4 : n <= 2 ? 5 : n <= 4 ? 8 : 14; }
+// Relative cost of a tile whose expert serves n tokens, from the measured
+// cycles of one warp's tile dot product: the variants for 2, 4 and 8 vectors
+// (tile_dot<NP>) take about the same time, about twice the 1-vector one.
+__device__ __forceinline__ int tile_cost(int n) { return n <= 1 ? 1 : 2; }
 
-// First item whose starting cost is at least `target`, items numbered expert
-// by expert (per_expert items each, all at the expert's tile cost).
+__device__ __forceinline__ int warp_excl_scan(int v, int &total) {
+  const int lane = threadIdx.x & 31;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  total = __shfl_sync(0xffffffffu, incl, 31);
+  return incl - v;
+}
+
+// One warp. Items are numbered expert by expert, per_expert items an expert,
+// each at its expert's tile cost (cost prefix cw); returns the first item
+// whose starting cost is at least `target` (U * per_expert if none). Expert u
+// holds that item when it is the first with target <= acc_u + (per_expert - 1)
+// w_u, acc_u = per_expert cw[u]: the item is then u's first if target <= acc_u,
+// else the ceil((target - acc_u) / w_u)-th.
 __device__ int item_at_cost(const Plan *pl, int U, int per_expert, long long target) {
-  long long acc = 0;
-  for (int u = 0; u < U; ++u) {
-    const int w = tile_cost(pl->nt[u]);
-    if (target <= acc) return u * per_expert;
-    const long long i = (target - acc + w - 1) / w;
-    if (i < per_expert) return u * per_expert + (int)i;
-    acc += (long long)per_expert * w;
+  const int lane = threadIdx.x & 31;
+  for (int u0 = 0; u0 < U; u0 += 32) {
+    const int u = u0 + lane;
+    bool hit = false;
+    long long acc = 0;
+    int w = 1;
+    if (u < U) {
+      w = tile_cost(pl->nt[u]);
+      acc = (long long)per_expert * pl->cw[u];
+      hit = target <= acc + (long long)(per_expert - 1) * w;
+    }
+    const unsigned b = __ballot_sync(0xffffffffu, hit);
+    if (b) {
+      const int src = __ffs(b) - 1;
+      const long long acc0 = __shfl_sync(0xffffffffu, acc, src);
+      const int w0 = __shfl_sync(0xffffffffu, w, src);
+      const int ui = u0 + src;
+      return target <= acc0 ? ui * per_expert : ui * per_expert + (int)((target - acc0 + w0 - 1) / w0);
+    }
   }
   return U * per_expert;
+}
+
+// Route table -> unique experts (ascending), their tokens (ascending) and
+// slots, and the tile-cost prefix; one warp, every step spread over the lanes.
+__device__ void build_plan(const int32_t *idx, const float *gate, int T, int k, int E, int32_t *status, Plan *pl) {
+  const int lane = threadIdx.x & 31;
+  const int P = T * k;
+  for (int w = lane; w < FD_MAXE / 4; w += 32) pl->tm[w] = 0u;
+  int pe[FD_MAXP / 32];
+  float pg[FD_MAXP / 32];
+#pragma unroll
+  for (int i = 0; i < FD_MAXP / 32; ++i) {
+    const int p = lane + 32 * i;
+    pe[i] = p < P ? idx[p] : 0;
+    pg[i] = p < P ? gate[p] : 0.0f;
+  }
+  __syncwarp();
+  int bad = 0;
+#pragma unroll
+  for (int i = 0; i < FD_MAXP / 32; ++i) {
+    const int p = lane + 32 * i;
+    if (p >= P) continue;
+    const int e = pe[i];
+    if (e < 0 || e >= E) {
+      bad = DEV_BAD_INDEX;
+      continue;
+    }
+    const unsigned bit = 1u << ((e & 3) * 8 + p / k);
+    if (atomicOr(&pl->tm[e >> 2], bit) & bit) bad = DEV_DUP_INDEX;   // the token names e twice
+  }
+  const unsigned badmask = __ballot_sync(0xffffffffu, bad != 0);
+  if (badmask) {
+    const int code = __shfl_sync(0xffffffffu, bad, __ffs(badmask) - 1);
+    if (lane == 0) {
+      pl->err = code;
+      set_status(status, code);
+    }
+    __syncwarp();
+    return;
+  }
+  __syncwarp();
+  // bitmap word `lane`: experts 32 lane .. 32 lane + 31
+  unsigned word = 0u;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const unsigned m = pl->tm[lane * 8 + q];
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+      if ((m >> (8 * b)) & 0xffu) word |= 1u << (4 * q + b);
+  }
+  int U;
+  const int wb = warp_excl_scan(__popc(word), U);
+  pl->bm[lane] = word;
+  pl->wbase[lane] = wb;
+  for (unsigned w2 = word, r = wb; w2; w2 &= w2 - 1u, ++r) {
+    const int e = lane * 32 + __ffs(w2) - 1;
+    pl->ue[r] = e;
+    pl->nt[r] = __popc((pl->tm[e >> 2] >> ((e & 3) * 8)) & 0xffu);
+  }
+  __syncwarp();
+  // token and cost prefixes over the unique experts (4 a lane, in order)
+  int nt4[FD_MAXP / 32], c4[FD_MAXP / 32], ntl = 0, cl = 0;
+#pragma unroll
+  for (int i = 0; i < FD_MAXP / 32; ++i) {
+    const int u = lane * (FD_MAXP / 32) + i;
+    nt4[i] = u < U ? pl->nt[u] : 0;
+    c4[i] = u < U ? tile_cost(nt4[i]) : 0;
+    ntl += nt4[i];
+    cl += c4[i];
+  }
+  int ntot, ctot;
+  int nb = warp_excl_scan(ntl, ntot), cb = warp_excl_scan(cl, ctot);
+#pragma unroll
+  for (int i = 0; i < FD_MAXP / 32; ++i) {
+    const int u = lane * (FD_MAXP / 32) + i;
+    if (u < U) {
+      pl->pbase[u] = nb;
+      pl->cw[u] = cb;
+    }
+    nb += nt4[i];
+    cb += c4[i];
+  }
+  if (lane == 0) {
+    pl->pbase[U] = ntot;
+    pl->cw[U] = ctot;
+    pl->U = U;
+    pl->err = 0;
+    pl->abort = 0;
+  }
+  __syncwarp();
+  // each pair's place among its expert's tokens (token order)
+#pragma unroll
+  for (int i = 0; i < FD_MAXP / 32; ++i) {
+    const int p = lane + 32 * i;
+    if (p < P) {
+      const int e = pe[i], t = p / k;
+      const int u = pl->wbase[e >> 5] + __popc(pl->bm[e >> 5] & ((1u << (e & 31)) - 1u));
+      const unsigned toks = (pl->tm[e >> 2] >> ((e & 3) * 8)) & 0xffu;
+      const int q = pl->pbase[u] + __popc(toks & ((1u << t) - 1u));
+      pl->ptok[q] = t;
+      pl->pslot[q] = p % k;
+      pl->pgate[q] = pg[i];
+    }
+  }
+  __syncwarp();
 }
 
 struct FfnArgs {
@@ -99,108 +235,6 @@ __host__ __device__ inline SmemLayout smem_layout(int nslots, int slot_bytes, in
   return o;
 }
 
-// Route table -> unique experts (ascending), their tokens (ascending) and slots.
-__device__ void build_plan(const FfnArgs &a, Plan *pl) {
-  const int lane = threadIdx.x & 31;
-  const int P = a.T * a.k;
-  pl->bm[lane] = 0u;
-  for (int p = lane; p < P; p += 32) {
-    pl->sidx[p] = a.idx[p];
-    pl->sgate[p] = a.gate[p];
-  }
-  __syncwarp();
-  int bad = 0;
-  for (int p = lane; p < P; p += 32) {
-    int e = pl->sidx[p];
-    if (e < 0 || e >= a.E) {
-      bad = DEV_BAD_INDEX;
-      continue;
-    }
-    int t = p / a.k, j = p % a.k;
-    for (int j2 = 0; j2 < j; ++j2)
-      if (pl->sidx[t * a.k + j2] == e) bad = DEV_DUP_INDEX;
-    atomicOr(&pl->bm[e >> 5], 1u << (e & 31));
-  }
-  unsigned badmask = __ballot_sync(0xffffffffu, bad != 0);
-  if (badmask) {
-    int first = __ffs(badmask) - 1;
-    int code = __shfl_sync(0xffffffffu, bad, first);
-    if (lane == 0) {
-      pl->err = code;
-      set_status(a.status, code);
-    }
-    return;
-  }
-  __syncwarp();
-  unsigned word = pl->bm[lane];
-  int cnt = __popc(word);
-  int incl = cnt;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  int wbase = incl - cnt;
-  int U = __shfl_sync(0xffffffffu, incl, 31);
-  {
-    unsigned w2 = word;
-    int r = wbase;
-    while (w2) {
-      int b = __ffs(w2) - 1;
-      w2 &= w2 - 1u;
-      pl->ue[r] = lane * 32 + b;
-      pl->nt[r] = 0;
-      ++r;
-    }
-  }
-  __syncwarp();
-  // per pair: expert rank u and position among the expert's tokens (token order)
-  int pu[FD_MAXP / 32], ppos[FD_MAXP / 32];
-#pragma unroll
-  for (int i = 0; i < FD_MAXP / 32; ++i) {
-    int p = lane + 32 * i;
-    pu[i] = -1;
-    if (p < P) {
-      int e = pl->sidx[p];
-      int wi = e >> 5;
-      unsigned wbits = pl->bm[wi];
-      int base = 0;  // experts in the bitmap words before wi
-      for (int q = 0; q < wi; ++q) base += __popc(pl->bm[q]);
-      pu[i] = base + __popc(wbits & ((1u << (e & 31)) - 1u));
-      int t = p / a.k;
-      int pos = 0;
-      for (int t2 = 0; t2 < t; ++t2)
-        for (int j2 = 0; j2 < a.k; ++j2) pos += (pl->sidx[t2 * a.k + j2] == e) ? 1 : 0;
-      ppos[i] = pos;
-      atomicAdd(&pl->nt[pu[i]], 1);
-    }
-  }
-  __syncwarp();
-  if (lane == 0) {
-    int s = 0;
-    for (int u = 0; u < U; ++u) {
-      pl->pbase[u] = s;
-      s += pl->nt[u];
-    }
-    pl->pbase[U] = s;
-    pl->U = U;
-    pl->err = 0;
-    pl->abort = 0;
-  }
-  __syncwarp();
-#pragma unroll
-  for (int i = 0; i < FD_MAXP / 32; ++i) {
-    int p = lane + 32 * i;
-    if (p < P) {
-      int q = pl->pbase[pu[i]] + ppos[i];
-      pl->ptok[q] = p / a.k;
-      pl->pslot[q] = p % a.k;
-      pl->pgate[q] = pl->sgate[p];
-    }
-  }
-  __syncwarp();
-}
-
 template <int BITS>
 __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -230,17 +264,22 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
   // Everything above overlaps the previous kernel; idx, gate and x are its outputs.
   pdl_wait();
   if (warp == 0) {
-    build_plan(a, pl);
+    build_plan(a.idx, a.gate, a.T, a.k, a.E, a.status, pl);
     // split both phases' items over the CTAs by cost, not by count: a tile
     // shared by 8 tokens costs several times a single-token tile
-    if (lane == 0 && !pl->err) {
-      long long W = 0;
-      for (int u = 0; u < pl->U; ++u) W += tile_cost(pl->nt[u]);
-      const long long W1 = W * 2 * I16, W2 = W * H16;
-      pl->lo1 = item_at_cost(pl, pl->U, 2 * I16, W1 * blockIdx.x / G);
-      pl->hi1 = item_at_cost(pl, pl->U, 2 * I16, W1 * (blockIdx.x + 1) / G);
-      pl->lo2 = item_at_cost(pl, pl->U, H16, W2 * blockIdx.x / G);
-      pl->hi2 = item_at_cost(pl, pl->U, H16, W2 * (blockIdx.x + 1) / G);
+    if (!pl->err) {
+      const int U = pl->U;
+      const long long W = pl->cw[U], W1 = W * 2 * I16, W2 = W * H16;
+      const int lo1 = item_at_cost(pl, U, 2 * I16, W1 * blockIdx.x / G);
+      const int hi1 = item_at_cost(pl, U, 2 * I16, W1 * (blockIdx.x + 1) / G);
+      const int lo2 = item_at_cost(pl, U, H16, W2 * blockIdx.x / G);
+      const int hi2 = item_at_cost(pl, U, H16, W2 * (blockIdx.x + 1) / G);
+      if (lane == 0) {
+        pl->lo1 = lo1;
+        pl->hi1 = hi1;
+        pl->lo2 = lo2;
+        pl->hi2 = hi2;
+      }
     }
   }
   __syncthreads();
@@ -258,6 +297,7 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
     // its barrier, which is what a parity wait can tell apart.
     int my_last = -1;
     bool aborted = false;
+    const uint64_t pol = l2_evict_first();
     for (int n = lane; lane < S && n < ntot; n += S) {
       const int s = n % S, it = n / S;
       if (n >= S) {
@@ -284,7 +324,7 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
         bytes = (uint32_t)tdn;
       }
       mbar_arrive_expect_tx(&full[s], bytes);
-      bulk_g2s(ring + (size_t)s * a.slot_bytes, src, bytes, &full[s]);
+      bulk_g2s_hint(ring + (size_t)s * a.slot_bytes, src, bytes, &full[s], pol);
       my_last = n;
     }
     // never leave with copies in flight: wait for this lane's copies whose slot

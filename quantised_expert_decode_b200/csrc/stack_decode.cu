@@ -426,6 +426,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
       // CTA's down tiles; lane 30: next layer's router rows.
       fence_proxy_async();   // ring memory was last read with ordinary loads
       const uint8_t *gu = a.gu[l];
+      const uint64_t pol = l2_evict_first();
       const int first = nring + ((lane - nring % S) % S + S) % S;  // first item of slot `lane`
       for (int n = first; lane < S && n < nring + nitems; n += S) {
         const int s = n % S;
@@ -444,7 +445,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
         const int j = u / I16, r = u % I16;
         const uint8_t *src = gu + (((size_t)st->idx[j] * 2 + mat) * I16 + r) * (size_t)tgu;
         mbar_arrive_expect_tx(&full[s], (uint32_t)tgu);
-        bulk_g2s(ring + (size_t)s * a.slot_bytes, src, (uint32_t)tgu, &full[s]);
+        bulk_g2s_hint(ring + (size_t)s * a.slot_bytes, src, (uint32_t)tgu, &full[s], pol);
       }
       if ((lane == 31 || lane == 30) && rows) {
         // The down tiles and the next layer's router rows are needed only after
@@ -471,12 +472,12 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
           const uint8_t *dn = a.dn[l];
           mbar_arrive_expect_tx(dnbar, (uint32_t)(k * tdn));
           for (int j = 0; j < k; ++j)
-            bulk_g2s(dnbuf + (size_t)j * tdn, dn + ((size_t)st->idx[j] * H16 + c) * (size_t)tdn, (uint32_t)tdn,
-                     dnbar);
+            bulk_g2s_hint(dnbuf + (size_t)j * tdn, dn + ((size_t)st->idx[j] * H16 + c) * (size_t)tdn, (uint32_t)tdn,
+                          dnbar, pol);
         }
         if (ok && lane == 30 && l + 1 < L) {
           mbar_arrive_expect_tx(wrtbar, (uint32_t)(16 * E * 4));
-          bulk_g2s(wrtbuf, a.wrt + ((size_t)(l + 1) * H + r0) * E, (uint32_t)(16 * E * 4), wrtbar);
+          bulk_g2s_hint(wrtbuf, a.wrt + ((size_t)(l + 1) * H + r0) * E, (uint32_t)(16 * E * 4), wrtbar, pol);
         }
       }
       nring += nitems;
