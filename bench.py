@@ -495,6 +495,7 @@ def measure_stack(args, cfg, seed=SEED, full=True):
         phases = {n: float(v) / mhz for n, v in zip(names, rel)}
         # the slowest CTA's gate/up tiles hold the first grid barrier
         phases["tiles_done_max_cta"] = float(np.max(tr[:, :, 3] - tr[:, :, 0], axis=1).mean()) / mhz
+        phases["down_done_max_cta"] = float(np.max(tr[:, rows, 5] - tr[:, rows, 0], axis=1).mean()) / mhz
     tstack.close()
     del layers, routers, biases, xs
     free_device()

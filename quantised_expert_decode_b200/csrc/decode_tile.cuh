@@ -38,6 +38,16 @@ __device__ __forceinline__ float i2f_small(int v) {
 // fraction of the rate and were the busiest pipe of the tile loop).
 __device__ __forceinline__ float limb_pair(int hi, int lo) { return fmaf(i2f_small(hi), 256.0f, i2f_small(lo)); }
 
+// The same value for a tile of BITS-bit codes. With 2-bit codes each block sum
+// is at most 32 * 3 * 128 = 12,288 in magnitude, so hi * 256 + lo stays below
+// 2^22 and forms exactly in integers, then converts through the magic number
+// in one step (three operations instead of five).
+template <int BITS>
+__device__ __forceinline__ float limb_pair_b(int hi, int lo) {
+  if (BITS == 2) return i2f_small(hi * 256 + lo);
+  return limb_pair(hi, lo);
+}
+
 __device__ __forceinline__ float h2f(uint32_t bits16) { return __half2float(__ushort_as_half((unsigned short)bits16)); }
 
 // Quantise a 128-element chunk (4 blocks of 32) held one float4 per lane: lane
@@ -214,8 +224,8 @@ __device__ __noinline__ Acc tile_dot(const uint8_t *tile, int nblk, const uint8_
       for (int q = 0; q < NQ; ++q) {
         if (ov[q] >= 0) {
           const int bo = c * 4 + sb * BS + obeta;
-          const float v0 = limb_pair(D[sb][q][0], D[sb][q][1]);
-          const float v1 = limb_pair(D[sb][q][2], D[sb][q][3]);
+          const float v0 = limb_pair_b<BITS>(D[sb][q][0], D[sb][q][1]);
+          const float v1 = limb_pair_b<BITS>(D[sb][q][2], D[sb][q][3]);
           const float2 ss = lsc[(size_t)ov[q] * nblk + bo];
           const uint2 dm = *reinterpret_cast<const uint2 *>(sbase + (bo * 8 + g) * 8);
           const float sw = ss.x * wgt;
@@ -354,8 +364,8 @@ __device__ __noinline__ float2 tile_dot1(const uint8_t *tile, int nblk, const ui
 #pragma unroll
         for (int sb = 0; sb < 2; ++sb) {
           const int bo = (c0 + ch) * 4 + sb * 2 + oP;
-          const float v0 = limb_pair(D[ch][sb][0], D[ch][sb][1]);
-          const float v1 = limb_pair(D[ch][sb][2], D[ch][sb][3]);
+          const float v0 = limb_pair_b<BITS>(D[ch][sb][0], D[ch][sb][1]);
+          const float v1 = limb_pair_b<BITS>(D[ch][sb][2], D[ch][sb][3]);
           const float2 ss = lsc[bo];
           const uint2 dm = *reinterpret_cast<const uint2 *>(sbase + (bo * 8 + g) * 8);
           const float sw = ss.x * wgt;

@@ -51,10 +51,11 @@ struct Plan {
   int lo1, hi1, lo2, hi2;   // this CTA's gate/up and down item ranges
 };
 
-// Relative cost of a tile whose expert serves n tokens, from the measured
-// cycles of one warp's tile dot product: the variants for 2, 4 and 8 vectors
-// (tile_dot<NP>) take about the same time, about twice the 1-vector one.
-__device__ __forceinline__ int tile_cost(int n) { return n <= 1 ? 1 : 2; }
+// Relative cost of a tile whose expert serves n tokens. With a warp per SM
+// sub-partition or more the tiles are issue-bound, so the cost follows the
+// instructions of the tile-dot variant for n vectors (NP = 1, 2, 4, 8: about
+// 15, 23, 46 and 90 a block and lane).
+__device__ __forceinline__ int tile_cost(int n) { return n <= 1 ? 2 : n <= 2 ? 3 : n <= 4 ? 6 : 12; }
 
 __device__ __forceinline__ int warp_excl_scan(int v, int &total) {
   const int lane = threadIdx.x & 31;

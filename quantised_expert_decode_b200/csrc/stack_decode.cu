@@ -342,6 +342,10 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
       float4 zv[4];
       unsigned long long lh[4], ll[4];
       float bv[4];
+      const double *sq = a.ssq + (size_t)par * H16;
+      double sv[4];   // this lane's first slice sums of squares (decode_canon.cuh's order)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) sv[m] = (l > 0 && lane + 32 * m < H16) ? __ldcg(sq + lane + 32 * m) : 0.0;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int q = tid + i * nth;
@@ -353,9 +357,10 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
         }
       }
       // every warp adds the slice sums of squares itself (same order, same value)
-      const double *sq = a.ssq + (size_t)par * H16;
       const double rinv =
-          l > 0 ? canon::norm_rinv(canon::warp_sumsq([&](int cc) { return __ldcg(sq + cc); }, H16), H, a.eps) : 1.0;
+          l > 0 ? canon::norm_rinv(canon::warp_sum_slices<4>(sv, [&](int cc) { return __ldcg(sq + cc); }, H16), H,
+                                   a.eps)
+                : 1.0;
       const float inv = __double2float_rn(rinv);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {

@@ -80,3 +80,16 @@ def test_limb_pair_recombination_is_exact_for_4_bit_codes():
     # 24 bits: the float64 evaluation is the exact value, and it survives float32
     fused = i2f_small(hi).astype(np.float64) * 256.0 + i2f_small(lo).astype(np.float64)
     assert np.array_equal(fused.astype(np.float32).astype(np.int64), exact)
+
+
+def test_limb_pair_recombination_is_exact_in_one_step_for_2_bit_codes():
+    """With 2-bit codes the epilogue forms hi * 256 + lo in integers and
+    converts it through the magic number 1.5 * 2^23 in one step, which is exact
+    only below 2^22: each block sum is at most 32 * 3 * 128 = 12,288."""
+    bound = 32 * 3 * 128
+    rs = np.random.default_rng(3)
+    hi = np.concatenate([[-bound, bound, 0], rs.integers(-bound, bound + 1, 100000)])
+    lo = np.concatenate([[-bound, bound, 0], rs.integers(-bound, bound + 1, 100000)])
+    v = hi.astype(np.int64) * 256 + lo
+    assert np.abs(v).max() < 2 ** 22
+    assert np.array_equal(i2f_small(v).astype(np.int64), v)
