@@ -110,6 +110,16 @@ __device__ __forceinline__ double slice_dot(W w, Z z) {
   return p;
 }
 
+// slice_dot with the activations already widened, zd[i] = f2d(z(i)): the same
+// value, for loops that reuse one slice of z over many router rows.
+template <class W>
+__device__ __forceinline__ double slice_dot_wide(W w, const double (&zd)[SLICE]) {
+  double p = 0.0;
+#pragma unroll
+  for (int i = 0; i < SLICE; ++i) p = fma(f2d(w(i)), zd[i], p);
+  return p;
+}
+
 // Sum of squares of one slice.
 template <class Z>
 __device__ __forceinline__ double slice_sumsq(Z z) {

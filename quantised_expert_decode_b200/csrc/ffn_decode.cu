@@ -213,6 +213,8 @@ struct FfnArgs {
   float *y;
   float *abuf;    // [P][2][I]
   float *part;    // [T][k][H]
+  uint8_t *xlimbs;  // [T][H/32][LIMB_REC] limbs of x, quantised once across the grid
+  float2 *xlsc;     // [T][H/32] their block scales
   unsigned *bar;  // grid barrier counter
   int32_t *status;
   int T, k, E, H, I;
@@ -229,7 +231,7 @@ struct SmemLayout {
 __host__ __device__ inline SmemLayout smem_layout(int nslots, int slot_bytes, int limb_bytes, int lsc_count) {
   SmemLayout o;
   o.bars = (size_t)nslots * slot_bytes;                       // slot_bytes is a multiple of 128
-  o.plan = (o.bars + (size_t)nslots * 16 + 15) & ~(size_t)15;
+  o.plan = (o.bars + (size_t)nslots * 16 + 8 + 15) & ~(size_t)15;   // full, empty per slot; the x-limb barrier
   o.limbs = (o.plan + sizeof(Plan) + 127) & ~(size_t)127;
   o.lsc = (o.limbs + (size_t)limb_bytes + 15) & ~(size_t)15;
   o.total = o.lsc + (size_t)lsc_count * 8;
@@ -245,6 +247,7 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
   uint8_t *ring = smem;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.bars);
   uint64_t *empty = full + S;
+  uint64_t *xbar = empty + S;
   Plan *pl = reinterpret_cast<Plan *>(smem + lay.plan);
   uint8_t *limbs = smem + lay.limbs;
   float2 *lsc = reinterpret_cast<float2 *>(smem + lay.lsc);
@@ -260,6 +263,7 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
+    mbar_init(xbar, 1);
     fence_mbar_init();
   }
   // Everything above overlaps the previous kernel; idx, gate and x are its outputs.
@@ -342,13 +346,43 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
 
   // ---------------------------------------------------------------- consumers --
   const int nth = NCW * 32;
-  // activation limbs of the T tokens
+  // Grid barrier of the consumer threads (the producer never joins one).
+  auto grid_sync = [&]() {
+    named_barrier_sync(CONSUMER_BAR, nth);
+    if (tid == 0) {
+      if (!*(volatile int *)&pl->abort && !grid_barrier_one_thread(a.bar, G)) {
+        set_status(a.status, DEV_TIMEOUT);
+        *(volatile int *)&pl->abort = 1;
+      }
+      __threadfence();
+    }
+    named_barrier_sync(CONSUMER_BAR, nth);
+  };
+
+  // Activation limbs of the T tokens: the 128-element chunks are spread over
+  // the grid (chunk task of CTA task % G), quantised once into the workspace,
+  // and after a grid barrier every CTA copies all of them into shared memory.
   {
-    const int nch = H / 128;
-    const float *x = a.x;
-    quant_tasks<NCW, 16>(a.T * nch, nch, nblkH, limbs, lsc, warp, lane, [&](int t, int c) {
-      return __ldcg(reinterpret_cast<const float4 *>(x + (size_t)t * H + c * 128) + lane);
-    });
+    const int nch = H / 128, ntask = a.T * nch;
+    for (int task = blockIdx.x + G * warp; task < ntask; task += G * NCW) {
+      const int t = task / nch, c = task % nch;
+      const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.x + (size_t)t * H + c * 128) + lane);
+      quant_chunk(v, a.xlimbs + (size_t)t * nblkH * LIMB_REC, a.xlsc + (size_t)t * nblkH, c, lane);
+    }
+  }
+  grid_sync();
+  {
+    const uint32_t lb = (uint32_t)(a.T * nblkH * LIMB_REC), sb = (uint32_t)(a.T * nblkH * 8);
+    if (tid == 0) {
+      fence_proxy_async();   // the limbs were written with ordinary stores
+      mbar_arrive_expect_tx(xbar, lb + sb);
+      bulk_g2s(limbs, a.xlimbs, lb, xbar);
+      bulk_g2s(lsc, a.xlsc, sb, xbar);
+    }
+    if (!mbar_wait(xbar, 0u, clock64() + WAIT_BUDGET_CYCLES)) {
+      set_status(a.status, DEV_TIMEOUT);
+      *(volatile int *)&pl->abort = 1;
+    }
   }
   named_barrier_sync(CONSUMER_BAR, nth);
 
@@ -399,15 +433,7 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
   }
 
   // grid barrier 1: every a_g / a_u is written
-  named_barrier_sync(CONSUMER_BAR, nth);
-  if (tid == 0) {
-    if (!*(volatile int *)&pl->abort && !grid_barrier_one_thread(a.bar, G)) {
-      set_status(a.status, DEV_TIMEOUT);
-      *(volatile int *)&pl->abort = 1;
-    }
-    __threadfence();
-  }
-  named_barrier_sync(CONSUMER_BAR, nth);
+  grid_sync();
   // all CTAs of this grid are resident now; the next kernel may start its prologue
   pdl_launch_dependents();
   bool ok = !*(volatile int *)&pl->abort;
@@ -473,15 +499,7 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
   }
 
   // grid barrier 2: every gated expert output is written
-  named_barrier_sync(CONSUMER_BAR, nth);
-  if (tid == 0) {
-    if (!*(volatile int *)&pl->abort && !grid_barrier_one_thread(a.bar, G)) {
-      set_status(a.status, DEV_TIMEOUT);
-      *(volatile int *)&pl->abort = 1;
-    }
-    __threadfence();
-  }
-  named_barrier_sync(CONSUMER_BAR, nth);
+  grid_sync();
   if (*(volatile int *)&pl->abort) return;
 
   // phase 3: y[t] = sum_j part[t][j] in slot order
@@ -510,6 +528,8 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
 size_t ws_bar_bytes() { return 256; }
 size_t ws_abuf_bytes(int T, int k, int I) { return (((size_t)T * k * 2 * I * 4) + 255) & ~(size_t)255; }
 size_t ws_part_bytes(int T, int k, int H) { return (((size_t)T * k * H * 4) + 255) & ~(size_t)255; }
+size_t ws_xlimb_bytes(int T, int H) { return (((size_t)T * (H / 32) * LIMB_REC) + 255) & ~(size_t)255; }
+size_t ws_xlsc_bytes(int T, int H) { return (((size_t)T * (H / 32) * 8) + 255) & ~(size_t)255; }
 
 }  // namespace
 }  // namespace qmoe
@@ -524,7 +544,7 @@ using namespace qmoe;
 
 extern "C" size_t qmoe_decode_workspace_bytes(int T, int k, int H, int I) {
   if (T < 1 || k < 1 || H < 1 || I < 1) return 0;
-  return ws_bar_bytes() + ws_abuf_bytes(T, k, I) + ws_part_bytes(T, k, H);
+  return ws_bar_bytes() + ws_abuf_bytes(T, k, I) + ws_part_bytes(T, k, H) + ws_xlimb_bytes(T, H) + ws_xlsc_bytes(T, H);
 }
 
 qmoe_status qmoe::ffn_decode_launch(const qmoe_experts *ex, const float *x, int T, const int32_t *idx,
@@ -555,6 +575,8 @@ qmoe_status qmoe::ffn_decode_launch(const qmoe_experts *ex, const float *x, int 
   a.bar = reinterpret_cast<unsigned *>(ws);
   a.abuf = reinterpret_cast<float *>(ws + ws_bar_bytes());
   a.part = reinterpret_cast<float *>(ws + ws_bar_bytes() + ws_abuf_bytes(T, k, I));
+  a.xlimbs = reinterpret_cast<uint8_t *>(ws + ws_bar_bytes() + ws_abuf_bytes(T, k, I) + ws_part_bytes(T, k, ex->H));
+  a.xlsc = reinterpret_cast<float2 *>(a.xlimbs + ws_xlimb_bytes(T, ex->H));
   a.status = dev_status;
   a.T = T; a.k = k; a.E = ex->E; a.H = H; a.I = I;
 

@@ -291,9 +291,11 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
       st->abort = 1;
     } else {
       bool ok = true;
+      double zd[canon::SLICE];
+#pragma unroll
+      for (int i = 0; i < canon::SLICE; ++i) zd[i] = canon::f2d(st->ztmp[i]);
       for (int e = tid; e < E; e += nth)
-        ok &= add_fixed(&a.lacc[e], &a.lacc[E + e],
-                        canon::slice_dot([&](int i) { return wrtbuf[i * E + e]; }, [&](int i) { return st->ztmp[i]; }));
+        ok &= add_fixed(&a.lacc[e], &a.lacc[E + e], canon::slice_dot_wide([&](int i) { return wrtbuf[i * E + e]; }, zd));
       if (!ok) set_status(a.status, DEV_RANGE);
     }
   }
@@ -590,10 +592,11 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
         if (mbar_wait(wrtbar, (uint32_t)((l + 1) & 1), clock64() + WAIT_BUDGET_CYCLES)) {
           unsigned long long *la = a.lacc + (size_t)(par ^ 1) * 2 * E;
           bool rok = true;
+          double zd[canon::SLICE];
+#pragma unroll
+          for (int i = 0; i < canon::SLICE; ++i) zd[i] = canon::f2d(st->ztmp[i]);
           for (int e = tid; e < E; e += nth)
-            rok &= add_fixed(la + e, la + E + e,
-                             canon::slice_dot([&](int i) { return wrtbuf[i * E + e]; },
-                                              [&](int i) { return st->ztmp[i]; }));
+            rok &= add_fixed(la + e, la + E + e, canon::slice_dot_wide([&](int i) { return wrtbuf[i * E + e]; }, zd));
           if (!rok) set_status(a.status, DEV_RANGE);
         } else {
           set_status(a.status, DEV_TIMEOUT);
