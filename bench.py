@@ -224,6 +224,11 @@ TRAFFIC_PROFILES = {
     "stack_decode": ("stack_decode_decode48_ncu.md",
                      ("stack_decode.cu", "decode_tile.cuh", "common.cuh", "layout.cuh", "route_common.cuh")),
     "pf_gemm1": ("pf_gemm_prefill4096_ncu.md", ("prefill.cu", "tc05.cuh", "common.cuh", "layout.cuh")),
+    # per algorithmic byte (a launch's bytes depend on its routes): scaled to the measured launches
+    "ffn_decode_t8": ("ffn_decode_verify8_ncu.md",
+                      ("ffn_decode.cu", "decode_tile.cuh", "common.cuh", "layout.cuh", "decode_canon.cuh")),
+    "ffn_decode_t1": ("ffn_decode_layer1_ncu.md",
+                      ("ffn_decode.cu", "decode_tile.cuh", "common.cuh", "layout.cuh", "decode_canon.cuh")),
 }
 
 
@@ -235,9 +240,10 @@ def kernel_source_hash(names):
     return h.hexdigest()[:16]
 
 
-def stored_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel's
-    sources have not changed since the counters were taken (else None)."""
+def stored_traffic(kernel, key="dram_bytes_per_launch"):
+    """DRAM bytes per launch (or per algorithmic byte) from the committed ncu
+    summary, if the kernel's sources have not changed since the counters were
+    taken (else None)."""
     if kernel not in TRAFFIC_PROFILES:
         return None
     fname, sources = TRAFFIC_PROFILES[kernel]
@@ -253,9 +259,16 @@ def stored_traffic(kernel):
     if vals.get("kernel_source_sha256_16") != kernel_source_hash(sources):
         return None
     try:
-        return float(vals["dram_bytes_per_launch"])
+        return float(vals[key])
     except (KeyError, ValueError):
         return None
+
+
+def scaled_traffic(kernel, algorithmic_bytes):
+    """DRAM bytes of a launch of `algorithmic_bytes`, from a committed capture's
+    traffic per algorithmic byte (the launch reads what its routes select)."""
+    r = stored_traffic(kernel, "dram_bytes_per_algorithmic_byte")
+    return None if r is None else r * float(algorithmic_bytes)
 
 
 # --------------------------------------------------------- oracle timing --
@@ -520,7 +533,8 @@ def measure_stack(args, cfg, seed=SEED, full=True):
     out.update({
         "roofline": {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": hbm,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": stored_traffic("stack_decode") if (fused and cfg.L == 48) else None,
+                     "traffic": (stored_traffic("stack_decode") if cfg.L == 48 else None) if fused
+                     else scaled_traffic("ffn_decode_t8" if cfg.T > 1 else "ffn_decode_t1", launch_bytes),
                      "algorithmic_bytes_per_launch": launch_bytes, "avg_launch_us": 1e6 * launch_s,
                      "timing": f"CUDA event nodes around the kernel node(s) of a graph, mean of {n_t} replays"},
         "stack": {"path": "fused persistent kernel" if fused else "per-layer kernels (route + FFN) with PDL",
@@ -640,7 +654,8 @@ def run_layer(args, cfg):
                                    f"router + FFN launches, CUDA events around both"},
             "roofline": {"bound": "hbm", "kernel": "ffn_decode_kernel", "achieved": achieved, "peak": hbm,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
-                         "traffic": None, "algorithmic_bytes_per_launch": ffn_bytes,
+                         "traffic": scaled_traffic("ffn_decode_t1", ffn_bytes),
+                         "algorithmic_bytes_per_launch": ffn_bytes,
                          "avg_launch_us": 1e3 * statistics.mean(ffn_ms),
                          "median_launch_us": 1e3 * statistics.median(ffn_ms),
                          "timing": "CUDA events around each FFN launch (a second pass, event between router and "
