@@ -55,7 +55,7 @@ typedef enum {
   QMOE_ERR_TIMEOUT = 6,       /* a device-side wait exceeded its budget */
   QMOE_ERR_DEVICE_STATUS = 7, /* invalid routed index seen on the device */
   QMOE_ERR_RANGE = 8          /* decode activations too large for the exact router sums:
-                                 a 16-element slice's partial logit reached 2^31 */
+                                 a 16-element slice's partial logit reached 2^19 */
 } qmoe_status;
 
 enum { QMOE_Q2 = 2, QMOE_Q4 = 4 };        /* block formats (bits per code) */
@@ -118,12 +118,14 @@ qmoe_status qmoe_pack(int fmt, int kind, int E, int H, int I,
  * (x_dtype QMOE_F32) or bf16 (QMOE_BF16). Outputs: idx int32 [T,k] and
  * gate fp32 [T,k]. Workspace: qmoe_route_workspace_bytes(T, E) bytes, zeroed
  * once before first use (it is left zeroed by every completed call).
- * Limits: 1 <= k <= 16, k <= E <= 1024, H multiple of 128, T >= 1.
+ * Limits: 1 <= k <= 16, k <= E <= 1024, H multiple of 128, T >= 1; with fp32
+ * x and T <= 8 also H <= 65,536.
  * T <= 8 with fp32 x runs the decode router: every 16-element slice partial
- * sum_h x*Wr is a float64 fused multiply-add chain, split into two exact
- * integers and summed exactly, so the logit does not depend on how the work is
- * split (the fused layer stack forms the same logits); one warp per token then
- * selects from shared memory. Larger T or bf16 x runs the prefill router:
+ * sum_h x*Wr is a float64 fused multiply-add chain, rounded to an integer in
+ * units of 2^-32 and summed exactly, so the logit does not depend on how the
+ * work is split (the fused layer stack forms the same logits); one warp per
+ * token then selects from shared memory. A slice partial of magnitude 2^19 or
+ * more sets QMOE_ERR_RANGE in the status word. Larger T or bf16 x runs the prefill router:
  * approximate logits on the integer tensor cores (16-bit fixed point in two
  * 8-bit limbs) with a proven error bound pick a few candidates per token,
  * whose float64 logits (exact products, float64 sums) decide the selection
@@ -162,7 +164,8 @@ qmoe_status qmoe_rmsnorm_residual(const float *x_in, const float *y, float eps, 
  * ticket) held in one fixed device array of QMOE_ROUTE_FIXED_SCRATCH_BYTES
  * bytes inside the library; nothing is allocated.
  * Limits: 1 <= T <= QMOE_ROUTE_FIXED_MAX_T, E <= QMOE_ROUTE_FIXED_MAX_E,
- * 1 <= k <= 16, H a multiple of 128; larger requests return UNSUPPORTED.
+ * 1 <= k <= 16, H a multiple of 128 and at most 65,536; larger requests
+ * return UNSUPPORTED.
  * The first call on each device looks up the array's address and zeroes it
  * synchronously (cudaGetSymbolAddress, cudaMemset; the ticket must start at
  * zero and every completed call leaves it at zero). Make that first call
@@ -171,7 +174,7 @@ qmoe_status qmoe_rmsnorm_residual(const float *x_in, const float *y, float eps, 
  * them on one stream. */
 #define QMOE_ROUTE_FIXED_MAX_T 8
 #define QMOE_ROUTE_FIXED_MAX_E 1024
-#define QMOE_ROUTE_FIXED_SCRATCH_BYTES (QMOE_ROUTE_FIXED_MAX_T * 2 * QMOE_ROUTE_FIXED_MAX_E * 8 + 256)
+#define QMOE_ROUTE_FIXED_SCRATCH_BYTES (QMOE_ROUTE_FIXED_MAX_T * QMOE_ROUTE_FIXED_MAX_E * 8 + 256)
 qmoe_status qmoe_route_fixed(const float *Wr, const float *bias, const float *x, int T, int H, int E, int k,
                              int32_t *idx, float *gate, int32_t *dev_status, qmoe_stream_t stream);
 
@@ -306,10 +309,11 @@ int qmoe_stack_kernels_per_replay(const qmoe_stack *stack);
 uint32_t *qmoe_stack_barrier_word(const qmoe_stack *stack);
 /* Which path the stack runs. QMOE_PATH_FUSED (single-token stacks whose
  * geometry fits one SM's shared memory): one persistent kernel runs all L
- * layers with two grid barriers per layer; router logits there are formed from
- * exact fixed-point partial sums (resolution 2^-40 per partial) instead of one
- * float64 dot product per expert. QMOE_PATH_LAYERWISE: qmoe_residual_route and
- * qmoe_ffn_decode per layer, chained with programmatic dependent launch. */
+ * layers with two grid barriers per layer. QMOE_PATH_LAYERWISE:
+ * qmoe_residual_route and qmoe_ffn_decode per layer, chained with
+ * programmatic dependent launch. Both paths form a token's router logits from
+ * the same integer sums of rounded 16-element slice partials (2^-32 units) and
+ * give the same bits. */
 int qmoe_stack_path(const qmoe_stack *stack);
 /* Per-layer durations (ms) of the most recent completed replay of a
  * QMOE_STACK_TIMING stack: route_ms[l] spans layer l's router (with its fused

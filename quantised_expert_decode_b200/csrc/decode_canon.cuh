@@ -11,8 +11,8 @@
 //   partials   a slice's router partial sum_i Wr[e][16c+i] z[16c+i] and its
 //              sum of squares sum_i z[16c+i]^2 are float64 fma chains in
 //              element order i = 0..15;
-//   logits     each router partial is split into two integers (hi in units
-//              of 2^-20, lo in units of 2^-60); integers add exactly in any
+//   logits     each router partial is rounded to an integer in units of
+//              2^-32 (one rounding, to nearest); integers add exactly in any
 //              order, so a row summed by one warp and a row summed over 128
 //              CTAs with atomics agree;
 //   squares    the slice sums of squares are added in one fixed order: lane l
@@ -26,8 +26,12 @@
 //   combine    y = sum_j gate_j * r_j in slot order, one rounding per multiply
 //              and per add; z_next = x + y.
 //
-// A router partial of magnitude 2^31 or more (or NaN) cannot be split exactly;
-// it is reported through the device status (DEV_RANGE) instead.
+// A router partial of magnitude 2^19 or more (or NaN) is reported through the
+// device status (DEV_RANGE) instead: below it the integer stays under 2^51, so
+// one magic-number addition rounds it, and the sum of up to 2^12 slices
+// (H <= 65,536) cannot overflow 64 bits. Slice partials of normalised
+// activations are of order 1; the rounding (at most 2^-33 a slice) moves a
+// 128-slice logit by less than 2e-8.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -39,35 +43,23 @@ namespace canon {
 namespace {
 
 constexpr int SLICE = 16;
-constexpr double FIX_HI_INV = 1.0 / 1048576.0;              // 2^-20
-constexpr double FIX_LO = 1152921504606846976.0;            // 2^60
-constexpr double FIX_LO_INV = 1.0 / 1152921504606846976.0;  // 2^-60
-constexpr double FIX_RANGE = 2147483648.0;                  // 2^31
-constexpr double MAGIC_HI = 6442450944.0;                   // 1.5 * 2^32: its ulp is 2^-20
-constexpr double MAGIC_LO = 6755399441055744.0;             // 1.5 * 2^52: its ulp is 1
+constexpr double FIX_UNIT = 4294967296.0;                   // 2^32
+constexpr double FIX_UNIT_INV = 1.0 / 4294967296.0;         // 2^-32
+constexpr double FIX_RANGE = 524288.0;                       // 2^19
+constexpr double MAGIC = 6755399441055744.0;                 // 1.5 * 2^52: its ulp is 1
 
-// p -> (hi, lo) with p = hi 2^-20 + lo 2^-60 up to the rounding of lo, in
-// float64 adds and integer subtractions only (no conversion instruction):
-//   t = p + 1.5 * 2^32 rounds p to the nearest multiple of 2^-20 (the ulp of
-//     t, which stays in [2^32, 2^33) for |p| < 2^31), and the integer hi sits
-//     in t's low mantissa bits: hi = bits(t) - bits(1.5 * 2^32);
-//   r = p - (t - 1.5 * 2^32) is exact (a multiple of min(ulp(p), 2^-20) below
-//     2^-21 in magnitude);
-//   u = r * 2^60 + 1.5 * 2^52 rounds r * 2^60 (exact, below 2^39) to an
-//     integer, lo = bits(u) - bits(1.5 * 2^52).
-// Both roundings are to nearest, ties to even. Returns false (and zeros) when
-// |p| >= 2^31 or p is NaN.
-__device__ __forceinline__ bool split(double p, long long &hi, long long &lo) {
+// p -> v = round(p * 2^32) in one fused multiply-add: p * 2^32 is exact, the
+// addition of 1.5 * 2^52 rounds it to an integer (to nearest, ties to even;
+// the sum stays in [2^52, 2^53) for |p| < 2^19), and the integer sits in the
+// sum's low mantissa bits: v = bits(t) - bits(1.5 * 2^52). No conversion
+// instruction. Returns false (and 0) when |p| >= 2^19 or p is NaN.
+__device__ __forceinline__ bool fix(double p, long long &v) {
   if (!(fabs(p) < FIX_RANGE)) {
-    hi = 0;
-    lo = 0;
+    v = 0;
     return false;
   }
-  const double t = __dadd_rn(p, MAGIC_HI);
-  const double r = __dsub_rn(p, __dsub_rn(t, MAGIC_HI));
-  const double u = __fma_rn(r, FIX_LO, MAGIC_LO);
-  hi = __double_as_longlong(t) - __double_as_longlong(MAGIC_HI);
-  lo = __double_as_longlong(u) - __double_as_longlong(MAGIC_LO);
+  const double t = __fma_rn(p, FIX_UNIT, MAGIC);
+  v = __double_as_longlong(t) - __double_as_longlong(MAGIC);
   return true;
 }
 
@@ -81,11 +73,9 @@ __device__ __forceinline__ double i64_to_f64(long long v) {
   return __fma_rn(h, 4294967296.0, l);
 }
 
-// Exact integer totals -> float64 (two exact scalings, one rounding in the add;
-// each total is exact in float64 below 2^53).
-__device__ __forceinline__ double join(long long hi, long long lo) {
-  return __dadd_rn(__dmul_rn(i64_to_f64(hi), FIX_HI_INV), __dmul_rn(i64_to_f64(lo), FIX_LO_INV));
-}
+// An exact integer total -> float64 (one rounding above 2^53, then an exact
+// scaling).
+__device__ __forceinline__ double unfix(long long v) { return __dmul_rn(i64_to_f64(v), FIX_UNIT_INV); }
 
 // float -> float64, exactly, for normal numbers by moving the bits (IEEE 754
 // binary32 -> binary64: the exponent rebiased by 1023 - 127, the 23 mantissa
@@ -176,14 +166,7 @@ __device__ __forceinline__ float silu(float a) { return __fdiv_rn(a, __fadd_rn(1
 
 __device__ __forceinline__ float hval(float a_g, float a_u) { return __fmul_rn(silu(a_g), a_u); }
 
-// Warp-wide exact sum of (hi, lo) pairs.
-__device__ __forceinline__ void warp_sum_fix(long long &hi, long long &lo) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    hi += __shfl_xor_sync(0xffffffffu, hi, o);
-    lo += __shfl_xor_sync(0xffffffffu, lo, o);
-  }
-}
+
 
 }  // namespace
 }  // namespace canon

@@ -44,17 +44,17 @@ struct RouteArgs {
   int ns;              // hidden-axis ranges per expert group
   int32_t *idx;
   float *gate;
-  unsigned long long *lacc;   // workspace [T][2 hi|lo][E] exact partial-logit sums (two's complement)
+  unsigned long long *lacc;   // workspace [T][E] exact partial-logit sums (2^-32 units, two's complement)
   unsigned *ticket;           // workspace
   int32_t *status;
 };
 
 // Dynamic shared memory of one CTA: the largest of the staged activations
 // (float64 [RT_CHUNK * 16][TT]), the per-warp integer sums
-// ([RT_WARPS][TT][2][32]) and, in the last CTA, the logits ([T][E]).
+// ([RT_WARPS][TT][32]) and, in the last CTA, the logits ([T][E]).
 inline size_t route_smem_bytes(int TT, int E) {
   size_t z = (size_t)RT_CHUNK * canon::SLICE * TT * 8;
-  size_t r = (size_t)RT_WARPS * TT * 2 * RT_GROUP * 8;
+  size_t r = (size_t)RT_WARPS * TT * RT_GROUP * 8;
   size_t l = (size_t)TT * E * 8;
   size_t m = z > r ? z : r;
   return m > l ? m : l;
@@ -117,17 +117,16 @@ template <int M>
 __device__ __forceinline__ void route_token_select(const RouteArgs &a, int t, double rinv, double *lg,
                                                    TopkScratch *sc) {
   const int lane = threadIdx.x & 31, E = a.E;
-  unsigned long long *ph = a.lacc + (size_t)t * 2 * E;
-  unsigned long long hv[M], lv[M];
+  unsigned long long *ph = a.lacc + (size_t)t * E;
+  unsigned long long hv[M];
   float bv[M];
 #pragma unroll
   for (int j = 0; j < M; ++j) {
     const int e = lane + 32 * j;
-    hv[j] = lv[j] = 0ull;
+    hv[j] = 0ull;
     bv[j] = 0.0f;
     if (e < E) {
       hv[j] = __ldcg(ph + e);
-      lv[j] = __ldcg(ph + E + e);
       if (a.bias) bv[j] = __ldg(a.bias + e);
     }
   }
@@ -137,12 +136,10 @@ __device__ __forceinline__ void route_token_select(const RouteArgs &a, int t, do
     const int e = lane + 32 * j;
     key[j] = 0u;
     if (e < E) {
-      const double v = canon::logit(canon::join((long long)hv[j], (long long)lv[j]), rinv,
-                                    a.bias ? canon::f2d(bv[j]) : 0.0);
+      const double v = canon::logit(canon::unfix((long long)hv[j]), rinv, a.bias ? canon::f2d(bv[j]) : 0.0);
       lg[e] = v;
       key[j] = logit_key(v);
       ph[e] = 0ull;
-      ph[E + e] = 0ull;
     }
   }
   __syncwarp();
@@ -177,9 +174,9 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_decode_kernel(RouteArgs a
   pdl_wait();
   pdl_launch_dependents();
 
-  long long hi[TT], lo[TT];
+  long long acc[TT];
 #pragma unroll
-  for (int t = 0; t < TT; ++t) hi[t] = lo[t] = 0;
+  for (int t = 0; t < TT; ++t) acc[t] = 0;
   bool ok = true;
   double *zd = rsm;   // [RT_CHUNK * 16][TT]
   int cc = c0;
@@ -206,10 +203,9 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_decode_kernel(RouteArgs a
     }
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
-      long long h1, l1;
-      ok &= canon::split(p[t], h1, l1);
-      hi[t] += h1;
-      lo[t] += l1;
+      long long v1;
+      ok &= canon::fix(p[t], v1);
+      acc[t] += v1;
     }
   };
   for (; cc < c1; cc += RT_CHUNK) {
@@ -256,21 +252,18 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_decode_kernel(RouteArgs a
 
   // sum the warps' integers, then one pair of atomics per (token, expert)
   __syncthreads();
-  unsigned long long *red = reinterpret_cast<unsigned long long *>(rsm);   // [warp][TT][2][32]
+  unsigned long long *red = reinterpret_cast<unsigned long long *>(rsm);   // [warp][TT][32]
 #pragma unroll
-  for (int t = 0; t < TT; ++t) {
-    red[((warp * TT + t) * 2 + 0) * RT_GROUP + lane] = (unsigned long long)hi[t];
-    red[((warp * TT + t) * 2 + 1) * RT_GROUP + lane] = (unsigned long long)lo[t];
-  }
+  for (int t = 0; t < TT; ++t) red[(warp * TT + t) * RT_GROUP + lane] = (unsigned long long)acc[t];
   __syncthreads();
-  for (int i = tid; i < TT * 2 * RT_GROUP; i += RT_THREADS) {
-    const int t = i / (2 * RT_GROUP), which = (i / RT_GROUP) & 1, ln = i % RT_GROUP;
+  for (int i = tid; i < TT * RT_GROUP; i += RT_THREADS) {
+    const int t = i / RT_GROUP, ln = i % RT_GROUP;
     const int ee = g * RT_GROUP + ln;
     if (t < T && ee < E) {
       unsigned long long v = 0;
 #pragma unroll
-      for (int w = 0; w < RT_WARPS; ++w) v += red[((w * TT + t) * 2 + which) * RT_GROUP + ln];
-      atomicAdd(a.lacc + ((size_t)t * 2 + which) * E + ee, v);
+      for (int w = 0; w < RT_WARPS; ++w) v += red[(w * TT + t) * RT_GROUP + ln];
+      atomicAdd(a.lacc + (size_t)t * E + ee, v);
     }
   }
 
@@ -323,8 +316,8 @@ __global__ void __launch_bounds__(256) rmsnorm_residual_kernel(const float *x, c
   for (int h = tid; h < H; h += 256) out[(size_t)t * H + h] = __fmul_rn(__fadd_rn(xr[h], yr[h]), inv);
 }
 
-// Workspace: the exact sums [T][2][E] int64, then a 256-byte ticket block.
-size_t decode_lacc_bytes(int T, int E) { return (((size_t)T * 2 * E * sizeof(unsigned long long)) + 255) & ~(size_t)255; }
+// Workspace: the exact sums [T][E] int64, then a 256-byte ticket block.
+size_t decode_lacc_bytes(int T, int E) { return (((size_t)T * E * sizeof(unsigned long long)) + 255) & ~(size_t)255; }
 size_t decode_ws_bytes(int T, int E) { return decode_lacc_bytes(T, E) + 256; }
 
 template <int TT>
@@ -387,7 +380,7 @@ static qmoe_status check_route_common(const float *Wr, int T, int H, int E, int 
   if (!Wr || !idx || !gate || !ws || !status) return QMOE_ERR_INVALID_ARG;
   if (!aligned16(Wr) || !aligned16(ws)) return QMOE_ERR_INVALID_ARG;
   if (T < 1 || H < 128 || E < 1 || k < 1) return QMOE_ERR_INVALID_ARG;
-  if (H % 128) return QMOE_ERR_UNSUPPORTED;
+  if (H % 128 || H > 65536) return QMOE_ERR_UNSUPPORTED;   // exact sums of at most 4096 slices
   if (k > 16 || k > E || E > 1024) return QMOE_ERR_UNSUPPORTED;
   return QMOE_OK;
 }
@@ -460,10 +453,10 @@ extern "C" qmoe_status qmoe_residual_route(const float *x_in, const float *y, fl
 namespace qmoe {
 namespace {
 
-constexpr size_t FIXED_SUMS_BYTES = (size_t)QMOE_ROUTE_FIXED_MAX_T * 2 * QMOE_ROUTE_FIXED_MAX_E * 8;
+constexpr size_t FIXED_SUMS_BYTES = (size_t)QMOE_ROUTE_FIXED_MAX_T * QMOE_ROUTE_FIXED_MAX_E * 8;
 static_assert(QMOE_ROUTE_FIXED_SCRATCH_BYTES == FIXED_SUMS_BYTES + 256, "fixed scratch layout");
 
-// [0, FIXED_SUMS_BYTES): the exact partial-logit sums ([T][2][E] int64, laid
+// [0, FIXED_SUMS_BYTES): the exact partial-logit sums ([T][E] int64, laid
 // out for the call's own T and E); then the 256-byte ticket block. Both must
 // start at zero, and each completed call leaves them at zero.
 __device__ __align__(256) unsigned char g_route_scratch[QMOE_ROUTE_FIXED_SCRATCH_BYTES];
@@ -500,7 +493,7 @@ extern "C" qmoe_status qmoe_route_fixed(const float *Wr, const float *bias, cons
   if (!Wr || !x || !idx || !gate || !dev_status) return QMOE_ERR_INVALID_ARG;
   if (!aligned16(Wr) || !aligned16(x)) return QMOE_ERR_INVALID_ARG;
   if (T < 1 || H < 128 || E < 1 || k < 1) return QMOE_ERR_INVALID_ARG;
-  if (H % 128 || k > 16 || k > E) return QMOE_ERR_UNSUPPORTED;
+  if (H % 128 || H > 65536 || k > 16 || k > E) return QMOE_ERR_UNSUPPORTED;
   if (T > QMOE_ROUTE_FIXED_MAX_T || E > QMOE_ROUTE_FIXED_MAX_E) return QMOE_ERR_UNSUPPORTED;
   void *scratch = nullptr;
   const qmoe_status st = fixed_scratch(&scratch);

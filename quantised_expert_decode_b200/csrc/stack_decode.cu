@@ -76,7 +76,7 @@ struct StackArgs {
   int32_t *idx_rec;           // [L][k]
   float *gate_rec;            // [L][k]
   float *zbuf;                // [2][H]
-  unsigned long long *lacc;   // [2 parity][2 hi|lo][E] integer partial-logit sums (two's complement)
+  unsigned long long *lacc;   // [2 parity][E] integer partial-logit sums (2^-32 units, two's complement)
   double *ssq;                // [2 parity][H/16] slice sums of squares
   uint8_t *lbuf;              // [k][I/32][LIMB_REC]: limbs of h
   float2 *lscg;               // [k][I/32]: (s, s * sum X) of h's blocks
@@ -134,17 +134,13 @@ __host__ __device__ inline SkLayout sk_layout(int bits, int E, int H, int I, int
   return o;
 }
 
-// Adds one slice partial to an exact (hi, lo) integer total; false when the
-// partial is out of the range the split covers.
-__device__ __forceinline__ bool add_fixed(unsigned long long *hi, unsigned long long *lo, double p) {
-  long long h, l;
-  const bool ok = canon::split(p, h, l);
-  atomicAdd(hi, (unsigned long long)h);
-  atomicAdd(lo, (unsigned long long)l);
+// Adds one slice partial to an exact integer total; false when the partial is
+// out of the fixed-point range.
+__device__ __forceinline__ bool add_fixed(unsigned long long *acc, double p) {
+  long long v;
+  const bool ok = canon::fix(p, v);
+  atomicAdd(acc, (unsigned long long)v);
   return ok;
-}
-__device__ __forceinline__ double read_fixed(const unsigned long long *hi, const unsigned long long *lo) {
-  return canon::join((long long)__ldcg(hi), (long long)__ldcg(lo));
 }
 
 // Consumer-side grid barrier: the 256 consumer threads meet, one thread joins
@@ -295,7 +291,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
 #pragma unroll
       for (int i = 0; i < canon::SLICE; ++i) zd[i] = canon::f2d(st->ztmp[i]);
       for (int e = tid; e < E; e += nth)
-        ok &= add_fixed(&a.lacc[e], &a.lacc[E + e], canon::slice_dot_wide([&](int i) { return wrtbuf[i * E + e]; }, zd));
+        ok &= add_fixed(&a.lacc[e], canon::slice_dot_wide([&](int i) { return wrtbuf[i * E + e]; }, zd));
       if (!ok) set_status(a.status, DEV_RANGE);
     }
   }
@@ -340,9 +336,9 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
       // one batch of loads: sum of squares, z, partial logits, bias
       const float4 *zb = reinterpret_cast<const float4 *>(a.zbuf + (size_t)par * H);
       const float *b = a.bias[l];
-      const unsigned long long *la = a.lacc + (size_t)par * 2 * E;
+      const unsigned long long *la = a.lacc + (size_t)par * E;
       float4 zv[4];
-      unsigned long long lh[4], ll[4];
+      unsigned long long lh[4];
       float bv[4];
       const double *sq = a.ssq + (size_t)par * H16;
       double sv[4];   // this lane's first slice sums of squares (decode_canon.cuh's order)
@@ -354,7 +350,6 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
         if (q < H / 4) zv[i] = __ldcg(zb + q);
         if (q < E) {
           lh[i] = __ldcg(la + q);
-          ll[i] = __ldcg(la + E + q);
           bv[i] = b ? __ldg(b + q) : 0.0f;
         }
       }
@@ -375,7 +370,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
           reinterpret_cast<float4 *>(xs)[q] = v;
         }
         if (q < E) {
-          const double lv = canon::logit(canon::join((long long)lh[i], (long long)ll[i]), rinv, canon::f2d(bv[i]));
+          const double lv = canon::logit(canon::unfix((long long)lh[i]), rinv, canon::f2d(bv[i]));
           logits[q] = lv;
           keytab[key_slot(q, MK)] = logit_key(lv);
         }
@@ -388,14 +383,14 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
         reinterpret_cast<float4 *>(xs)[q] = v;
       }
       for (int q = tid + 4 * nth; q < E; q += nth) {
-        const double lv = canon::logit(read_fixed(la + q, la + E + q), rinv, b ? canon::f2d(b[q]) : 0.0);
+        const double lv = canon::logit(canon::unfix((long long)__ldcg(la + q)), rinv, b ? canon::f2d(b[q]) : 0.0);
         logits[q] = lv;
         keytab[key_slot(q, MK)] = logit_key(lv);
       }
       // clear the other parity's accumulators for the next layer (read last by
       // every CTA before the previous barriers)
-      unsigned long long *lz = a.lacc + (size_t)(par ^ 1) * 2 * E;
-      for (int e = c * nth + tid; e < 2 * E; e += G * nth) lz[e] = 0ull;
+      unsigned long long *lz = a.lacc + (size_t)(par ^ 1) * E;
+      for (int e = c * nth + tid; e < E; e += G * nth) lz[e] = 0ull;
       named_barrier_sync(CONS_BAR, nth);
       if (tid == 0) trace_point(a, l, TP_LOGITS);
       if (warp == 0) {
@@ -590,13 +585,13 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
       if (tid == 0) trace_point(a, l, TP_Z);
       if (ok && l + 1 < L) {
         if (mbar_wait(wrtbar, (uint32_t)((l + 1) & 1), clock64() + WAIT_BUDGET_CYCLES)) {
-          unsigned long long *la = a.lacc + (size_t)(par ^ 1) * 2 * E;
+          unsigned long long *la = a.lacc + (size_t)(par ^ 1) * E;
           bool rok = true;
           double zd[canon::SLICE];
 #pragma unroll
           for (int i = 0; i < canon::SLICE; ++i) zd[i] = canon::f2d(st->ztmp[i]);
           for (int e = tid; e < E; e += nth)
-            rok &= add_fixed(la + e, la + E + e, canon::slice_dot_wide([&](int i) { return wrtbuf[i * E + e]; }, zd));
+            rok &= add_fixed(la + e, canon::slice_dot_wide([&](int i) { return wrtbuf[i * E + e]; }, zd));
           if (!rok) set_status(a.status, DEV_RANGE);
         } else {
           set_status(a.status, DEV_TIMEOUT);
@@ -628,7 +623,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
   }
   // leave lacc[0] clear for the next launch's layer-0 partials (its last
   // reader finished long before the last barrier)
-  for (int e = c * nth + tid; e < 2 * E; e += G * nth) a.lacc[e] = 0ull;
+  for (int e = c * nth + tid; e < E; e += G * nth) a.lacc[e] = 0ull;
 }
 
 }  // namespace
@@ -661,7 +656,7 @@ bool fused_stack_plan(int fmt, int E, int H, int I, int k, FusedPlan *p) {
 size_t fused_stack_ws_bytes(int L, int E, int H, int I, int k) {
   auto a = [](size_t v) { return (v + 255) & ~(size_t)255; };
   const size_t nb = (size_t)k * (I / 32);
-  return a((size_t)L * H * E * 4) + a(4 * (size_t)E * 8) + a(2 * (size_t)(H / 16) * 8) + a(2 * (size_t)H * 4) +
+  return a((size_t)L * H * E * 4) + a(2 * (size_t)E * 8) + a(2 * (size_t)(H / 16) * 8) + a(2 * (size_t)H * 4) +
          a(nb * LIMB_REC) + a(nb * 8) + 256 + 3 * a((size_t)L * 8);
 }
 
@@ -671,7 +666,7 @@ FusedBufs fused_carve(void *ws, int L, int E, int H, int I, int k) {
   char *p = static_cast<char *>(ws);
   FusedBufs b;
   b.wrt = reinterpret_cast<float *>(p); p += a((size_t)L * H * E * 4);
-  b.lacc = reinterpret_cast<unsigned long long *>(p); p += a(4 * (size_t)E * 8);
+  b.lacc = reinterpret_cast<unsigned long long *>(p); p += a(2 * (size_t)E * 8);
   b.ssq = reinterpret_cast<double *>(p); p += a(2 * (size_t)(H / 16) * 8);
   b.zbuf = reinterpret_cast<float *>(p); p += a(2 * (size_t)H * 4);
   const size_t nb = (size_t)k * (I / 32);

@@ -19,7 +19,7 @@ struct FusedPlan {
 // Device buffers of the fused path, carved from the stack's workspace.
 struct FusedBufs {
   float *wrt;                      // [L][H][E] transposed routers
-  unsigned long long *lacc;         // [2][2][E] integer partial-logit sums
+  unsigned long long *lacc;         // [2][E] integer partial-logit sums (2^-32 units)
   double *ssq;                     // [2][H/16] slice sums of squares
   float *zbuf;
   uint8_t *lbuf;                   // limbs of h, [k][I/32][96]

@@ -93,3 +93,19 @@ def test_limb_pair_recombination_is_exact_in_one_step_for_2_bit_codes():
     v = hi.astype(np.int64) * 256 + lo
     assert np.abs(v).max() < 2 ** 22
     assert np.array_equal(i2f_small(v).astype(np.int64), v)
+
+
+def test_router_partial_fixed_point_rounds_once_to_the_nearest_integer():
+    """Router slice partials become integers in units of 2^-32 through one
+    fused multiply-add with 1.5 * 2^52 (its ulp is 1): for |p| < 2^19 the
+    product p * 2^32 is exact and below 2^51, so the integer read from the
+    sum's bits is p * 2^32 rounded to nearest (ties to even); 4096 such
+    integers (H = 65,536) add without overflowing 64 bits."""
+    rs = np.random.default_rng(11)
+    p = np.concatenate([rs.uniform(-2.0 ** 19, 2.0 ** 19, 20000), rs.standard_normal(20000) * 1e-3,
+                        [2.0 ** 19 - 1e-6, -(2.0 ** 19 - 1e-6), 0.0, -0.0, 2.0 ** -33, 3 * 2.0 ** -33, -(2.0 ** -33)]])
+    magic = np.float64(1.5 * 2.0 ** 52)
+    t = p * 2.0 ** 32 + magic            # the product is exact, the sum rounds once (float64)
+    v = t.view(np.int64) - magic.view(np.int64)
+    assert np.array_equal(v, np.rint(p * 2.0 ** 32).astype(np.int64))   # rint: to nearest, ties to even
+    assert 4096 * (2 ** 51 - 1) < 2 ** 63      # each |v| <= 2^51 - 1

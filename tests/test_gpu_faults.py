@@ -71,7 +71,7 @@ def test_fused_stack_grid_barrier_runs_out_then_a_fresh_stack_passes():
 @pytest.mark.parametrize("layerwise", [False, True])
 def test_activations_beyond_the_exact_sum_range_are_reported(layerwise):
     """x_0 of magnitude ~1e12: a router partial over one 16-element slice
-    exceeds 2^31, so the stack reports QMOE_ERR_RANGE; every route it took is
+    exceeds 2^19, so the stack reports QMOE_ERR_RANGE; every route it took is
     still a set of distinct experts in [0, E)."""
     cfg = configs.get(0).with_(L=3, residual=True)
     layers, routers, _ = device_layers(SEED, cfg, 3)
