@@ -70,33 +70,43 @@ __device__ __forceinline__ int warp_excl_scan(int v, int &total) {
 }
 
 // One warp. Items are numbered expert by expert, per_expert items an expert,
-// each at its expert's tile cost (cost prefix cw); returns the first item
-// whose starting cost is at least `target` (U * per_expert if none). Expert u
-// holds that item when it is the first with target <= acc_u + (per_expert - 1)
-// w_u, acc_u = per_expert cw[u]: the item is then u's first if target <= acc_u,
-// else the ceil((target - acc_u) / w_u)-th.
-__device__ int item_at_cost(const Plan *pl, int U, int per_expert, long long target) {
+// each at its expert's tile cost (cost prefix cw). For each of the NT targets
+// returns the first item whose starting cost is at least that target
+// (U * per_expert if none). Expert u holds that item when it is the first with
+// target <= acc_u + (per_expert - 1) w_u, acc_u = per_expert cw[u]: the item is
+// then u's first if target <= acc_u, else the ceil((target - acc_u) / w_u)-th.
+// All targets are resolved in one pass over the experts, in 32-bit arithmetic
+// (the caller checks the costs fit).
+template <int NT>
+__device__ __forceinline__ void items_at_costs(const Plan *pl, int U, int per_expert, const int (&target)[NT],
+                                               int (&item)[NT]) {
   const int lane = threadIdx.x & 31;
+  bool done[NT];
+#pragma unroll
+  for (int q = 0; q < NT; ++q) {
+    done[q] = false;
+    item[q] = U * per_expert;
+  }
   for (int u0 = 0; u0 < U; u0 += 32) {
     const int u = u0 + lane;
-    bool hit = false;
-    long long acc = 0;
-    int w = 1;
+    int acc = 0, w = 1;
     if (u < U) {
       w = tile_cost(pl->nt[u]);
-      acc = (long long)per_expert * pl->cw[u];
-      hit = target <= acc + (long long)(per_expert - 1) * w;
+      acc = per_expert * pl->cw[u];
     }
-    const unsigned b = __ballot_sync(0xffffffffu, hit);
-    if (b) {
-      const int src = __ffs(b) - 1;
-      const long long acc0 = __shfl_sync(0xffffffffu, acc, src);
-      const int w0 = __shfl_sync(0xffffffffu, w, src);
-      const int ui = u0 + src;
-      return target <= acc0 ? ui * per_expert : ui * per_expert + (int)((target - acc0 + w0 - 1) / w0);
+#pragma unroll
+    for (int q = 0; q < NT; ++q) {
+      const unsigned b = __ballot_sync(0xffffffffu, u < U && target[q] <= acc + (per_expert - 1) * w);
+      if (!done[q] && b) {
+        const int src = __ffs(b) - 1;
+        const int acc0 = __shfl_sync(0xffffffffu, acc, src);
+        const int w0 = __shfl_sync(0xffffffffu, w, src);
+        const int ui = u0 + src;
+        item[q] = target[q] <= acc0 ? ui * per_expert : ui * per_expert + (target[q] - acc0 + w0 - 1) / w0;
+        done[q] = true;
+      }
     }
   }
-  return U * per_expert;
 }
 
 // Route table -> unique experts (ascending), their tokens (ascending) and
@@ -107,7 +117,7 @@ __device__ void build_plan(const int32_t *idx, const float *gate, int T, int k, 
   for (int w = lane; w < FD_MAXE / 4; w += 32) pl->tm[w] = 0u;
   int pe[FD_MAXP / 32];
   float pg[FD_MAXP / 32];
-#pragma unroll
+#pragma unroll 1
   for (int i = 0; i < FD_MAXP / 32; ++i) {
     const int p = lane + 32 * i;
     pe[i] = p < P ? idx[p] : 0;
@@ -115,7 +125,7 @@ __device__ void build_plan(const int32_t *idx, const float *gate, int T, int k, 
   }
   __syncwarp();
   int bad = 0;
-#pragma unroll
+#pragma unroll 1
   for (int i = 0; i < FD_MAXP / 32; ++i) {
     const int p = lane + 32 * i;
     if (p >= P) continue;
@@ -140,10 +150,10 @@ __device__ void build_plan(const int32_t *idx, const float *gate, int T, int k, 
   __syncwarp();
   // bitmap word `lane`: experts 32 lane .. 32 lane + 31
   unsigned word = 0u;
-#pragma unroll
+#pragma unroll 1
   for (int q = 0; q < 8; ++q) {
     const unsigned m = pl->tm[lane * 8 + q];
-#pragma unroll
+#pragma unroll 1
     for (int b = 0; b < 4; ++b)
       if ((m >> (8 * b)) & 0xffu) word |= 1u << (4 * q + b);
   }
@@ -159,7 +169,7 @@ __device__ void build_plan(const int32_t *idx, const float *gate, int T, int k, 
   __syncwarp();
   // token and cost prefixes over the unique experts (4 a lane, in order)
   int nt4[FD_MAXP / 32], c4[FD_MAXP / 32], ntl = 0, cl = 0;
-#pragma unroll
+#pragma unroll 1
   for (int i = 0; i < FD_MAXP / 32; ++i) {
     const int u = lane * (FD_MAXP / 32) + i;
     nt4[i] = u < U ? pl->nt[u] : 0;
@@ -169,7 +179,7 @@ __device__ void build_plan(const int32_t *idx, const float *gate, int T, int k, 
   }
   int ntot, ctot;
   int nb = warp_excl_scan(ntl, ntot), cb = warp_excl_scan(cl, ctot);
-#pragma unroll
+#pragma unroll 1
   for (int i = 0; i < FD_MAXP / 32; ++i) {
     const int u = lane * (FD_MAXP / 32) + i;
     if (u < U) {
@@ -188,7 +198,7 @@ __device__ void build_plan(const int32_t *idx, const float *gate, int T, int k, 
   }
   __syncwarp();
   // each pair's place among its expert's tokens (token order)
-#pragma unroll
+#pragma unroll 1
   for (int i = 0; i < FD_MAXP / 32; ++i) {
     const int p = lane + 32 * i;
     if (p < P) {
@@ -273,17 +283,20 @@ __global__ void __launch_bounds__(FD_THREADS, 1) ffn_decode_kernel(FfnArgs a) {
     // split both phases' items over the CTAs by cost, not by count: a tile
     // shared by 8 tokens costs several times a single-token tile
     if (!pl->err) {
+      // total costs: at most 128 experts x 12 x (2 I / 16 or H / 16) items,
+      // times G < 2^31 for the shapes the launch admits (checked there)
       const int U = pl->U;
       const long long W = pl->cw[U], W1 = W * 2 * I16, W2 = W * H16;
-      const int lo1 = item_at_cost(pl, U, 2 * I16, W1 * blockIdx.x / G);
-      const int hi1 = item_at_cost(pl, U, 2 * I16, W1 * (blockIdx.x + 1) / G);
-      const int lo2 = item_at_cost(pl, U, H16, W2 * blockIdx.x / G);
-      const int hi2 = item_at_cost(pl, U, H16, W2 * (blockIdx.x + 1) / G);
+      const int t1[2] = {(int)(W1 * blockIdx.x / G), (int)(W1 * (blockIdx.x + 1) / G)};
+      const int t2[2] = {(int)(W2 * blockIdx.x / G), (int)(W2 * (blockIdx.x + 1) / G)};
+      int r1[2], r2[2];
+      items_at_costs<2>(pl, U, 2 * I16, t1, r1);
+      items_at_costs<2>(pl, U, H16, t2, r2);
       if (lane == 0) {
-        pl->lo1 = lo1;
-        pl->hi1 = hi1;
-        pl->lo2 = lo2;
-        pl->hi2 = hi2;
+        pl->lo1 = r1[0];
+        pl->hi1 = r1[1];
+        pl->lo2 = r2[0];
+        pl->hi2 = r2[1];
       }
     }
   }
@@ -561,6 +574,10 @@ qmoe_status qmoe::ffn_decode_launch(const qmoe_experts *ex, const float *x, int 
       ex->down_bytes != qmoe_packed_bytes(ex->fmt, QMOE_DOWN, ex->E, ex->H, ex->I))
     return QMOE_ERR_GEOMETRY;
   if (T < 1 || T > FD_MAXT || k < 1 || k > FD_MAXK || k > ex->E) return QMOE_ERR_UNSUPPORTED;
+  // the cost split runs in 32-bit integers: at most 128 experts x cost 12 x items
+  // an expert, times the grid
+  if ((long long)FD_MAXP * 12 * ((2 * ex->I > ex->H ? 2 * ex->I : ex->H) / 16) * num_sms() >= (1LL << 31))
+    return QMOE_ERR_UNSUPPORTED;
   if (workspace_bytes < qmoe_decode_workspace_bytes(T, k, ex->H, ex->I)) return QMOE_ERR_WORKSPACE;
 
   const int bits = ex->fmt, H = ex->H, I = ex->I;
