@@ -143,7 +143,7 @@ __device__ __forceinline__ void route_token_select(const RouteArgs &a, int t, do
     }
   }
   __syncwarp();
-  warp_topk_keys<M>(key, [&](int e) { return lg[e]; }, E, a.k, a.idx + t * a.k, a.gate + t * a.k, sc);
+  warp_topk_keys<M, true>(key, [&](int e) { return lg[e]; }, E, a.k, a.idx + t * a.k, a.gate + t * a.k, sc);
 }
 
 template <int TT, bool RESID>

@@ -199,7 +199,9 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 // key[j] = key of expert l + 32 j (0 for e >= E), and val(e) returns expert
 // e's float64 logit (for the candidates only). Candidate positions come from
 // one ballot per key column, so no step waits on a chain of shuffles.
-template <int M, class Val>
+// COMPACT keeps the shuffle loops rolled: for a selection that runs once per
+// launch, the instruction fetches of unrolled code cost more than the loop.
+template <int M, bool COMPACT = false, class Val>
 __device__ __forceinline__ void warp_topk_keys(const unsigned (&key)[M], Val val, int E, int k, int32_t *idx_out,
                                                float *gate_out, TopkScratch *sc) {
   const int lane = threadIdx.x & 31;
@@ -207,7 +209,7 @@ __device__ __forceinline__ void warp_topk_keys(const unsigned (&key)[M], Val val
 #pragma unroll
   for (int j = 1; j < M; ++j) lmax = max(lmax, key[j]);
   int rank = 0;
-#pragma unroll
+#pragma unroll(COMPACT ? 1 : 32)
   for (int s2 = 0; s2 < 32; ++s2) {
     const unsigned o = __shfl_sync(0xffffffffu, lmax, s2);
     rank += (o > lmax || (o == lmax && s2 < lane)) ? 1 : 0;
@@ -237,14 +239,14 @@ __device__ __forceinline__ void warp_topk_keys(const unsigned (&key)[M], Val val
     }
     int r = 0;
     if (total <= 16) {
-#pragma unroll
+#pragma unroll(COMPACT ? 1 : 16)
       for (int i2 = 0; i2 < 16; ++i2) {
         const double v2 = __shfl_sync(0xffffffffu, cv, i2);
         const int e2 = __shfl_sync(0xffffffffu, ce, i2);
         r += (i2 < total && ranks_above(v2, e2, cv, ce)) ? 1 : 0;
       }
     } else {
-#pragma unroll
+#pragma unroll(COMPACT ? 1 : 32)
       for (int i2 = 0; i2 < 32; ++i2) {
         const double v2 = __shfl_sync(0xffffffffu, cv, i2);
         const int e2 = __shfl_sync(0xffffffffu, ce, i2);
