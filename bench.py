@@ -11,9 +11,11 @@ weights with its own roofline, clocks and CPU-oracle baseline:
   config1_layer    one Q2 decode layer, one token; steps cycle over 16 layers (weights > L2)
   config3_verify   8 correlated tokens through 48 Q4 layers (verify batch)
   config4_prefill  a 4096-token bf16 chunk through one Q4 layer
+  mixed48_decode   the 48-layer single-token stack with every fourth layer in Q4
+                   (mixed-bit stack: the fused kernel takes each layer's format)
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode48|verify48|layer|prefill] [--headline-only]
+                    [--workload decode48|verify48|mixed48|layer|prefill] [--headline-only]
 
 N > 1 runs N independent replicas (one process per GPU under torchrun; the
 path has no exchange step), timed on the device, max over ranks.
@@ -37,7 +39,8 @@ METRIC = "MoE decode tokens/s over 48 layers; HBM GB/s on weight bytes vs peak"
 PREFILL_METRIC = "MoE prefill tokens/s (4096-token bf16 chunk, one 512-expert Q4 layer); tensor TFLOP/s vs peak"
 SEED = 0
 LAYER_CYCLE = 16      # distinct layers the single-layer steps cycle over (weights > L2)
-WORKLOADS = {"decode48": 2, "verify48": 3, "layer": 1, "prefill": 4}
+WORKLOADS = {"decode48": 2, "verify48": 3, "mixed48": 2, "layer": 1, "prefill": 4}
+MIXED_EVERY = 4       # mixed48: layers 0, 4, 8, ... in Q4, the others in Q2
 
 
 def parse():
@@ -77,11 +80,19 @@ def tensor_peak():
     return 1590.0, "fallback (burst)"
 
 
+def format_desc(cfg):
+    if not cfg.fmt_layers:
+        return f"Q{cfg.fmt}"
+    n4 = sum(1 for f in cfg.fmt_layers if f == 4)
+    return f"mixed: Q4 in {n4} of {cfg.L} layers (every {MIXED_EVERY}th from layer 0), Q2 in the rest"
+
+
 def workload_desc(cfg, T):
     return {"workload": f"{cfg.L}-layer routed-MoE decode stack: {cfg.E} experts/layer, hidden {cfg.H}, "
-                        f"intermediate {cfg.I}, top-{cfg.k}, Q{cfg.fmt} blocks, {T} token(s)/step, residual RMSNorm",
+                        f"intermediate {cfg.I}, top-{cfg.k}, {format_desc(cfg)} blocks, {T} token(s)/step, "
+                        f"residual RMSNorm",
             "layers": cfg.L, "experts_per_layer": cfg.E, "hidden": cfg.H, "intermediate": cfg.I, "top_k": cfg.k,
-            "format": f"Q{cfg.fmt}", "tokens_per_step": T, "seed": SEED,
+            "format": format_desc(cfg), "tokens_per_step": T, "seed": SEED,
             "l2": "no flush: each step streams ~0.85-3.5 GB of distinct experts (> 126 MB L2); "
                   "a fresh token is drawn for every step"}
 
@@ -222,7 +233,8 @@ def barrier(world):
 TRAFFIC_PROFILES = {
     # kernel -> (committed ncu summary, sources that define the kernel)
     "stack_decode": ("stack_decode_decode48_ncu.md",
-                     ("stack_decode.cu", "decode_tile.cuh", "common.cuh", "layout.cuh", "route_common.cuh")),
+                     ("stack_decode.cu", "decode_tile.cuh", "common.cuh", "layout.cuh", "route_common.cuh",
+                      "decode_canon.cuh")),
     "pf_gemm1": ("pf_gemm_prefill4096_ncu.md", ("prefill.cu", "tc05.cuh", "common.cuh", "layout.cuh")),
     # per algorithmic byte (a launch's bytes depend on its routes): scaled to the measured launches
     "ffn_decode_t8": ("ffn_decode_verify8_ncu.md",
@@ -292,8 +304,8 @@ def oracle_token_time(cfg, x0, n_layers):
     from synth import gen
     x = x0.astype(np.float64)
     spent = 0.0
-    bits = cfg.format.bits
     for l in range(n_layers):
+        bits = cfg.for_layer(l).format.bits
         Wr, b = gen.router(SEED, cfg, l), gen.bias(SEED, cfg, l)
         t0 = time.perf_counter()
         idx, g, _ = moe.route(x, Wr, b, cfg.k)
@@ -334,7 +346,6 @@ def run_reference(args, cfg, T):
     import numpy as np
     from oracle import moe
     from synth import gen
-    bits = cfg.format.bits
     x = gen.tokens(SEED, cfg, 0).astype(np.float64)
     state = {"l": 0, "idx": None, "g": None, "raw": None, "outs": {}}
 
@@ -348,9 +359,9 @@ def run_reference(args, cfg, T):
             idx, g, _ = moe.route(state.get("x", x), Wr, b, cfg.k)
             t += time.perf_counter() - t0
             state["idx"], state["g"] = idx, g
-            e0 = int(idx[0, 0])
         e = int(state["idx"][0, j])
         raw = gen.expert(SEED, cfg, l, e)
+        bits = cfg.for_layer(l).format.bits
         t0 = time.perf_counter()
         W = tuple(moe.dequantize(raw[n + "_codes"], raw[n + "_scales"], bits) for n in ("gate", "up", "down"))
         xx = state.get("x", x)
@@ -515,7 +526,7 @@ def measure_stack(args, cfg, seed=SEED, full=True):
     free_device()
 
     hbm, peak_kind = peaks()
-    ffn_bytes = [u * cfg.expert_bytes() for u in uniq]
+    ffn_bytes = [u * cfg.for_layer(l).expert_bytes() for l, u in enumerate(uniq)]
     expert_bytes_step = sum(ffn_bytes)
     router_bytes_step = cfg.L * cfg.router_bytes()
     step_s = ms / 1e3 / args.steps
@@ -533,7 +544,8 @@ def measure_stack(args, cfg, seed=SEED, full=True):
     out.update({
         "roofline": {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": hbm,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": (stored_traffic("stack_decode") if cfg.L == 48 else None) if fused
+                     "traffic": (stored_traffic("stack_decode") if cfg.L == 48 and not cfg.fmt_layers
+                                 else None) if fused
                      else scaled_traffic("ffn_decode_t8" if cfg.T > 1 else "ffn_decode_t1", launch_bytes),
                      "algorithmic_bytes_per_launch": launch_bytes, "avg_launch_us": 1e6 * launch_s,
                      "timing": f"CUDA event nodes around the kernel node(s) of a graph, mean of {n_t} replays"},
@@ -889,8 +901,10 @@ def main():
     cfg = configs.get(WORKLOADS[args.workload])
     if args.workload == "prefill" and args.tokens:
         cfg = cfg.with_(T=args.tokens)
-    if args.workload in ("decode48", "verify48") and args.layers:
+    if args.workload in ("decode48", "verify48", "mixed48") and args.layers:
         cfg = cfg.with_(L=args.layers)
+    if args.workload == "mixed48":
+        cfg = configs.mixed(cfg, MIXED_EVERY)
     if args.impl == "reference" and args.workload == "prefill":
         run_prefill_reference(args, cfg)
         return
@@ -917,8 +931,11 @@ def main():
             c3 = configs.get(3)
             line["config3_verify"] = sub_line(stack_line(args, c3, measure_stack(args, c3)))
             line["config4_prefill"] = sub_line(run_prefill(args, configs.get(4)))
+            mx = configs.mixed(cfg, MIXED_EVERY)
+            line["mixed48_decode"] = sub_line(stack_line(args, mx, measure_stack(args, mx)))
             line["gpu_launches_all_workloads"] = (line["gpu_launches"] + sum(
-                line[k_]["gpu_launches"] for k_ in ("config1_layer", "config3_verify", "config4_prefill")))
+                line[k_]["gpu_launches"] for k_ in ("config1_layer", "config3_verify", "config4_prefill",
+                                                    "mixed48_decode")))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -10,8 +10,9 @@
  *        paragraph).
  *   [P3] pyshine, Strata source-tree tour - "Understanding the Architecture":
  *        48 captured layer graphs fed through fixed-address device buffers; a
- *        gate-weighted moe_combine summed on the device; wrong expert geometry
- *        refused rather than mis-indexed; router_top10.cu routes each token to
+ *        gate-weighted moe_combine summed on the device; expert buffers whose
+ *        geometry disagrees get an error, never a read at wrong offsets;
+ *        router_top10.cu routes each token to
  *        ten experts; batched prefill in chunks of up to 8,192 tokens.
  *
  * Conventions shared by every call
@@ -281,7 +282,7 @@ typedef struct {
   float eps;
   const float *const *Wr;      /* L device pointers, fp32 [E,H] */
   const float *const *bias;    /* NULL or L device pointers (entries may be NULL) */
-  const qmoe_experts *layers;  /* L handles with identical E/H/I/fmt */
+  const qmoe_experts *layers;  /* L handles with identical E/H/I; fmt may differ per layer */
   int flags;                   /* 0 or a combination of QMOE_STACK_TIMING, QMOE_STACK_LAYERWISE */
 } qmoe_stack_desc;
 
@@ -308,7 +309,8 @@ int qmoe_stack_kernels_per_replay(const qmoe_stack *stack);
  * QMOE_ERR_TIMEOUT after about one second instead of hanging. */
 uint32_t *qmoe_stack_barrier_word(const qmoe_stack *stack);
 /* Which path the stack runs. QMOE_PATH_FUSED (single-token stacks whose
- * geometry fits one SM's shared memory): one persistent kernel runs all L
+ * geometry fits one SM's shared memory; a stack that mixes formats is laid
+ * out for Q4 and takes each layer's format in turn): one persistent kernel runs all L
  * layers with two grid barriers per layer. QMOE_PATH_LAYERWISE:
  * qmoe_residual_route and qmoe_ffn_decode per layer, chained with
  * programmatic dependent launch. Both paths form a token's router logits from

@@ -27,7 +27,7 @@ class Layer:
         """float64 (Wg [I,H], Wu [I,H], Wd [H,I]) of expert ``e``."""
         if e not in self._cache:
             raw = gen.expert(self.seed, self.cfg, self.layer, e)
-            bits = self.cfg.format.bits
+            bits = self.cfg.for_layer(self.layer).format.bits
             self._cache[e] = tuple(
                 moe.dequantize(raw[n + "_codes"], raw[n + "_scales"], bits)
                 for n in ("gate", "up", "down"))

@@ -48,11 +48,19 @@ struct Layout {
   qmoe::FusedPlan fplan;
 };
 
+// The stack's block format, or 0 when its layers mix formats.
+int stack_fmt(const qmoe_stack_desc *d) {
+  for (int l = 1; l < d->L; ++l)
+    if (d->layers[l].fmt != d->layers[0].fmt) return 0;
+  return d->layers[0].fmt;
+}
+
 Layout layout_of(const qmoe_stack_desc *d) {
   const qmoe_experts &e = d->layers[0];
   Layout l;
+  const int fmt = stack_fmt(d);
   l.use_fused = d->T == 1 && !(d->flags & QMOE_STACK_LAYERWISE) &&
-                qmoe::fused_stack_plan(e.fmt, e.E, e.H, e.I, d->k, &l.fplan);
+                qmoe::fused_stack_plan(fmt ? fmt : QMOE_Q4, e.E, e.H, e.I, d->k, &l.fplan);
   l.fused = l.use_fused ? al(qmoe::fused_stack_ws_bytes(d->L, e.E, e.H, e.I, d->k)) : 0;
   l.trace = (l.use_fused && (d->flags & QMOE_STACK_TIMING))
                 ? al((size_t)d->L * qmoe::num_sms() * qmoe::fused_trace_points() * sizeof(long long))
@@ -73,7 +81,8 @@ qmoe_status check_desc(const qmoe_stack_desc *d) {
   const qmoe_experts &e0 = d->layers[0];
   for (int l = 0; l < d->L; ++l) {
     const qmoe_experts &e = d->layers[l];
-    if (e.E != e0.E || e.H != e0.H || e.I != e0.I || e.fmt != e0.fmt) return QMOE_ERR_GEOMETRY;
+    if (e.E != e0.E || e.H != e0.H || e.I != e0.I) return QMOE_ERR_GEOMETRY;  // formats may differ
+    if (e.fmt != QMOE_Q2 && e.fmt != QMOE_Q4) return QMOE_ERR_UNSUPPORTED;
     if (e.gate_up_bytes != qmoe_packed_bytes(e.fmt, QMOE_GATE_UP, e.E, e.H, e.I) ||
         e.down_bytes != qmoe_packed_bytes(e.fmt, QMOE_DOWN, e.E, e.H, e.I))
       return QMOE_ERR_GEOMETRY;
@@ -171,7 +180,7 @@ extern "C" qmoe_status qmoe_stack_create(const qmoe_stack_desc *d, void *workspa
   qmoe_stack *s = new (std::nothrow) qmoe_stack();
   if (!s) return QMOE_ERR_CUDA;
   const qmoe_experts &e0 = d->layers[0];
-  s->L = d->L; s->T = d->T; s->k = d->k; s->E = e0.E; s->H = e0.H; s->I = e0.I; s->fmt = e0.fmt;
+  s->L = d->L; s->T = d->T; s->k = d->k; s->E = e0.E; s->H = e0.H; s->I = e0.I; s->fmt = stack_fmt(d);
   s->eps = d->eps;
   s->Wr.assign(d->Wr, d->Wr + d->L);
   s->bias.assign(d->L, nullptr);

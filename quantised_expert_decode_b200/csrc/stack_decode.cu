@@ -70,6 +70,7 @@ struct StackArgs {
   const uint8_t *const *gu;   // [L] packed gate/up tiles per layer
   const uint8_t *const *dn;   // [L] packed down tiles per layer
   const float *const *bias;   // [L], entries may be null
+  const int32_t *fmt;         // [L] block format per layer (read when the kernel's BITS is 0)
   const float *wrt;           // [L][H][E] routers, transposed
   const float *x_in;          // [H]
   float *x_out;               // [H]
@@ -206,12 +207,26 @@ __device__ __noinline__ void quant_h_block(const StackArgs &a, const float *hl, 
   if (lane == 0) a.lscg[(size_t)j * nblkI + b] = make_float2(sc, __fmul_rn(sc, (float)sx));
 }
 
+// A tile's dot product in the layer's block format: BITS when the stack has
+// one format, else the layer's own (bl).
+template <int BITS>
+__device__ __forceinline__ float2 tile_dot_fmt(int bl, const uint8_t *tile, int nblk, const uint8_t *limbs,
+                                               const float2 *lsc) {
+  if constexpr (BITS != 0) {
+    return tile_dot1<BITS, 1>(tile, nblk, limbs, lsc);
+  } else {
+    return bl == QMOE_Q2 ? tile_dot1<QMOE_Q2, 1>(tile, nblk, limbs, lsc) : tile_dot1<QMOE_Q4, 1>(tile, nblk, limbs, lsc);
+  }
+}
+
+// BITS: the stack's block format, or 0 for a stack whose layers mix formats
+// (shared memory laid out for the widest, Q4; tile sizes per layer).
 template <int BITS>
 __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int S = a.nslots;
   const int H = a.H, I = a.I, E = a.E, k = a.k, L = a.L;
-  const SkLayout lay = sk_layout(BITS, E, H, I, k, S, a.slot_bytes, (int)gridDim.x);
+  const SkLayout lay = sk_layout(BITS ? BITS : QMOE_Q4, E, H, I, k, S, a.slot_bytes, (int)gridDim.x);
   uint8_t *ring = smem + lay.ring;
   uint8_t *dnbuf = smem + lay.dnbuf;
   float *wrtbuf = reinterpret_cast<float *>(smem + lay.wrtbuf);
@@ -232,7 +247,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nblkH = H / 32, nblkI = I / 32, I16 = I / 16, H16 = H / 16;
-  const int tgu = tile_bytes(BITS, H), tdn = tile_bytes(BITS, I);
+  const int tgu0 = tile_bytes(BITS ? BITS : QMOE_Q4, H), tdn0 = tile_bytes(BITS ? BITS : QMOE_Q4, I);
   const int G = (int)gridDim.x, c = blockIdx.x;
   const bool rows = c < H16;
   const int r0 = 16 * c;
@@ -324,6 +339,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
 
   for (int l = 0; l < L; ++l) {
     const int par = l & 1;
+    const int bl = BITS ? BITS : __ldg(a.fmt + l);
+    const int tgu = BITS ? tgu0 : tile_bytes(bl, H), tdn = BITS ? tdn0 : tile_bytes(bl, I);
     if (tid == 0) {
       trace_point(a, l, TP_START);
       // points of phases a CTA has no work in stay 0
@@ -505,7 +522,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
       if (!wait_full(n)) break;
       if (tid == 0 && m == 0) trace_point(a, l, TP_FIRST_TILE);
       const int i = ilo + m, u = i >> 1, mat = i & 1, j = u / I16, r = u % I16;
-      const float2 o = tile_dot1<BITS, 1>(ring + (size_t)(n % S) * a.slot_bytes, nblkH, limbs, lsc);
+      const float2 o = tile_dot_fmt<BITS>(bl, ring + (size_t)(n % S) * a.slot_bytes, nblkH, limbs, lsc);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[n % S]);
       // this tile's 16 rows into the local block: a_g / a_u of rows 16 (r & 1) ..
@@ -556,8 +573,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
       bool ok = mbar_wait(dnbar, (uint32_t)(l & 1), clock64() + WAIT_BUDGET_CYCLES);
       if (ok) {
         for (int j = warp; j < k; j += SK_NCW) {
-          const float2 o = tile_dot1<BITS, 1>(dnbuf + (size_t)j * tdn, nblkI, limbs + (size_t)j * nblkI * LIMB_REC,
-                                           lsc + (size_t)j * nblkI);
+          const float2 o = tile_dot_fmt<BITS>(bl, dnbuf + (size_t)j * tdn, nblkI,
+                                              limbs + (size_t)j * nblkI * LIMB_REC, lsc + (size_t)j * nblkI);
           if ((lane & 3) == 0) {
             const int g = lane >> 2;
             ytmp[j * 16 + g] = o.x;
@@ -657,7 +674,7 @@ size_t fused_stack_ws_bytes(int L, int E, int H, int I, int k) {
   auto a = [](size_t v) { return (v + 255) & ~(size_t)255; };
   const size_t nb = (size_t)k * (I / 32);
   return a((size_t)L * H * E * 4) + a(2 * (size_t)E * 8) + a(2 * (size_t)(H / 16) * 8) + a(2 * (size_t)H * 4) +
-         a(nb * LIMB_REC) + a(nb * 8) + 256 + 3 * a((size_t)L * 8);
+         a(nb * LIMB_REC) + a(nb * 8) + 256 + 3 * a((size_t)L * 8) + a((size_t)L * 4);
 }
 
 
@@ -675,7 +692,8 @@ FusedBufs fused_carve(void *ws, int L, int E, int H, int I, int k) {
   b.bar = reinterpret_cast<unsigned *>(p); p += 256;
   b.gu = reinterpret_cast<const uint8_t **>(p); p += a((size_t)L * 8);
   b.dn = reinterpret_cast<const uint8_t **>(p); p += a((size_t)L * 8);
-  b.bias = reinterpret_cast<const float **>(p);
+  b.bias = reinterpret_cast<const float **>(p); p += a((size_t)L * 8);
+  b.fmt = reinterpret_cast<int32_t *>(p);
   return b;
 }
 
@@ -700,14 +718,17 @@ qmoe_status fused_prepare(const FusedBufs &b, int L, int E, int H, const float *
     note_launch();
   }
   std::vector<const void *> gu(L), dn(L), bi(L);
+  std::vector<int32_t> fm(L);
   for (int l = 0; l < L; ++l) {
     gu[l] = layers[l].gate_up;
     dn[l] = layers[l].down;
     bi[l] = bias ? bias[l] : nullptr;
+    fm[l] = layers[l].fmt;
   }
   if (cudaMemcpyAsync((void *)b.gu, gu.data(), L * 8, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync((void *)b.dn, dn.data(), L * 8, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync((void *)b.bias, bi.data(), L * 8, cudaMemcpyHostToDevice, s) != cudaSuccess)
+      cudaMemcpyAsync((void *)b.bias, bi.data(), L * 8, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync((void *)b.fmt, fm.data(), L * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return QMOE_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return QMOE_ERR_CUDA;
   return cuda_status(cudaGetLastError());
@@ -718,7 +739,7 @@ qmoe_status fused_launch(const FusedBufs &b, const FusedPlan &p, int fmt, int L,
                          long long *trace, cudaStream_t s, bool cooperative) {
   StackArgs a{};
   a.L = L; a.E = E; a.H = H; a.I = I; a.k = k; a.eps = eps;
-  a.gu = b.gu; a.dn = b.dn; a.bias = b.bias; a.wrt = b.wrt;
+  a.gu = b.gu; a.dn = b.dn; a.bias = b.bias; a.fmt = b.fmt; a.wrt = b.wrt;
   a.x_in = x_in; a.x_out = x_out; a.idx_rec = idx_rec; a.gate_rec = gate_rec;
   a.zbuf = b.zbuf; a.lacc = b.lacc; a.ssq = b.ssq; a.bar = b.bar; a.status = status;
   a.lbuf = b.lbuf; a.lscg = b.lscg;
@@ -730,7 +751,9 @@ qmoe_status fused_launch(const FusedBufs &b, const FusedPlan &p, int fmt, int L,
   const int G = num_sms();
   a.w_rows = 1;
   a.w_free = 1;
-  const void *fn = fmt == 2 ? (const void *)stack_decode_kernel<2> : (const void *)stack_decode_kernel<4>;
+  const void *fn = fmt == QMOE_Q2   ? (const void *)stack_decode_kernel<QMOE_Q2>
+                   : fmt == QMOE_Q4 ? (const void *)stack_decode_kernel<QMOE_Q4>
+                                    : (const void *)stack_decode_kernel<0>;
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) != cudaSuccess)
     return QMOE_ERR_CUDA;
   cudaLaunchConfig_t cfg{};
@@ -743,8 +766,9 @@ qmoe_status fused_launch(const FusedBufs &b, const FusedPlan &p, int fmt, int L,
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = cooperative ? 1 : 0;
-  cudaError_t e = fmt == 2 ? cudaLaunchKernelEx(&cfg, stack_decode_kernel<2>, a)
-                           : cudaLaunchKernelEx(&cfg, stack_decode_kernel<4>, a);
+  cudaError_t e = fmt == QMOE_Q2   ? cudaLaunchKernelEx(&cfg, stack_decode_kernel<QMOE_Q2>, a)
+                  : fmt == QMOE_Q4 ? cudaLaunchKernelEx(&cfg, stack_decode_kernel<QMOE_Q4>, a)
+                                   : cudaLaunchKernelEx(&cfg, stack_decode_kernel<0>, a);
   note_launch();
   return cuda_status(e);
 }

@@ -27,13 +27,18 @@ struct FusedBufs {
   unsigned *bar;
   const uint8_t **gu, **dn;
   const float **bias;
+  int32_t *fmt;                    // [L] block format of each layer
 };
 
+// fmt: the stack's one block format, or QMOE_Q4 for a stack that mixes
+// formats (its shared-memory layout is the widest format's).
 bool fused_stack_plan(int fmt, int E, int H, int I, int k, FusedPlan *p);
 size_t fused_stack_ws_bytes(int L, int E, int H, int I, int k);
 FusedBufs fused_carve(void *ws, int L, int E, int H, int I, int k);
 qmoe_status fused_prepare(const FusedBufs &b, int L, int E, int H, const float *const *Wr,
                           const qmoe_experts *layers, const float *const *bias, cudaStream_t s);
+// fmt: the stack's block format, or 0 when the layers mix formats (the kernel
+// then reads each layer's format from the prepared table).
 // trace: null, or [L][grid][fused_trace_points()] int64 SM-clock stamps per
 // layer and CTA (layer start, top-k done, gate/up tiles start and done, first
 // grid barrier passed, down tiles done, second grid barrier passed).

@@ -66,6 +66,7 @@ class Config:
     residual: bool  # x <- RMSNorm(x + y) between layers
     eps: float = 1e-6
     router_std: float = 0.02
+    fmt_layers: tuple = ()   # per-layer block format (mixed-bit stack); empty: every layer is `fmt`
 
     @property
     def format(self) -> Fmt:
@@ -78,6 +79,14 @@ class Config:
 
     def router_bytes(self) -> int:
         return self.E * self.H * 4
+
+    def for_layer(self, layer: int) -> "Config":
+        """This configuration with layer ``layer``'s block format (a mixed-bit
+        stack gives its layers different formats; the streams do not depend
+        on the format)."""
+        if not self.fmt_layers:
+            return self
+        return replace(self, fmt=self.fmt_layers[layer], fmt_layers=())
 
     def with_(self, **kw) -> "Config":
         return replace(self, **kw)
@@ -104,3 +113,10 @@ CONFIGS = {
 
 def get(cid: int) -> Config:
     return CONFIGS[cid]
+
+
+def mixed(cfg: Config, every: int = 4) -> Config:
+    """``cfg`` as a mixed-bit stack: layers 0, every, 2 every, ... in Q4, the
+    others in Q2. Same configuration id, so its Q2 layers are ``cfg``'s own
+    when ``cfg`` is a Q2 stack."""
+    return cfg.with_(fmt_layers=tuple(Q4 if l % every == 0 else Q2 for l in range(cfg.L)))

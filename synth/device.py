@@ -52,7 +52,7 @@ def fill_codes(seed: int, cfg: Config, layer: int, mat: int, dst, e0: int = 0) -
 
 def fill_scales(seed: int, cfg: Config, layer: int, mat: int, dst, e0: int = 0) -> None:
     """dst: uint16 tensor [E, rows, K/32, 2] (fp16 bit patterns of (d, m))."""
-    f = cfg.format
+    f = cfg.for_layer(layer).format
     E = dst.shape[0]
     nblk = dst[0].numel() // 2
     rc = lib().synth_fill_scales(seed & rng.MASK64, cfg.cid, layer, e0, E, WHAT_SCALES[mat], nblk,

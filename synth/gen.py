@@ -64,6 +64,7 @@ def scale_pairs(key: int, nblocks: int, fmt: int) -> np.ndarray:
 
 def expert_matrix(seed: int, cfg: Config, layer: int, expert: int, mat: int):
     """(codes uint8 [rows, K*bits/8], scales uint16 [rows, K/32, 2])."""
+    cfg = cfg.for_layer(layer)
     rows, K = matrix_shape(cfg, mat)
     bits = cfg.format.bits
     codes = code_bytes(codes_key(seed, cfg, layer, expert, mat), rows * K * bits // 8)

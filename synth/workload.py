@@ -18,11 +18,14 @@ def device_layers(seed: int, cfg: Config, n_layers: int | None = None, dev="cuda
     from quantised_expert_decode_b200.model import PackedLayer
 
     n = cfg.L if n_layers is None else n_layers
-    canon = device.alloc_canonical(cfg, dev)
+    canon, canon_fmt = None, None
     layers, routers, biases = [], [], []
     for l in range(first, first + n):
+        lc = cfg.for_layer(l)
+        if canon_fmt != lc.fmt:   # the canonical code buffers depend on the format
+            canon, canon_fmt = device.alloc_canonical(lc, dev), lc.fmt
         device.fill_layer(seed, cfg, l, canon)
-        layers.append(PackedLayer(cfg.fmt, cfg.E, cfg.H, cfg.I, dev).pack(canon))
+        layers.append(PackedLayer(lc.fmt, cfg.E, cfg.H, cfg.I, dev).pack(canon))
         routers.append(torch.from_numpy(gen.router(seed, cfg, l)).to(dev))
         b = gen.bias(seed, cfg, l)
         biases.append(None if b is None else torch.from_numpy(b).to(dev))

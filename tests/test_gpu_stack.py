@@ -225,3 +225,56 @@ def test_fused_phase_trace_is_ordered_and_layer_times_add_up():
     assert torch.equal(plain.x_out, st.x_out)     # stamping changes no result
     plain.close()
     st.close()
+
+
+
+MIXED6 = (configs.Q2, configs.Q4, configs.Q4, configs.Q2, configs.Q4, configs.Q2)
+
+
+@pytest.mark.parametrize("layerwise", [False, True])
+def test_mixed_bit_stack_small_geometry(layerwise):
+    """A stack whose layers use different block formats (Q2 and Q4 per layer)
+    matches the oracle on both paths: the fused kernel takes each layer's
+    format in turn, the per-layer kernels get each layer's handle."""
+    cfg = configs.get(0).with_(L=6, residual=True, fmt_layers=MIXED6)
+    stack, x0, built = _run(cfg, 6, layerwise=layerwise)
+    assert [l.fmt for l in built[0]] == list(MIXED6)
+    assert stack.path == (L.PATH_LAYERWISE if layerwise else L.PATH_FUSED)
+    _compare(cfg, stack, x0, 6, built, layerwise)
+    stack.close()
+
+
+def test_mixed_bit_stack_decode_geometry_and_verify_batch():
+    """Decode geometry (512 experts, H 2048, I 768, top-10) with a block
+    format per layer: one token (fused kernel) and an 8-token verify batch
+    (per-layer kernels) match the oracle; the per-layer path gives the fused
+    path's bits, and every token of the batch equals that token decoded
+    alone, bit for bit."""
+    n = 4
+    fl = (configs.Q4, configs.Q2, configs.Q2, configs.Q4)
+    cfg1 = configs.get(2).with_(L=n, fmt_layers=fl)
+    built = device_layers(SEED, cfg1, n)
+    layers, routers, biases = built
+    assert sum(l.nbytes for l in layers) == sum(cfg1.E * cfg1.for_layer(l).expert_bytes() for l in range(n))
+    one, x0, _ = _run(cfg1, n, built=built)
+    assert one.path == L.PATH_FUSED
+    _compare(cfg1, one, x0, n, built)
+    one_lw, _, _ = _run(cfg1, n, built=built, layerwise=True)
+    _same_bits(one, one_lw)
+
+    cfg8 = cfg1.with_(T=8, x_kind="correlated")   # same configuration id: same layers
+    batch, xb, _ = _run(cfg8, n, built=built)
+    assert batch.path == L.PATH_LAYERWISE
+    _compare(cfg8, batch, xb, n, built, layerwise=True)
+    x8 = torch.from_numpy(xb).cuda()
+    for t in range(cfg8.T):
+        for s in (one, one_lw):
+            s.x_in.copy_(x8[t:t + 1])
+            s.decode()
+            torch.cuda.synchronize()
+            assert s.status() == 0
+            assert torch.equal(s.idx[:, 0], batch.idx[:, t]), (t, s.path)
+            assert torch.equal(s.gate[:, 0], batch.gate[:, t]), (t, s.path)
+            assert torch.equal(s.x_out[0], batch.x_out[t]), (t, s.path)
+    for s in (one, one_lw, batch):
+        s.close()

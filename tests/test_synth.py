@@ -96,3 +96,28 @@ def test_expert_matrix_shapes():
     cfg4 = configs.get(4)
     assert cfg4.expert_bytes() == 2_949_120
     assert configs.get(1).expert_bytes() == 1_769_472
+
+
+def test_mixed_bit_stack_layers_are_the_uniform_layers():
+    """A mixed-bit stack (a block format per layer) draws layer l's codes and
+    scales from the same streams as the uniform stack of layer l's format,
+    and the oracle dequantises each layer with that layer's bits."""
+    from oracle import workload as W
+    base = configs.get(0).with_(L=3, residual=True)
+    mixed = base.with_(fmt_layers=(configs.Q2, configs.Q4, configs.Q2))
+    assert mixed.for_layer(1).fmt == configs.Q4 and mixed.for_layer(1).fmt_layers == ()
+    assert base.for_layer(1) is base
+    for l in range(3):
+        uni = base.with_(fmt=mixed.fmt_layers[l])
+        a, b = gen.expert(0, mixed, l, 7), gen.expert(0, uni, l, 7)
+        assert a.keys() == b.keys()
+        for n in a:
+            assert np.array_equal(a[n], b[n]), (l, n)
+        bits = 8 * a["gate_codes"].shape[1] // base.H
+        assert bits == mixed.fmt_layers[l]
+        for wa, wb in zip(W.Layer(0, mixed, l).expert(7), W.Layer(0, uni, l).expert(7)):
+            assert np.array_equal(wa, wb)
+    # the Q4 layer really is four-bit: 16 distinct code levels per block
+    w = W.Layer(0, mixed, 1).expert(3)[0]
+    blk = w[0, :32]
+    assert len(np.unique(blk)) > 4
