@@ -237,6 +237,9 @@ TRAFFIC_PROFILES = {
                       "decode_canon.cuh")),
     "pf_gemm1": ("pf_gemm_prefill4096_ncu.md", ("prefill.cu", "tc05.cuh", "common.cuh", "layout.cuh")),
     # per algorithmic byte (a launch's bytes depend on its routes): scaled to the measured launches
+    "stack_decode_mixed": ("stack_decode_mixed48_ncu.md",
+                           ("stack_decode.cu", "decode_tile.cuh", "common.cuh", "layout.cuh", "route_common.cuh",
+                            "decode_canon.cuh")),
     "ffn_decode_t8": ("ffn_decode_verify8_ncu.md",
                       ("ffn_decode.cu", "decode_tile.cuh", "common.cuh", "layout.cuh", "decode_canon.cuh")),
     "ffn_decode_t1": ("ffn_decode_layer1_ncu.md",
@@ -541,12 +544,16 @@ def measure_stack(args, cfg, seed=SEED, full=True):
         launch_bytes = float(statistics.mean(ffn_bytes))
         launch_s = float(ffn_ms.mean()) / 1e3
         achieved = statistics.mean(b / (t / 1e3) for b, t in zip(ffn_bytes, ffn_ms)) / 1e9
+    if fused and cfg.fmt_layers:
+        traffic = scaled_traffic("stack_decode_mixed", launch_bytes)
+    elif fused:
+        traffic = stored_traffic("stack_decode") if cfg.L == 48 else None
+    else:
+        traffic = scaled_traffic("ffn_decode_t8" if cfg.T > 1 else "ffn_decode_t1", launch_bytes)
     out.update({
         "roofline": {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": hbm,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": (stored_traffic("stack_decode") if cfg.L == 48 and not cfg.fmt_layers
-                                 else None) if fused
-                     else scaled_traffic("ffn_decode_t8" if cfg.T > 1 else "ffn_decode_t1", launch_bytes),
+                     "traffic": traffic,
                      "algorithmic_bytes_per_launch": launch_bytes, "avg_launch_us": 1e6 * launch_s,
                      "timing": f"CUDA event nodes around the kernel node(s) of a graph, mean of {n_t} replays"},
         "stack": {"path": "fused persistent kernel" if fused else "per-layer kernels (route + FFN) with PDL",
