@@ -61,6 +61,10 @@ enum {
   TP_START = 0, TP_TOPK, TP_TILES, TP_TILES_DONE, TP_BAR1, TP_DOWN_DONE, TP_BAR2, TP_LOGITS,
   TP_FIRST_TILE, TP_LIMBS, TP_DOWN_TILES, TP_Z
 };
+// z and its slice sums of squares are written in Z_COPIES copies and CTA c
+// reads copy c % Z_COPIES: every CTA reads all of them right after a grid
+// barrier, and fewer readers per cache line shorten phase A.
+constexpr int Z_COPIES = 4;
 constexpr int CONS_BAR = 1;   // the consumer warps
 constexpr int PLAN_BAR = 2;   // consumer warp 0 and the producer warp
 
@@ -76,9 +80,9 @@ struct StackArgs {
   float *x_out;               // [H]
   int32_t *idx_rec;           // [L][k]
   float *gate_rec;            // [L][k]
-  float *zbuf;                // [2][H]
+  float *zbuf;                // [Z_COPIES][2 parity][H]
   unsigned long long *lacc;   // [2 parity][E] integer partial-logit sums (2^-32 units, two's complement)
-  double *ssq;                // [2 parity][H/16] slice sums of squares
+  double *ssq;                // [Z_COPIES][2 parity][H/16] slice sums of squares
   uint8_t *lbuf;              // [k][I/32][LIMB_REC]: limbs of h
   float2 *lscg;               // [k][I/32]: (s, s * sum X) of h's blocks
   unsigned *bar;
@@ -294,7 +298,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
     if (tid < 16) {
       const float z = a.x_in[r0 + tid];
       st->ztmp[tid] = z;
-      a.zbuf[r0 + tid] = z;
+      for (int cp = 0; cp < Z_COPIES; ++cp) a.zbuf[(size_t)cp * 2 * H + r0 + tid] = z;
     }
     named_barrier_sync(CONS_BAR, nth);
     if (!mbar_wait(wrtbar, 0u, clock64() + WAIT_BUDGET_CYCLES)) {
@@ -351,13 +355,14 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
     // ------------------------------------------------------------------ A --
     if (!producer && !*(volatile int *)&st->abort) {
       // one batch of loads: sum of squares, z, partial logits, bias
-      const float4 *zb = reinterpret_cast<const float4 *>(a.zbuf + (size_t)par * H);
+      const int zc = c % Z_COPIES;
+      const float4 *zb = reinterpret_cast<const float4 *>(a.zbuf + ((size_t)zc * 2 + par) * H);
       const float *b = a.bias[l];
       const unsigned long long *la = a.lacc + (size_t)par * E;
       float4 zv[4];
       unsigned long long lh[4];
       float bv[4];
-      const double *sq = a.ssq + (size_t)par * H16;
+      const double *sq = a.ssq + ((size_t)zc * 2 + par) * H16;
       double sv[4];   // this lane's first slice sums of squares (decode_canon.cuh's order)
 #pragma unroll
       for (int m = 0; m < 4; ++m) sv[m] = (l > 0 && lane + 32 * m < H16) ? __ldcg(sq + lane + 32 * m) : 0.0;
@@ -593,10 +598,12 @@ __global__ void __launch_bounds__(SK_THREADS, 1) stack_decode_kernel(StackArgs a
           for (int j = 0; j < k; ++j) y = canon::combine_step(y, st->gate[j], ytmp[j * 16 + lane]);  // slot order
           const float z = __fadd_rn(xs[r0 + lane], y);
           st->ztmp[lane] = z;
-          a.zbuf[(size_t)(par ^ 1) * H + r0 + lane] = z;
+#pragma unroll
+          for (int cp = 0; cp < Z_COPIES; ++cp) a.zbuf[((size_t)cp * 2 + (par ^ 1)) * H + r0 + lane] = z;
         }
         __syncwarp();
-        if (lane == 0) a.ssq[(size_t)(par ^ 1) * H16 + c] = canon::slice_sumsq([&](int i) { return st->ztmp[i]; });
+        if (lane < Z_COPIES)
+          a.ssq[((size_t)lane * 2 + (par ^ 1)) * H16 + c] = canon::slice_sumsq([&](int i) { return st->ztmp[i]; });
       }
       named_barrier_sync(CONS_BAR, nth);
       if (tid == 0) trace_point(a, l, TP_Z);
@@ -673,7 +680,7 @@ bool fused_stack_plan(int fmt, int E, int H, int I, int k, FusedPlan *p) {
 size_t fused_stack_ws_bytes(int L, int E, int H, int I, int k) {
   auto a = [](size_t v) { return (v + 255) & ~(size_t)255; };
   const size_t nb = (size_t)k * (I / 32);
-  return a((size_t)L * H * E * 4) + a(2 * (size_t)E * 8) + a(2 * (size_t)(H / 16) * 8) + a(2 * (size_t)H * 4) +
+  return a((size_t)L * H * E * 4) + a(2 * (size_t)E * 8) + a(Z_COPIES * 2 * (size_t)(H / 16) * 8) + a(Z_COPIES * 2 * (size_t)H * 4) +
          a(nb * LIMB_REC) + a(nb * 8) + 256 + 3 * a((size_t)L * 8) + a((size_t)L * 4);
 }
 
@@ -684,8 +691,8 @@ FusedBufs fused_carve(void *ws, int L, int E, int H, int I, int k) {
   FusedBufs b;
   b.wrt = reinterpret_cast<float *>(p); p += a((size_t)L * H * E * 4);
   b.lacc = reinterpret_cast<unsigned long long *>(p); p += a(2 * (size_t)E * 8);
-  b.ssq = reinterpret_cast<double *>(p); p += a(2 * (size_t)(H / 16) * 8);
-  b.zbuf = reinterpret_cast<float *>(p); p += a(2 * (size_t)H * 4);
+  b.ssq = reinterpret_cast<double *>(p); p += a(Z_COPIES * 2 * (size_t)(H / 16) * 8);
+  b.zbuf = reinterpret_cast<float *>(p); p += a(Z_COPIES * 2 * (size_t)H * 4);
   const size_t nb = (size_t)k * (I / 32);
   b.lbuf = reinterpret_cast<uint8_t *>(p); p += a(nb * LIMB_REC);
   b.lscg = reinterpret_cast<float2 *>(p); p += a(nb * 8);

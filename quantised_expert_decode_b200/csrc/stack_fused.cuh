@@ -20,8 +20,8 @@ struct FusedPlan {
 struct FusedBufs {
   float *wrt;                      // [L][H][E] transposed routers
   unsigned long long *lacc;         // [2][E] integer partial-logit sums (2^-32 units)
-  double *ssq;                     // [2][H/16] slice sums of squares
-  float *zbuf;
+  double *ssq;                     // [copies][2][H/16] slice sums of squares
+  float *zbuf;                     // [copies][2][H] residual stream z
   uint8_t *lbuf;                   // limbs of h, [k][I/32][96]
   float2 *lscg;                    // block scales of h, [k][I/32]
   unsigned *bar;
