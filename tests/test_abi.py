@@ -168,6 +168,16 @@ def test_stack_descriptor_checks_without_gpu():
     h[1] = ex_(64, 256, 128)
     out = ctypes.c_void_p()
     assert lib.qmoe_stack_create(ctypes.byref(d), FAKE, 16, None, ctypes.byref(out)) == 4
+    # layers of different block formats form one stack (mixed-bit)
+    uniform = lib.qmoe_stack_workspace_bytes(ctypes.byref(d))
+    h[1] = L.qmoe_experts(64, 256, 128, 4, FAKE, FAKE, q.qmoe_packed_bytes(4, 0, 64, 256, 128),
+                          q.qmoe_packed_bytes(4, 1, 64, 256, 128))
+    assert lib.qmoe_stack_workspace_bytes(ctypes.byref(d)) > 0
+    h[1].down_bytes = q.qmoe_packed_bytes(2, 1, 64, 256, 128)          # Q2 size under a Q4 handle
+    assert lib.qmoe_stack_workspace_bytes(ctypes.byref(d)) == 0
+    h[1] = L.qmoe_experts(64, 256, 128, 3, FAKE, FAKE, 0, 0)             # no such format
+    assert lib.qmoe_stack_workspace_bytes(ctypes.byref(d)) == 0
+    assert lib.qmoe_stack_create(ctypes.byref(d), FAKE, uniform, None, ctypes.byref(out)) == 3
 
 
 def test_status_strings():
