@@ -13,9 +13,10 @@ weights with its own roofline, clocks and CPU-oracle baseline:
   config4_prefill  a 4096-token bf16 chunk through one Q4 layer
   mixed48_decode   the 48-layer single-token stack with every fourth layer in Q4
                    (mixed-bit stack: the fused kernel takes each layer's format)
+  ngram_gather     16 hashed rows per token of a 2^22 x 256 Q4 n-gram table, 4096 tokens
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode48|verify48|mixed48|layer|prefill] [--headline-only]
+                    [--workload decode48|verify48|mixed48|layer|prefill|ngram] [--headline-only]
 
 N > 1 runs N independent replicas (one process per GPU under torchrun; the
 path has no exchange step), timed on the device, max over ranks.
@@ -39,7 +40,9 @@ METRIC = "MoE decode tokens/s over 48 layers; HBM GB/s on weight bytes vs peak"
 PREFILL_METRIC = "MoE prefill tokens/s (4096-token bf16 chunk, one 512-expert Q4 layer); tensor TFLOP/s vs peak"
 SEED = 0
 LAYER_CYCLE = 16      # distinct layers the single-layer steps cycle over (weights > L2)
-WORKLOADS = {"decode48": 2, "verify48": 3, "mixed48": 2, "layer": 1, "prefill": 4}
+WORKLOADS = {"decode48": 2, "verify48": 3, "mixed48": 2, "layer": 1, "prefill": 4, "ngram": None}
+NGRAM_METRIC = ("n-gram row gather tokens/s (16 hashed rows of a 2^22 x 256 Q4 table per token, 4096-token "
+                "chunk); HBM GB/s on row and output bytes vs peak")
 MIXED_EVERY = 4       # mixed48: layers 0, 4, 8, ... in Q4, the others in Q2
 
 
@@ -236,6 +239,7 @@ TRAFFIC_PROFILES = {
                      ("stack_decode.cu", "decode_tile.cuh", "common.cuh", "layout.cuh", "route_common.cuh",
                       "decode_canon.cuh")),
     "pf_gemm1": ("pf_gemm_prefill4096_ncu.md", ("prefill.cu", "tc05.cuh", "common.cuh", "layout.cuh")),
+    "ngram_gather": ("ngram_gather_ngram4096_ncu.md", ("ngram.cu", "common.cuh")),
     # per algorithmic byte (a launch's bytes depend on its routes): scaled to the measured launches
     "stack_decode_mixed": ("stack_decode_mixed48_ncu.md",
                            ("stack_decode.cu", "decode_tile.cuh", "common.cuh", "layout.cuh", "route_common.cuh",
@@ -902,9 +906,162 @@ def run_prefill(args, cfg):
     return line
 
 
+def ngram_oracle_time(nc, n_tok):
+    """Seconds the oracle takes to hash ``n_tok`` tokens and dequantise their
+    16 rows each (row bytes drawn from the generator beforehand, not timed)."""
+    import numpy as np
+    from oracle import ngram
+    from synth import gen
+    ids = gen.ngram_ids(SEED, nc, 0, T=n_tok)
+    rows = ngram.rows(SEED, ids, nc.R)
+    codes, scales = gen.ngram_rows(SEED, nc, 0, rows.ravel())
+    t0 = time.perf_counter()
+    r2 = ngram.rows(SEED, ids, nc.R)
+    ngram.gather(codes, scales, np.arange(r2.size).reshape(r2.shape))
+    return time.perf_counter() - t0
+
+
+def run_ngram(args, nc):
+    """The n-gram row gather over a device-resident table: one launch per
+    4096-token chunk, a fresh chunk of ids per step."""
+    import numpy as np
+    import torch
+
+    import quantised_expert_decode_b200 as q
+    from synth import device, gen
+
+    rank, world, local = dist_env()
+    T, D, R = nc.T, nc.D, nc.R
+    codes, scales = device.ngram_table(SEED, nc)
+    n_in = min(args.steps + args.warmup, 16)
+    ids_host = [gen.ngram_ids(SEED + 1000 * rank, nc, s) for s in range(n_in)]
+    ids = [torch.from_numpy(a).cuda() for a in ids_host]
+    out = torch.empty((T, 16, D), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+
+    def step(s, events=None):
+        if events:
+            events[0].record(stream)
+        q.qmoe_ngram_gather(ids[s % n_in], T, SEED, codes, scales, R, D, out, None, stream)
+        if events:
+            events[1].record(stream)
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+    clocks = clock_sampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = q.qmoe_launch_count()
+    e0.record(stream)
+    for s in range(args.steps):
+        step(args.warmup + s)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = q.qmoe_launch_count() - n0
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    clk = clocks.stop()
+    # per-launch durations for the roofline (events around each launch)
+    for s in range(args.steps):
+        step(args.warmup + s, ev[s])
+    torch.cuda.synchronize()
+    launch_us = 1e3 * statistics.mean(es[0].elapsed_time(es[1]) for es in ev)
+    # one decode token: 16 rows, a latency-bound launch
+    one = torch.empty((1, 16, D), dtype=torch.float32, device="cuda")
+    e6, e7 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e6.record(stream)
+    for s in range(args.steps):
+        q.qmoe_ngram_gather(ids[s % n_in][:1], 1, SEED, codes, scales, R, D, one, None, stream)
+    e7.record(stream)
+    torch.cuda.synchronize()
+    one_us = 1e3 * e6.elapsed_time(e7) / args.steps
+    # end to end: pinned ids -> device, gather, rows -> pinned host
+    idh = [torch.from_numpy(a).pin_memory() for a in ids_host]
+    outh = torch.empty((T, 16, D), dtype=torch.float32).pin_memory()
+    idd = torch.empty((T, 3), dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    barrier(world)
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for s in range(args.steps):
+        idd.copy_(idh[s % n_in], non_blocking=True)
+        q.qmoe_ngram_gather(idd, T, SEED, codes, scales, R, D, out, None, stream)
+        outh.copy_(out, non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(e2.elapsed_time(e3), world)
+
+    hbm, peak_kind = peaks()
+    launch_bytes = T * (12 + 16 * (nc.row_bytes() + 4 * D))
+    achieved = launch_bytes / (launch_us / 1e6) / 1e9
+    line = {
+        "metric": NGRAM_METRIC, "value": replica_throughput(world, args.steps, T, ms), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u8 Q4 codes + fp16 scales -> f32 (exact), u64 hash",
+        "data": "synthetic (seeded SplitMix64 table and token ids)",
+        "config": {"workload": f"n-gram row gather: {T} tokens x 16 rows of a {R}-row x {D} Q4 table "
+                               f"({R * nc.row_bytes() / 1e9:.2f} GB, one layer)",
+                   "tokens_per_step": T, "rows": R, "row_elems": D, "vocab": nc.vocab, "seed": SEED,
+                   "l2": f"no flush: the table ({R * nc.row_bytes() / 1e6:.0f} MB) is larger than L2 and each "
+                         "step draws fresh ids", "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "kernel": "ngram_gather_kernel", "achieved": achieved, "peak": hbm,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": stored_traffic("ngram_gather") if (T, D, R) == (4096, 256, 1 << 22) else None,
+                     "algorithmic_bytes_per_launch": launch_bytes, "avg_launch_us": launch_us,
+                     "timing": "CUDA events around each launch on the launching stream"},
+        "one_token_us": one_us,
+        "e2e": {"value": world * args.steps * T / (ms_e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * 12, "d2h_bytes_per_step": T * 16 * D * 4,
+                "path": "pinned int32 ids -> device, qmoe_ngram_gather, fp32 rows -> pinned host"},
+        "clocks": clk, "gpu_launches": launches,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_tok = T
+        t = ngram_oracle_time(nc, n_tok)
+        line["cpu_baseline"] = {"value": n_tok / t, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"hash and 16-row dequantisation of {n_tok} tokens ({t:.2f} s); "
+                                          "row bytes drawn beforehand"}
+    del codes, scales, out, ids
+    free_device()
+    return line
+
+
 def main():
     args = parse()
     from synth import configs
+    if args.workload == "ngram":
+        rank = dist_env()[0]
+        if args.impl == "reference":
+            if rank == 0:
+                nc = configs.NGRAM
+                for _ in range(args.warmup):
+                    ngram_oracle_time(nc, nc.T)
+                t = sum(ngram_oracle_time(nc, nc.T) for _ in range(args.steps))
+                v = args.steps * nc.T / t
+                print(json.dumps({"impl": "reference", "metric": NGRAM_METRIC, "value": v, "unit": "tokens/s",
+                                  "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                                  "ms_per_step": 1e3 * t / args.steps,
+                                  "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                                  "data": "synthetic", "config": {"workload": "n-gram row gather (oracle)"},
+                                  "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": blas_threads(),
+                                                   "kind": "oracle",
+                                                   "sample": f"one {nc.T}-token chunk: hash and 16-row dequantisation"},
+                                  "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                                          "d2h_bytes_per_step": 0}}), flush=True)
+            return
+        _, world, local = dist_env()
+        init_dist(local, world)
+        line = run_ngram(args, configs.NGRAM)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     cfg = configs.get(WORKLOADS[args.workload])
     if args.workload == "prefill" and args.tokens:
         cfg = cfg.with_(T=args.tokens)
@@ -940,9 +1097,12 @@ def main():
             line["config4_prefill"] = sub_line(run_prefill(args, configs.get(4)))
             mx = configs.mixed(cfg, MIXED_EVERY)
             line["mixed48_decode"] = sub_line(stack_line(args, mx, measure_stack(args, mx)))
+            line["ngram_gather"] = sub_line(run_ngram(args, configs.NGRAM), keep=(
+                "metric", "value", "unit", "ms_per_step", "config", "roofline", "cpu_baseline", "e2e", "clocks",
+                "gpu_launches", "one_token_us"))
             line["gpu_launches_all_workloads"] = (line["gpu_launches"] + sum(
                 line[k_]["gpu_launches"] for k_ in ("config1_layer", "config3_verify", "config4_prefill",
-                                                    "mixed48_decode")))
+                                                    "mixed48_decode", "ngram_gather")))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -346,6 +346,36 @@ qmoe_status qmoe_stack_decode(qmoe_stack *stack, qmoe_stream_t stream);
 qmoe_status qmoe_stack_decode_host(qmoe_stack *stack, const float *x_host, float *x_out_host,
                                    qmoe_stream_t stream);
 
+/* ------------------------------------------------------- n-gram row gather --
+ * [P3] "Understanding the Architecture": besides the expert packs the model
+ * keeps a large per-layer token-embedding table; a token's last three ids
+ * are hashed into 16 row indices and only those rows are read. The pages fix
+ * neither the hash nor the row format (a third-party 4-bit type), so both are
+ * self-defined here, with SplitMix64's finaliser (Steele, Lea & Flood,
+ * OOPSLA 2014) as the mixing function:
+ *   mix64(z): z ^= z >> 30; z *= 0xBF58476D1CE4E5B9; z ^= z >> 27;
+ *             z *= 0x94D049BB133111EB; z ^= z >> 31          (mod 2^64)
+ *   G = 0x9E3779B97F4A7C15
+ *   h = mix64(seed + G); then for each id of (a, b, c) in that order
+ *       h = mix64(h ^ u), u = the id's 32-bit pattern zero-extended
+ *   row i (i = 0..15) = floor(mix64(h + (i + 1) G) * R / 2^64)
+ * Row format: the Q4 block format of this library in canonical layout, codes
+ * uint8 [R][D/2] (code j of a row in byte j/2, low nibble for even j) and
+ * scales uint16 [R][D/32][2] (fp16 d, m per 32-element block); w = d q + m,
+ * exact in fp32.
+ *
+ * ngrams: device int32 [T][3], token t's ids (a, b, c) = (id_{t-2}, id_{t-1},
+ *         id_t); any values (the caller pads the first positions).
+ * out:    device fp32 [T][16][D]; out[t][i] = dequantised row i of token t.
+ * rows:   device int32 [T][16] (the row indices), or NULL.
+ * Limits: 1 <= R <= 2^31 - 1, D a multiple of 32 up to 8192, T >= 1.
+ * Alignment: codes, out 16 bytes; ngrams, scales, rows 4 bytes.
+ * Errors: INVALID_ARG (null or misaligned pointers, T < 1, R < 1),
+ * UNSUPPORTED (D outside the limits). Asynchronous on `stream`. */
+qmoe_status qmoe_ngram_gather(const int32_t *ngrams, int T, uint64_t seed, const uint8_t *codes,
+                              const uint16_t *scales, int64_t R, int D, float *out, int32_t *rows,
+                              qmoe_stream_t stream);
+
 /* ------------------------------------------------------------------- misc -- */
 /* Synchronous: copies *dev_status to the host and maps it to a status. */
 qmoe_status qmoe_read_status(const int32_t *dev_status);

@@ -7,7 +7,8 @@ without the built library every entry point raises.
 """
 from ._lib import (BF16, DOWN, F32, GATE_UP, Q2, Q4, QmoeError, exported_symbols, lib,  # noqa: F401
                    qmoe_bucket, qmoe_bucket_workspace_bytes, qmoe_ffn_prefill, qmoe_ffn_prefill_timed, qmoe_prefill_workspace_bytes,
-                   qmoe_decode_workspace_bytes, qmoe_experts, qmoe_ffn_decode, qmoe_launch_count, qmoe_pack,
+                   qmoe_decode_workspace_bytes, qmoe_experts, qmoe_ffn_decode, qmoe_launch_count, qmoe_ngram_gather,
+                   qmoe_pack,
                    qmoe_packed_bytes, qmoe_read_status, qmoe_residual_route, qmoe_rmsnorm_residual, qmoe_route,
                    qmoe_route_fixed, qmoe_route_workspace_bytes, qmoe_stack_buffers, qmoe_stack_create, qmoe_stack_decode,
                    qmoe_stack_decode_host, qmoe_stack_desc, qmoe_stack_destroy, qmoe_stack_kernels_per_replay, qmoe_stack_layer_times,

@@ -72,6 +72,7 @@ _SIGS = {
     "qmoe_stack_decode": (_I, [_VP, _VP]),
     "qmoe_stack_layer_times": (_I, [_VP, _VP, _VP]),
     "qmoe_stack_decode_host": (_I, [_VP, _VP, _VP, _VP]),
+    "qmoe_ngram_gather": (_I, [_VP, _I, ctypes.c_uint64, _VP, _VP, ctypes.c_int64, _I, _VP, _VP, _VP]),
     "qmoe_read_status": (_I, [_VP]),
     "qmoe_status_string": (ctypes.c_char_p, [_I]),
     "qmoe_launch_count": (ctypes.c_uint64, []),
@@ -189,6 +190,13 @@ def qmoe_ffn_prefill(experts: qmoe_experts, x, T, idx, gate, k, y, workspace, de
     _check("qmoe_ffn_prefill", lib().qmoe_ffn_prefill(
         ctypes.byref(experts), _p(x), T, _p(idx), _p(gate), k, _p(y), _p(workspace),
         workspace.numel() * workspace.element_size(), _p(dev_status), _s(stream)))
+
+
+def qmoe_ngram_gather(ngrams, T, seed, codes, scales, R, D, out, rows=None, stream=None) -> None:
+    """``ngrams`` int32 [T, 3]; ``codes`` uint8 [R, D/2]; ``scales`` int16/uint16 [R, D/32, 2];
+    ``out`` fp32 [T, 16, D]; ``rows`` int32 [T, 16] or None."""
+    _check("qmoe_ngram_gather", lib().qmoe_ngram_gather(_p(ngrams), T, seed & ((1 << 64) - 1), _p(codes), _p(scales),
+                                                        R, D, _p(out), _p(rows), _s(stream)))
 
 
 PREFILL_ATOMIC_COMBINE = 1

@@ -26,6 +26,9 @@ WHAT_ROUTER = 7
 WHAT_BIAS = 8
 WHAT_X = 9
 WHAT_NOISE = 10
+WHAT_NGRAM_CODES = 11
+WHAT_NGRAM_SCALES = 12
+WHAT_NGRAM_IDS = 13
 
 
 @dataclass(frozen=True)
@@ -113,6 +116,35 @@ CONFIGS = {
 
 def get(cid: int) -> Config:
     return CONFIGS[cid]
+
+
+@dataclass(frozen=True)
+class NgramConfig:
+    """An n-gram row table of one layer and a chunk of tokens that read it.
+
+    The pages size the whole table at 51.2 billion elements (about 28.8 GB)
+    for 48 layers (pyshine Strata tour, "Understanding the Architecture"),
+    about a billion elements a layer; 2^22 rows of 256 give 2^30.  Rows use
+    the Q4 block format; ids are uniform over a 2^17-token vocabulary."""
+    cid: int = 5
+    R: int = 1 << 22
+    D: int = 256
+    T: int = 4096
+    vocab: int = 1 << 17
+    fmt: int = Q4
+
+    @property
+    def format(self) -> Fmt:
+        return FORMATS[self.fmt]
+
+    def row_bytes(self) -> int:
+        return self.D // BLOCK * self.format.bytes_per_block
+
+    def with_(self, **kw) -> "NgramConfig":
+        return replace(self, **kw)
+
+
+NGRAM = NgramConfig()
 
 
 def mixed(cfg: Config, every: int = 4) -> Config:

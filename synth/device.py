@@ -81,3 +81,24 @@ def fill_layer(seed: int, cfg: Config, layer: int, bufs: dict, e0: int = 0) -> d
         fill_codes(seed, cfg, layer, mat, bufs[name + "_codes"], e0)
         fill_scales(seed, cfg, layer, mat, bufs[name + "_scales"], e0)
     return bufs
+
+
+def ngram_table(seed: int, ncfg, layer: int = 0, device="cuda", R: int | None = None) -> tuple:
+    """Device codes uint8 [R, D/2] and scales int16 [R, D/32, 2] of an n-gram
+    row table (same bytes as ``gen.ngram_rows``)."""
+    import torch
+    from .configs import WHAT_NGRAM_CODES, WHAT_NGRAM_SCALES
+    R = ncfg.R if R is None else R
+    D, f = ncfg.D, ncfg.format
+    codes = torch.empty((R, D * f.bits // 8), dtype=torch.uint8, device=device)
+    scales = torch.empty((R, D // BLOCK, 2), dtype=torch.int16, device=device)
+    rc = lib().synth_fill_codes(seed & rng.MASK64, ncfg.cid, layer, 0, R, WHAT_NGRAM_CODES, codes[0].numel(),
+                                codes.data_ptr(), _stream())
+    if rc:
+        raise RuntimeError(f"synth_fill_codes failed ({rc})")
+    rc = lib().synth_fill_scales(seed & rng.MASK64, ncfg.cid, layer, 0, R, WHAT_NGRAM_SCALES, D // BLOCK,
+                                 float(np.float64(f.d_lo)), float(f.d_hi - f.d_lo), float(f.m_coef),
+                                 scales.data_ptr(), _stream())
+    if rc:
+        raise RuntimeError(f"synth_fill_scales failed ({rc})")
+    return codes, scales

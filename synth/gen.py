@@ -25,8 +25,9 @@ from __future__ import annotations
 import numpy as np
 
 from . import rng
-from .configs import (BLOCK, DOWN, GATE, UP, WHAT_BIAS, WHAT_CODES, WHAT_NOISE,
-                      WHAT_ROUTER, WHAT_SCALES, WHAT_X, Config, FORMATS)
+from .configs import (BLOCK, DOWN, GATE, UP, WHAT_BIAS, WHAT_CODES, WHAT_NGRAM_CODES, WHAT_NGRAM_IDS,
+                      WHAT_NGRAM_SCALES, WHAT_NOISE, WHAT_ROUTER, WHAT_SCALES, WHAT_X, Config, FORMATS,
+                      NgramConfig)
 
 
 def matrix_shape(cfg: Config, mat: int) -> tuple[int, int]:
@@ -142,3 +143,28 @@ def tokens(seed: int, cfg: Config, step: int = 0, T: int | None = None):
     if cfg.x_kind == "bf16":
         return f32_to_bf16_bits(z.astype(np.float32))
     raise ValueError(cfg.x_kind)
+
+
+# ------------------------------------------------------- n-gram row tables --
+def ngram_rows(seed: int, ncfg: NgramConfig, layer: int, rows) -> tuple[np.ndarray, np.ndarray]:
+    """Canonical codes uint8 [n, D/2] and scales uint16 [n, D/32, 2] of table
+    rows ``rows`` (row r is the stream pair keyed like expert r of an expert
+    layer; the device fill draws the same bytes)."""
+    rows = np.asarray(rows, dtype=np.int64).reshape(-1)
+    D = ncfg.D
+    codes = np.empty((len(rows), D * ncfg.format.bits // 8), dtype=np.uint8)
+    scales = np.empty((len(rows), D // BLOCK, 2), dtype=np.uint16)
+    for n, r in enumerate(rows):
+        codes[n] = code_bytes(rng.stream_key(seed, ncfg.cid, layer, int(r), WHAT_NGRAM_CODES), codes.shape[1])
+        scales[n] = scale_pairs(rng.stream_key(seed, ncfg.cid, layer, int(r), WHAT_NGRAM_SCALES), D // BLOCK,
+                                ncfg.fmt).reshape(D // BLOCK, 2)
+    return codes, scales
+
+
+def ngram_ids(seed: int, ncfg: NgramConfig, step: int = 0, T: int | None = None) -> np.ndarray:
+    """int32 [T, 3]: token t's ids (t-2, t-1, t) of a chunk of T + 2 ids drawn
+    uniformly from the vocabulary (64-bit draws reduced by multiply-high)."""
+    T = ncfg.T if T is None else T
+    words = rng.outputs(rng.stream_key(seed, ncfg.cid, step, 0, WHAT_NGRAM_IDS), 0, T + 2)
+    ids = np.array([(int(w) * ncfg.vocab) >> 64 for w in words], dtype=np.int32)
+    return np.stack([ids[:-2], ids[1:-1], ids[2:]], axis=1)

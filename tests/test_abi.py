@@ -180,6 +180,18 @@ def test_stack_descriptor_checks_without_gpu():
     assert lib.qmoe_stack_create(ctypes.byref(d), FAKE, uniform, None, ctypes.byref(out)) == 3
 
 
+def test_ngram_gather_argument_checks_without_gpu():
+    lib = q.lib()
+    def call(ng=FAKE, T=2, codes=FAKE, scales=FAKE, R=4, D=32, out=FAKE, rows=None):
+        return lib.qmoe_ngram_gather(ng, T, 0, codes, scales, R, D, out, rows, None)
+    assert call(D=48) == 3 and call(D=0) == 3 and call(D=8192 + 32) == 3     # D outside the limits
+    assert call(R=0) == 1 and call(R=2**31) == 1                              # table size
+    assert call(T=0) == 1                                                     # no tokens
+    assert call(codes=FAKE + 4) == 1 and call(out=FAKE + 8) == 1              # 16-byte alignment
+    assert call(ng=FAKE + 2) == 1 and call(rows=FAKE + 1) == 1                # 4-byte alignment
+    assert call(ng=None) == 1 and call(scales=None) == 1 and call(out=None) == 1
+
+
 def test_status_strings():
     assert q.qmoe_status_string(0) == "ok"
     assert "geometry" in q.qmoe_status_string(2)
