@@ -73,3 +73,24 @@ def test_replica_throughput_sums_work_over_the_slowest_rank():
     # 4 replicas, 10 steps of 1 token each, slowest rank 20 ms: 40 tokens / 0.02 s
     assert bench.replica_throughput(4, 10, 1, 20.0) == pytest.approx(2000.0)
     assert bench.max_over_ranks(3.5, 1) == 3.5
+
+
+def test_workload_descriptions_name_the_block_formats():
+    from synth import configs
+    cfg = configs.get(2)
+    assert bench.format_desc(cfg) == "Q2"
+    mx = configs.mixed(cfg, bench.MIXED_EVERY)
+    assert len(mx.fmt_layers) == 48 and mx.fmt_layers[:5] == (4, 2, 2, 2, 4)
+    assert bench.format_desc(mx).startswith("mixed: Q4 in 12 of 48 layers")
+    # a mixed stack's bytes per layer follow each layer's own format
+    per_layer = [mx.for_layer(l).expert_bytes() for l in range(48)]
+    assert per_layer.count(2_949_120) == 12 and per_layer.count(1_769_472) == 36
+
+
+def test_ngram_workload_bytes():
+    """4096 tokens x 16 rows: 160-byte Q4 rows of 256 read, 1 KB of fp32 written
+    per row, 12 bytes of ids per token."""
+    from synth import configs
+    nc = configs.NGRAM
+    assert nc.row_bytes() == 160 and nc.R * nc.row_bytes() == 671_088_640
+    assert nc.T * (12 + 16 * (nc.row_bytes() + 4 * nc.D)) == 77_643_776
