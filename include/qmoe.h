@@ -370,8 +370,9 @@ qmoe_status qmoe_stack_decode_host(qmoe_stack *stack, const float *x_host, float
  * rows:   device int32 [T][16] (the row indices), or NULL.
  * Limits: 1 <= R <= 2^31 - 1, D a multiple of 32 up to 8192, T >= 1.
  * Alignment: codes, out 16 bytes; ngrams, scales, rows 4 bytes.
- * Errors: INVALID_ARG (null or misaligned pointers, T < 1, R < 1),
- * UNSUPPORTED (D outside the limits). Asynchronous on `stream`. */
+ * Errors: INVALID_ARG (null or misaligned pointers, T < 1, R outside
+ * [1, 2^31 - 1]), UNSUPPORTED (D outside the limits). Asynchronous on
+ * `stream`. */
 qmoe_status qmoe_ngram_gather(const int32_t *ngrams, int T, uint64_t seed, const uint8_t *codes,
                               const uint16_t *scales, int64_t R, int D, float *out, int32_t *rows,
                               qmoe_stream_t stream);
