@@ -121,3 +121,21 @@ def test_mixed_bit_stack_layers_are_the_uniform_layers():
     w = W.Layer(0, mixed, 1).expert(3)[0]
     blk = w[0, :32]
     assert len(np.unique(blk)) > 4
+
+
+def test_ngram_inputs():
+    """A chunk's triples are the sliding windows of one id sequence drawn over
+    the vocabulary; table rows are streams keyed by their row index."""
+    nc = configs.NGRAM.with_(T=500)
+    ids = gen.ngram_ids(0, nc, 0)
+    assert ids.shape == (500, 3) and ids.dtype == np.int32
+    assert np.array_equal(ids[1:, 0], ids[:-1, 1]) and np.array_equal(ids[1:, 1], ids[:-1, 2])
+    assert ids.min() >= 0 and ids.max() < nc.vocab
+    assert not np.array_equal(ids, gen.ngram_ids(0, nc, 1))                 # steps differ
+    codes, scales = gen.ngram_rows(0, nc, 0, [7, 7, 8])
+    assert codes.shape == (3, nc.D // 2) and scales.shape == (3, nc.D // 32, 2)
+    assert np.array_equal(codes[0], codes[1]) and not np.array_equal(codes[0], codes[2])
+    d = scales[:, :, 0].view(np.float16).astype(np.float64)
+    m = scales[:, :, 1].view(np.float16).astype(np.float64)
+    assert np.all((d >= 0.002 * (1 - 2**-10)) & (d <= 0.01 * (1 + 2**-10)))
+    assert np.array_equal(m, (-7.5 * d).astype(np.float16).astype(np.float64))
